@@ -1,0 +1,250 @@
+"""Seeded synthetic inputs for paged decode attention.
+
+This module only draws random numbers and lays them out as plain arrays.  It
+holds none of the method's arithmetic (no slot formula, no attention math), so
+both the CPU oracle (through the tests) and the CUDA path (through the tests and
+the benchmark) can consume the same inputs without sharing any computation.
+
+Floating-point tensors are returned as ``numpy.uint16`` arrays holding fp16 or
+bf16 bit patterns; ``dtype`` says which.  Values are drawn in fp32 and rounded
+to the storage type with round-to-nearest-even (numpy for fp16, torch for bf16).
+
+Workloads follow the five decode batches used throughout the project:
+
+* ``tiny``     4 seqs, 8/8 heads, D=64, B=16, fp16, 64-frame pool, L ~ U{1..100}
+* ``mha13b``   32 seqs, 40/40 heads, D=128, B=16, fp16, 4096 frames, L ~ U{1..2048}
+               (13B-shaped: 40 heads x 128 = the 5120 hidden size of the slides)
+* ``gqa8b``    256 seqs, 32/8 heads, D=128, B=16, bf16, 65536 frames,
+               L = clip(round(exp(N(ln 512, 1))), 16, 4096), K scaled by 0.5
+* ``shared``   16 prompts x 4 samples, 32/8 heads, D=128, B=16, bf16, prompt
+               1000 tokens, 0..200 private tokens per sample, 65536 frames
+* ``long``     4 seqs, 32/8 heads, D=128, B=32, bf16, 8192 frames,
+               L ~ U{16384..32768}
+
+Draw order inside one workload: context lengths, the physical frame order of
+the pool, q, K, V (for ``shared``: generated lengths, frame order, q, prompt K,
+prompt V, generated K, generated V).  The default seed of a workload is its
+position in the list above (0 for ``tiny`` ... 4 for ``long``).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+F16 = 0
+BF16 = 1
+DTYPE_NAMES = {F16: "f16", BF16: "bf16"}
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    seed: int
+    num_seqs: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    dtype: int
+    max_blocks_per_seq: int
+    scale: float
+    k_scale: float = 1.0
+    # length law: ("uniform", lo, hi) | ("lognormal", median, sigma, lo, hi) | ("shared", prompt, gmax)
+    lengths: tuple = ()
+    # shared-prefix workloads only
+    num_prompts: int = 0
+    samples_per_prompt: int = 0
+
+    @property
+    def group(self) -> int:
+        return self.num_heads // self.num_kv_heads
+
+    @property
+    def elt_bytes(self) -> int:
+        return 2
+
+    def with_block_size(self, block_size: int) -> "Workload":
+        """Same batch on a pool of the same token capacity with another block size."""
+        tokens = self.num_blocks * self.block_size
+        max_tokens = self.max_blocks_per_seq * self.block_size
+        return dataclasses.replace(
+            self,
+            name=f"{self.name}-B{block_size}",
+            block_size=block_size,
+            num_blocks=tokens // block_size,
+            max_blocks_per_seq=max_tokens // block_size,
+        )
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 0, 4, 8, 8, 64, 16, 64, F16, 7, 1.0 / 8.0,
+                     lengths=("uniform", 1, 100)),
+    "mha13b": Workload("mha13b", 1, 32, 40, 40, 128, 16, 4096, F16, 128, 1.0 / math.sqrt(128),
+                       lengths=("uniform", 1, 2048)),
+    "gqa8b": Workload("gqa8b", 2, 256, 32, 8, 128, 16, 65536, BF16, 256, 1.0 / math.sqrt(128),
+                      k_scale=0.5, lengths=("lognormal", 512, 1.0, 16, 4096)),
+    "shared": Workload("shared", 3, 64, 32, 8, 128, 16, 65536, BF16, 75, 1.0 / math.sqrt(128),
+                       lengths=("shared", 1000, 200), num_prompts=16, samples_per_prompt=4),
+    "long": Workload("long", 4, 4, 32, 8, 128, 32, 8192, BF16, 1024, 1.0 / math.sqrt(128),
+                     lengths=("uniform", 16384, 32768)),
+}
+
+
+def to_bits(x: np.ndarray, dtype: int) -> np.ndarray:
+    """Round fp32 values to fp16/bf16 (RNE) and return the bit patterns as uint16."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if dtype == F16:
+        return x.astype(np.float16).view(np.uint16)
+    if dtype == BF16:
+        import torch
+
+        return torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    raise ValueError(f"unknown dtype {dtype}")
+
+
+def _normal_bits(rng: np.random.Generator, shape, dtype: int, scale: float = 1.0,
+                 chunk: int = 1 << 24) -> np.ndarray:
+    """N(0, scale^2) values drawn in fp32 in chunks, stored as dtype bit patterns."""
+    n = int(np.prod(shape, dtype=np.int64))
+    out = np.empty(n, dtype=np.uint16)
+    for lo in range(0, n, chunk):
+        hi = min(n, lo + chunk)
+        x = rng.standard_normal(hi - lo, dtype=np.float32)
+        if scale != 1.0:
+            x *= np.float32(scale)
+        out[lo:hi] = to_bits(x, dtype)
+    return out.reshape(shape)
+
+
+def draw_lengths(w: Workload, rng: np.random.Generator) -> np.ndarray:
+    law = w.lengths
+    if law[0] == "uniform":
+        return rng.integers(law[1], law[2], size=w.num_seqs, endpoint=True).astype(np.int32)
+    if law[0] == "lognormal":
+        median, sigma, lo, hi = law[1:]
+        x = np.exp(rng.normal(math.log(median), sigma, size=w.num_seqs))
+        return np.clip(np.rint(x), lo, hi).astype(np.int32)
+    raise ValueError(law)
+
+
+@dataclasses.dataclass
+class DecodeInputs:
+    """One decode batch.
+
+    ``k_stream``/``v_stream`` hold every token's K/V in logical order, sequence
+    after sequence: sequence s owns rows ``offsets[s]:offsets[s+1]``, each row
+    ``[num_kv_heads, head_dim]``.  The last row of each sequence is the token the
+    decode step appends; the rows before it are the already-cached context.
+    ``frame_order`` is the order in which the pool hands out physical frames.
+    """
+    w: Workload
+    context_lens: np.ndarray  # int32 [S]
+    frame_order: np.ndarray   # int32 [N], a permutation of 0..N-1
+    q: np.ndarray             # uint16 [S, Hq, D]
+    k_stream: np.ndarray      # uint16 [sum L, Hkv, D]
+    v_stream: np.ndarray      # uint16 [sum L, Hkv, D]
+    offsets: np.ndarray       # int64 [S+1]
+
+    @property
+    def total_tokens(self) -> int:
+        return int(self.offsets[-1])
+
+
+def make_decode_inputs(name_or_w, seed: int | None = None, num_seqs: int | None = None,
+                       lengths: np.ndarray | None = None) -> DecodeInputs:
+    """Seeded decode batch for one of the workloads (not ``shared``).
+
+    ``num_seqs`` truncates the batch (the first sequences of the same draw of
+    lengths are kept, so a truncated batch is a prefix of the full one only in
+    its lengths); ``lengths`` overrides the drawn lengths (edge-case tests).
+    """
+    w = WORKLOADS[name_or_w] if isinstance(name_or_w, str) else name_or_w
+    if w.lengths and w.lengths[0] == "shared":
+        raise ValueError("use make_shared_inputs for the shared-prefix workload")
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    lens = draw_lengths(w, rng)
+    if lengths is not None:
+        lens = np.asarray(lengths, dtype=np.int32)
+    elif num_seqs is not None:
+        lens = lens[:num_seqs]
+    if num_seqs is not None or lengths is not None:
+        w = dataclasses.replace(w, num_seqs=int(lens.shape[0]))
+    frame_order = rng.permutation(w.num_blocks).astype(np.int32)
+    q = _normal_bits(rng, (w.num_seqs, w.num_heads, w.head_dim), w.dtype)
+    total = int(lens.astype(np.int64).sum())
+    k = _normal_bits(rng, (total, w.num_kv_heads, w.head_dim), w.dtype, w.k_scale)
+    v = _normal_bits(rng, (total, w.num_kv_heads, w.head_dim), w.dtype)
+    offsets = np.zeros(w.num_seqs + 1, dtype=np.int64)
+    np.cumsum(lens, out=offsets[1:])
+    return DecodeInputs(w, lens, frame_order, q, k, v, offsets)
+
+
+@dataclasses.dataclass
+class SharedInputs:
+    """Shared-prefix parallel sampling batch.
+
+    Prompt p is shared by samples ``p*n .. p*n+n-1`` (n = samples per prompt).
+    ``prompt_k[p]`` holds the prompt's K rows in logical order; sample i then
+    generates ``gen_lens[i]`` private tokens whose K rows are
+    ``gen_k[gen_offsets[i]:gen_offsets[i+1]]``.
+    """
+    w: Workload
+    prompt_len: int
+    gen_lens: np.ndarray      # int32 [S]
+    frame_order: np.ndarray   # int32 [N]
+    q: np.ndarray             # uint16 [S, Hq, D]
+    prompt_k: np.ndarray      # uint16 [P, prompt_len, Hkv, D]
+    prompt_v: np.ndarray
+    gen_k: np.ndarray         # uint16 [sum g, Hkv, D]
+    gen_v: np.ndarray
+    gen_offsets: np.ndarray   # int64 [S+1]
+
+
+def make_shared_inputs(seed: int | None = None, num_prompts: int | None = None) -> SharedInputs:
+    w = WORKLOADS["shared"]
+    if num_prompts is not None:
+        w = dataclasses.replace(w, num_prompts=num_prompts,
+                                num_seqs=num_prompts * w.samples_per_prompt)
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    prompt_len, gmax = w.lengths[1], w.lengths[2]
+    gen = rng.integers(0, gmax, size=w.num_seqs, endpoint=True).astype(np.int32)
+    frame_order = rng.permutation(w.num_blocks).astype(np.int32)
+    q = _normal_bits(rng, (w.num_seqs, w.num_heads, w.head_dim), w.dtype)
+    pk = _normal_bits(rng, (w.num_prompts, prompt_len, w.num_kv_heads, w.head_dim), w.dtype)
+    pv = _normal_bits(rng, (w.num_prompts, prompt_len, w.num_kv_heads, w.head_dim), w.dtype)
+    total = int(gen.astype(np.int64).sum())
+    gk = _normal_bits(rng, (total, w.num_kv_heads, w.head_dim), w.dtype)
+    gv = _normal_bits(rng, (total, w.num_kv_heads, w.head_dim), w.dtype)
+    offs = np.zeros(w.num_seqs + 1, dtype=np.int64)
+    np.cumsum(gen, out=offs[1:])
+    return SharedInputs(w, prompt_len, gen, frame_order, q, pk, pv, gk, gv, offs)
+
+
+def make_token_rows(rng_seed: int, num_tokens: int, num_kv_heads: int, head_dim: int,
+                    dtype: int):
+    """Random new-token K and V rows ``[T, Hkv, D]`` (cache-write tests)."""
+    rng = np.random.default_rng(rng_seed)
+    k = _normal_bits(rng, (num_tokens, num_kv_heads, head_dim), dtype)
+    v = _normal_bits(rng, (num_tokens, num_kv_heads, head_dim), dtype)
+    return k, v
+
+
+def random_slots(rng_seed: int, num_tokens: int, num_slots: int, num_skipped: int = 0) -> np.ndarray:
+    """``num_tokens`` distinct slot indices in ``[0, num_slots)``; ``num_skipped``
+    of them (at random positions) replaced by -1, the padding sentinel."""
+    rng = np.random.default_rng(rng_seed)
+    slots = rng.choice(num_slots, size=num_tokens, replace=False).astype(np.int64)
+    if num_skipped:
+        slots[rng.choice(num_tokens, size=num_skipped, replace=False)] = -1
+    return slots
+
+
+def random_pool(rng_seed: int, num_blocks: int, num_kv_heads: int, block_size: int,
+                head_dim: int, dtype: int):
+    """A K pool and a V pool ``[N, Hkv, B, D]`` filled with N(0,1) values."""
+    rng = np.random.default_rng(rng_seed)
+    shape = (num_blocks, num_kv_heads, block_size, head_dim)
+    return _normal_bits(rng, shape, dtype), _normal_bits(rng, shape, dtype)
