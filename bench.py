@@ -1,0 +1,532 @@
+#!/usr/bin/env python
+"""Paged decode attention benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one decode step of the whole hot path over a batch whose K/V are
+already in the paged cache: the cache write of each sequence's new token
+(reshape_and_cache) followed by paged decode attention over the full context
+(pass 1 + the partition merge).  The copy-on-write block copy has no pairs in
+this batch (nothing is shared), so it issues no work.
+
+Default workload: the Llama-3-8B-shaped GQA batch (256 sequences, 32 query /
+8 kv heads, head_dim 128, bf16, block 16, log-normal contexts with median 512
+clipped to [16, 4096], 65536-frame shuffled pool).  Inputs are seeded and
+synthetic (``workloads.py``).  Timing: W warm-up steps, then K steps timed with
+CUDA events on the launching stream, the L2 flushed (256 MiB write) before each
+timed step, barrier + synchronize around the timed loop, max over ranks.
+
+Under torchrun every rank runs its own batch (seed + rank): the sequences of
+the job are sharded across GPUs with no collective in the data path (weak
+scaling); ``value`` is the bytes all ranks processed over the slowest rank's
+time.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "paged decode attn: HBM GB/s (% of B200 peak) and seqs/s; paged vs contiguous"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gqa8b", choices=["tiny", "mha13b", "gqa8b", "long"])
+    ap.add_argument("--block-size", type=int, default=0, help="override the workload's block size")
+    ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--no-contiguous", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU baseline sample budget")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def aggregate(ms_total: float, bytes_total: float, seqs_total: float, device=None):
+    """Max of the timed milliseconds and sums of the work over all ranks."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return ms_total, bytes_total, seqs_total
+    t = torch.tensor([ms_total], dtype=torch.float64, device=device)
+    w = torch.tensor([bytes_total, seqs_total], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    torch.distributed.all_reduce(w, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item()), float(w[0].item()), float(w[1].item())
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic():
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
+    with the kernel revision they were taken on; null when absent."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.25)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.remove(self.path)
+        except Exception:
+            return None
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+
+        sm = [num(r[1]) for r in rows]
+        smax = max(num(r[2]) for r in rows)
+        loaded = [c for c in sm if c > 0.5 * smax] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(num(r[3]) for r in rows)}
+
+
+# ------------------------------------------------------------------ workload
+def workload(args):
+    w = wl.WORKLOADS[args.workload]
+    if args.block_size and args.block_size != w.block_size:
+        w = w.with_block_size(args.block_size)
+    return w
+
+
+def algorithmic_bytes(w: wl.Workload, lens: np.ndarray) -> dict:
+    """Bytes the step must move: K and V of every context token (read), q (read)
+    and out (written); the cache write reads and writes one K and one V row per
+    sequence and reads its slot.  Block tables and context lengths are listed
+    apart (< 0.1 %)."""
+    elt = w.elt_bytes
+    S, Hq, Hkv, D = len(lens), w.num_heads, w.num_kv_heads, w.head_dim
+    kv = int(lens.astype(np.int64).sum()) * Hkv * D * 2 * elt
+    qo = 2 * S * Hq * D * elt
+    write = 2 * S * Hkv * D * elt * 2 + 8 * S
+    tables = 4 * int(np.sum((lens.astype(np.int64) + w.block_size - 1) // w.block_size)) + 4 * S
+    return {"decode": kv + qo, "cache_write": write, "step": kv + qo + write, "tables": tables}
+
+
+def build_gpu_batch(inp: wl.DecodeInputs, device):
+    """Pool, prefill write of every sequence's cached context and the decode step's
+    slots, all through the library (allocator + cache-write kernel)."""
+    from paged_kv_cache_419_b200.binding import BlockAllocator, reshape_and_cache
+
+    w = inp.w
+    S = w.num_seqs
+    td = torch.float16 if w.dtype == wl.F16 else torch.bfloat16
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(td).to(device)
+
+    alloc = BlockAllocator(w.num_blocks, w.block_size, inp.frame_order)
+    pre = [alloc.add_seq(s, int(inp.context_lens[s]) - 1) for s in range(S)]
+    new_slots, pairs = alloc.append_batch(np.arange(S, dtype=np.int32))
+    table, lens = alloc.block_table(np.arange(S, dtype=np.int32), w.max_blocks_per_seq)
+    shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+    k_cache = torch.zeros(shape, dtype=td, device=device)
+    v_cache = torch.zeros(shape, dtype=td, device=device)
+    last = inp.offsets[1:] - 1
+    keep = np.ones(inp.total_tokens, dtype=bool)
+    keep[last] = False
+    pre_slots = np.concatenate(pre)
+    rows = np.nonzero(keep)[0]
+    chunk = 1 << 16
+    for lo in range(0, pre_slots.size, chunk):
+        idx = rows[lo:lo + chunk]
+        reshape_and_cache(dev(inp.k_stream[idx]), dev(inp.v_stream[idx]), k_cache, v_cache,
+                          torch.from_numpy(pre_slots[lo:lo + chunk]).to(device))
+    return {
+        "q": dev(inp.q), "k_cache": k_cache, "v_cache": v_cache,
+        "tables": torch.from_numpy(table).to(device), "lens": torch.from_numpy(lens).to(device),
+        "new_k": dev(inp.k_stream[last]), "new_v": dev(inp.v_stream[last]),
+        "slots": torch.from_numpy(new_slots.astype(np.int64)).to(device),
+        "pairs": torch.from_numpy(pairs.astype(np.int64)).to(device),
+        "out": torch.empty(S, w.num_heads, w.head_dim, dtype=td, device=device),
+        "table_host": table, "lens_host": lens, "slots_host": new_slots,
+    }
+
+
+def build_contiguous(inp: wl.DecodeInputs, device):
+    w = inp.w
+    td = torch.float16 if w.dtype == wl.F16 else torch.bfloat16
+    max_ctx = w.max_blocks_per_seq * w.block_size
+    k = torch.zeros(w.num_seqs, w.num_kv_heads, max_ctx, w.head_dim, dtype=td, device=device)
+    v = torch.zeros_like(k)
+    ks = torch.from_numpy(inp.k_stream.view(np.int16)).view(td).to(device)
+    vs = torch.from_numpy(inp.v_stream.view(np.int16)).view(td).to(device)
+    for s in range(w.num_seqs):
+        a, e = int(inp.offsets[s]), int(inp.offsets[s + 1])
+        k[s, :, : e - a] = ks[a:e].transpose(0, 1)
+        v[s, :, : e - a] = vs[a:e].transpose(0, 1)
+    del ks, vs
+    return k, v
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, world, rank, local):
+    from paged_kv_cache_419_b200 import binding as pkv
+
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    device = torch.device("cuda", local)
+    w = workload(args)
+    inp = wl.make_decode_inputs(w, seed=w.seed + rank)
+    b = build_gpu_batch(inp, device)
+    nbytes = algorithmic_bytes(w, inp.context_lens)
+    part = args.partition
+    ws_bytes = pkv.decode_workspace_bytes(w.num_seqs, w.num_heads, w.head_dim,
+                                          w.max_blocks_per_seq * w.block_size, part)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    n_pairs = int(b["pairs"].shape[0])
+    max_parts = math.ceil(w.max_blocks_per_seq * w.block_size / part)
+    launches_per_step = 1 + 1 + (1 if max_parts > 1 else 0) + (1 if n_pairs else 0)
+
+    def step():
+        if n_pairs:
+            pkv.copy_blocks(b["k_cache"], b["v_cache"], b["pairs"])
+        pkv.reshape_and_cache(b["new_k"], b["new_v"], b["k_cache"], b["v_cache"], b["slots"])
+        pkv.paged_attention_decode(b["out"], b["q"], b["k_cache"], b["v_cache"], b["tables"], b["lens"],
+                                   w.scale, partition_size=part, workspace=ws)
+
+    for _ in range(max(args.warmup, 0)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if pkv.device_error():
+        raise RuntimeError("device error flags set during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(K):
+        flush.zero_()
+        e0, e1, e2 = ev[k]
+        e0.record()
+        if n_pairs:
+            pkv.copy_blocks(b["k_cache"], b["v_cache"], b["pairs"])
+        pkv.reshape_and_cache(b["new_k"], b["new_v"], b["k_cache"], b["v_cache"], b["slots"])
+        e1.record()
+        pkv.paged_attention_decode(b["out"], b["q"], b["k_cache"], b["v_cache"], b["tables"], b["lens"],
+                                   w.scale, partition_size=part, workspace=ws)
+        e2.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    step_ms = [ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]
+    decode_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    if pkv.device_error():
+        raise RuntimeError("device error flags set during the timed steps")
+
+    total_ms, total_bytes, total_seqs = aggregate(sum(step_ms), nbytes["step"] * K,
+                                                  w.num_seqs * K, device)
+    ms_per_step = total_ms / K
+    value = total_bytes / K / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    dec_ms = statistics.mean(decode_ms)
+    achieved = nbytes["decode"] / (dec_ms * 1e-3) / 1e9
+    traffic = profile_traffic()
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.DTYPE_NAMES[w.dtype], "data": "synthetic (seeded; workloads.py)",
+        "config": {
+            "workload": f"{w.name}: Llama-3-8B-shaped GQA decode step" if w.name == "gqa8b" else w.name,
+            "num_seqs_per_gpu": w.num_seqs, "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
+            "context_tokens_per_gpu": int(inp.context_lens.sum()), "partition_size": part,
+            "l2": "flushed before every timed step (256 MiB write); K/V read per step > L2",
+            "parallelism": f"dp{world} (sequences sharded, no collective)",
+        },
+        "seqs_per_s": round(total_seqs / (total_ms * 1e-3), 1),
+        "pct_of_nominal_8tbs": round(100 * value / NOMINAL_HBM_GBS, 2),
+        "bytes_per_step": nbytes,
+        "gpu_launches": launches_per_step * K,
+        "roofline": {
+            "bound": "hbm", "kernel": "paged_attention_decode (pass 1 + partition merge)",
+            "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": (traffic or {}).get("bytes_per_launch") if traffic else None,
+            "decode_ms": round(dec_ms, 5),
+        },
+        "clocks": clocks,
+    }
+
+    if not args.no_contiguous:
+        result["contiguous"] = contiguous_compare(args, inp, b, ws, flush, part, device)
+    if not args.no_e2e:
+        result["e2e"] = e2e_run(args, inp, b, ws, part, nbytes, device)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(inp, nbytes, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def contiguous_compare(args, inp, b, ws, flush, part, device):
+    """Paged vs contiguous decode, kernel level, same values and launch shape."""
+    from paged_kv_cache_419_b200 import binding as pkv
+
+    w = inp.w
+    k, v = build_contiguous(inp, device)
+    out_c = torch.empty_like(b["out"])
+    K = max(args.steps, 5)
+
+    def time_it(fn):
+        for _ in range(3):
+            flush.zero_()
+            fn()
+        evs = []
+        for _ in range(K):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(c) for a, c in evs)
+
+    t_paged = time_it(lambda: pkv.paged_attention_decode(
+        b["out"], b["q"], b["k_cache"], b["v_cache"], b["tables"], b["lens"], w.scale,
+        partition_size=part, workspace=ws))
+    t_contig = time_it(lambda: pkv.contiguous_attention_decode(
+        out_c, b["q"], k, v, b["lens"], w.scale, partition_size=part, workspace=ws))
+    same = bool(torch.equal(out_c, b["out"]))
+    del k, v
+    torch.cuda.empty_cache()
+    nb = algorithmic_bytes(w, inp.context_lens)["decode"]
+    return {"paged_ms": round(t_paged, 5), "contiguous_ms": round(t_contig, 5),
+            "paged_gbs": round(nb / (t_paged * 1e-3) / 1e9, 1),
+            "contiguous_gbs": round(nb / (t_contig * 1e-3) / 1e9, 1),
+            "overhead": round(t_paged / t_contig - 1.0, 4), "outputs_identical": same}
+
+
+def e2e_run(args, inp, b, ws, part, nbytes, device):
+    """The same step through the public API from pinned host buffers: host->device
+    copies of the step's inputs (q, the new token's K/V, its slots, the block tables
+    and context lengths) and the device->host read of the output are timed."""
+    from paged_kv_cache_419_b200 import binding as pkv
+
+    w = inp.w
+    host = {name: b[name].cpu().pin_memory() for name in ("q", "new_k", "new_v", "slots", "tables", "lens")}
+    out_h = torch.empty(b["out"].shape, dtype=b["out"].dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    dev = {name: torch.empty_like(b[name]) for name in host}
+
+    def step():
+        for name, t in host.items():
+            dev[name].copy_(t, non_blocking=True)
+        pkv.reshape_and_cache(dev["new_k"], dev["new_v"], b["k_cache"], b["v_cache"], dev["slots"])
+        pkv.paged_attention_decode(b["out"], dev["q"], b["k_cache"], b["v_cache"], dev["tables"],
+                                   dev["lens"], w.scale, partition_size=part, workspace=ws)
+        out_h.copy_(b["out"], non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = []
+    for _ in range(K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(c) for a, c in evs)
+    ms_max, _, _ = aggregate(ms, 0.0, 0.0, device)
+    return {"value": round(nbytes["step"] / (ms_max * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "ms_per_step": round(ms_max, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_pool(inp: wl.DecodeInputs):
+    """The batch's cache built on the host with the oracle's own allocator model
+    and scatter (the oracle's inputs never come from the CUDA path)."""
+    import oracle
+    from oracle.allocator_model import AllocatorModel
+
+    w = inp.w
+    m = AllocatorModel(w.num_blocks, w.block_size, inp.frame_order)
+    slots = []
+    for s in range(w.num_seqs):
+        slots += m.add_seq(s, int(inp.context_lens[s]))
+    shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+    kc = np.zeros(shape, np.uint16)
+    vc = np.zeros(shape, np.uint16)
+    oracle.reshape_and_cache(kc, vc, inp.k_stream, inp.v_stream, np.array(slots, np.int64), w.block_size)
+    tables, lens = m.block_table(range(w.num_seqs), w.max_blocks_per_seq)
+    return kc, vc, np.array(tables, np.int32), np.array(lens, np.int32)
+
+
+def cpu_baseline(inp, nbytes, seconds):
+    """The oracle (plain C, fp64, one thread) on this host over the same batch,
+    repeated until `seconds` have passed; GB/s with the same byte count."""
+    import oracle
+
+    w = inp.w
+    kc, vc, tables, lens = oracle_pool(inp)
+    runs, t0 = 0, time.perf_counter()
+    while True:
+        oracle.paged_decode(inp.q, kc, vc, tables, lens, w.scale, w.num_kv_heads, w.block_size, w.dtype)
+        runs += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    per = el / runs
+    return {"value": round(nbytes["decode"] / per / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "seqs_per_s": round(w.num_seqs / per, 2),
+            "sample": f"the whole {w.num_seqs}-sequence batch (decode attention only), {runs} run(s), "
+                      f"{el:.1f} s; host {os.cpu_count()} logical cores, oracle single-threaded"}
+
+
+def run_reference(args, world, rank, local):
+    """The CPU oracle as the reference arm: each step decodes a bounded sample of
+    the batch (its first 32 sequences) on one host core."""
+    if rank != 0:
+        return
+    import oracle
+
+    w = workload(args)
+    inp = wl.make_decode_inputs(w)
+    kc, vc, tables, lens = oracle_pool(inp)
+    n = min(32, w.num_seqs)
+    sample_bytes = algorithmic_bytes(w, inp.context_lens[:n])["decode"]
+
+    def one():
+        oracle.paged_decode(inp.q, kc, vc, tables, lens, w.scale, w.num_kv_heads, w.block_size, w.dtype,
+                            seqs=(0, n))
+
+    for _ in range(max(args.warmup, 0)):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = time.perf_counter() - t0
+    ms = el / args.steps * 1e3
+    value = sample_bytes / (ms * 1e-3) / 1e9
+    res = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded; workloads.py)",
+        "config": {"workload": f"{w.name}: Llama-3-8B-shaped GQA decode step" if w.name == "gqa8b" else w.name,
+                   "num_seqs_per_gpu": w.num_seqs, "sample_seqs": n},
+        "seqs_per_s": round(n / (ms * 1e-3), 2),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {n} of {w.num_seqs} sequences per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank, local)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

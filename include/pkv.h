@@ -1,0 +1,237 @@
+/*
+ * pkv.h - C ABI of the B200 paged KV-cache decode library (libpkv.so).
+ *
+ * The method: vLLM and PagedAttention (slides "vLLM and PagedAttention: Virtual
+ * Memory for LLM Serving", polomodov.tech; note "High-Throughput Serving with
+ * vLLM & PagedAttention", dataarena.dev; blog "vLLM PagedAttention architecture
+ * deep dive", kashiiupdatez.online).  A sequence's keys and values are stored in
+ * fixed-size blocks of B tokens that sit at arbitrary frames of one pool; a
+ * per-sequence block table maps logical block j to its physical frame.
+ *
+ * Conventions for every call:
+ *  - Device buffers are owned by the caller.  The library never allocates
+ *    device memory; calls that need scratch take a caller-provided workspace.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream) and never
+ *    synchronise, except where stated (pkv_device_error, PKV_VALIDATE=1).
+ *  - Every argument is checked on the host before anything is launched; a bad
+ *    argument returns an error and launches nothing.  A launch failure returns
+ *    PKV_ECUDA.  Kernels never trap: an index that is out of range in device
+ *    data (a table entry, a context length, a slot, a copy pair) is skipped or
+ *    clamped and reported through the sticky device error flags below.
+ *  - Element types: fp16 or bf16 for q, out and the caches (`dtype`).
+ *    All row-major, C order, 16-byte aligned base pointers.
+ *  - Shapes the decode kernels support: head_dim in {64, 128}, block_size in
+ *    {8, 16, 32}, num_heads / num_kv_heads in {1, 2, 4, 8}.  Anything else
+ *    returns PKV_EUNSUPPORTED.
+ *
+ * Environment: PKV_VALIDATE=1 makes the decode and cache-write calls copy the
+ * block tables / context lengths / slots back to the host, check every index
+ * the kernels would use, and return PKV_ERANGE instead of launching when one is
+ * out of range (this synchronises the stream).
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_EINVAL = -1,       /* null pointer, negative size, misaligned buffer, bad workspace */
+  PKV_EUNSUPPORTED = -2, /* a shape outside the supported set */
+  PKV_ECUDA = -3,        /* a CUDA runtime call or launch failed */
+  PKV_ENOMEM = -4,       /* block pool exhausted (allocator) */
+  PKV_ERANGE = -5        /* an index out of range (host-checked data, PKV_VALIDATE) */
+} pkv_status;
+
+typedef enum { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+/* Sticky device error flags (bit mask), set by kernels instead of trapping. */
+#define PKV_DEVERR_TABLE_ENTRY 1u  /* a block-table entry outside [0, num_blocks): frame 0 read instead */
+#define PKV_DEVERR_CONTEXT_LEN 2u  /* a context length < 0 or above the table's capacity: clamped */
+#define PKV_DEVERR_SLOT 4u         /* a slot >= num_blocks * block_size: row not written */
+#define PKV_DEVERR_COPY_PAIR 8u    /* a copy pair naming a frame outside [0, num_blocks): skipped */
+#define PKV_DEVERR_WAIT_TIMEOUT 16u /* a bounded shared-memory barrier wait expired: output invalid */
+
+/* Human-readable name of a status code (static storage). */
+const char* pkv_status_string(pkv_status status);
+
+/* Reads the device error flags of the current device into *flags_out after the
+ * work queued on `stream` has finished (synchronises `stream`); clears them
+ * when `clear` != 0. */
+pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention                                                         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Bytes of workspace the decode calls need: 0 when every sequence fits in one
+ * context partition (max_context_len <= partition_size), else
+ * num_seqs * num_heads * P * (head_dim + 2) * 4 rounded up to 256, with
+ * P = ceil(max_context_len / partition_size).  partition_size 0 = default (512).
+ * Returns 0 for invalid arguments as well; the decode call then rejects them.
+ */
+size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
+                                  int32_t max_context_len, int32_t partition_size);
+
+/*
+ * Paged decode attention (slides 9-10 "PagedAttention: attention block by block",
+ * "Block table: logical to physical"; dataarena note section 2).
+ *
+ * For each sequence s and query head h (kv head g = h / (num_heads/num_kv_heads)):
+ *   out[s,h,:] = sum_t softmax_t(scale * q[s,h,:] . K_s[t,:]) V_s[t,:],  t < context_lens[s]
+ * where token t of sequence s lives in frame p = block_tables[s, t / B] at
+ * offset t mod B:  K_s[t,:] = k_cache[p, g, t mod B, :]  (V likewise).
+ * Accumulation is fp32; out is rounded to `dtype` (round to nearest even).
+ * context_lens[s] == 0 gives out[s] = 0.
+ *
+ *   out          device [num_seqs, num_heads, head_dim]              dtype, written
+ *   q            device [num_seqs, num_heads, head_dim]              dtype
+ *   k_cache      device [num_blocks, num_kv_heads, block_size, head_dim] dtype
+ *   v_cache      device, same shape as k_cache
+ *   block_tables device int32 [num_seqs, max_blocks_per_seq]; only the first
+ *                ceil(context_lens[s] / block_size) entries of row s are read
+ *   context_lens device int32 [num_seqs], 0 <= context_lens[s] <= max_blocks_per_seq * block_size
+ *   partition_size tokens per context partition (0 = 512); a multiple of 32 in [32, 8192].
+ *                Contexts longer than one partition are split across CTAs and merged
+ *                in a second pass (log-sum-exp), which needs the workspace.
+ *   workspace    device scratch of pkv_decode_workspace_bytes(num_seqs, num_heads,
+ *                head_dim, max_blocks_per_seq * block_size, partition_size) bytes
+ *                (may be NULL when that is 0); 16-byte aligned; contents need no
+ *                initialisation and are garbage afterwards.
+ */
+pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* block_tables,
+                                      const int32_t* context_lens, int32_t num_seqs,
+                                      int32_t max_blocks_per_seq, int32_t num_blocks, float scale,
+                                      int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t block_size, pkv_dtype dtype, int32_t partition_size,
+                                      void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream);
+
+/*
+ * The same attention over a contiguous cache, one max-length reservation per
+ * sequence (the layout of slides 6-7 and the dataarena note section 1 that
+ * paging replaces).  Kept as the measurement baseline for the cost of the
+ * indirection (slide 19: "a 20-26 % slower kernel").
+ *
+ *   k, v   device [num_seqs, num_kv_heads, max_context_len, head_dim] dtype
+ *   context_lens device int32 [num_seqs], 0 <= context_lens[s] <= max_context_len
+ *   workspace: pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+ *   max_context_len, partition_size) bytes.  Other arguments as above.
+ */
+pkv_status pkv_contiguous_attention_decode(void* out, const void* q, const void* k, const void* v,
+                                           const int32_t* context_lens, int32_t num_seqs,
+                                           int32_t max_context_len, float scale, int32_t num_heads,
+                                           int32_t num_kv_heads, int32_t head_dim, pkv_dtype dtype,
+                                           int32_t partition_size, void* workspace,
+                                           size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Cache write and copy-on-write block copy                                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Cache write (slide 11 "New block only when the last fills": each new token's
+ * key and value go into the slot the allocator reserved for it).
+ * For every token i with slot = slot_mapping[i] >= 0 and every kv head g:
+ *   k_cache[slot / B, g, slot mod B, :] = key[i, g, :]   (and v_cache / value)
+ * A negative slot is padding and is skipped.  Byte copies: bit-exact.
+ *
+ *   key, value   device [num_tokens, num_kv_heads, head_dim] dtype
+ *   k_cache, v_cache device [num_blocks, num_kv_heads, block_size, head_dim] dtype, updated
+ *   slot_mapping device int64 [num_tokens]; slots must be distinct (two tokens
+ *                writing one slot race).  A slot >= num_blocks * block_size is
+ *                not written and sets PKV_DEVERR_SLOT.
+ *   head_dim * element size must be a multiple of 16 bytes.
+ */
+pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                                 const int64_t* slot_mapping, int32_t num_tokens,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int32_t num_blocks, pkv_dtype dtype, cudaStream_t stream);
+
+/*
+ * Copy-on-write block copy (slide 13 "Parallel samples: copy on write ... only
+ * the last block is ever copied"; dataarena note section 3.2).
+ * For each pair i: frame dst of k_cache and of v_cache becomes a copy of frame src.
+ *
+ *   src_dst_pairs device int64 [num_pairs, 2] = (src, dst) frame indices.  All
+ *                pairs run concurrently: destinations must be distinct and no
+ *                destination may be the source of another pair (the allocator's
+ *                copy lists satisfy this).  src == dst is a no-op.  A frame index
+ *                outside [0, num_blocks) skips the pair and sets PKV_DEVERR_COPY_PAIR.
+ *   block_bytes  bytes of one frame of one cache = num_kv_heads * block_size *
+ *                head_dim * element size; a multiple of 16.
+ */
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs,
+                           int32_t num_pairs, int64_t block_bytes, int32_t num_blocks,
+                           cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Host block allocator                                                     */
+/* ------------------------------------------------------------------------ */
+/*
+ * Refcounted block allocator (slides 10-14; dataarena note sections 2, 3.1,
+ * 3.2 and 4 step 2).  Host memory only; one handle per pool; not thread-safe.
+ *  - Free frames form a FIFO queue, initially frame_order[0..N-1] (NULL = 0..N-1).
+ *    A sequence takes frames from the head; a frame whose count drops to 0 goes
+ *    to the tail.
+ *  - A prompt of n tokens takes ceil(n / B) frames (all-or-nothing: PKV_ENOMEM and
+ *    no change when the pool has fewer free frames).
+ *  - Appending token t writes into the last block when it has room (t mod B != 0)
+ *    and its count is 1; when it has room but is shared (count > 1), the writer
+ *    gets a new frame and a copy pair (shared frame, new frame) is emitted for
+ *    pkv_copy_blocks, to run before the cache write.  When t mod B == 0 a new
+ *    frame is taken and nothing is copied.
+ *  - fork() shares every frame of the parent (counts + 1); free() drops the counts.
+ *  - slot = frame * B + t mod B.
+ */
+typedef struct pkv_allocator pkv_allocator;
+
+typedef struct {
+  int64_t used_blocks;    /* frames with count > 0 */
+  int64_t free_blocks;    /* frames in the free queue */
+  int64_t tokens;         /* sum of the live sequences' lengths */
+  int64_t shared_blocks;  /* frames with count > 1 */
+  int64_t logical_blocks; /* sum of the live sequences' table lengths */
+} pkv_alloc_stats_t;
+
+pkv_status pkv_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* frame_order,
+                            pkv_allocator** out);
+void pkv_alloc_destroy(pkv_allocator* alloc);
+/* New sequence with prompt_len tokens; slots_out (host int64 [prompt_len], may be
+ * NULL) receives the slot of every prompt token. */
+pkv_status pkv_alloc_add_seq(pkv_allocator* alloc, int32_t seq_id, int32_t prompt_len,
+                             int64_t* slots_out);
+/* child shares all of parent's frames (parallel sampling, beam search). */
+pkv_status pkv_alloc_fork(pkv_allocator* alloc, int32_t parent, int32_t child);
+/* Reserve the slot of the next token of seq_id; *cow_src/*cow_dst = -1 unless a
+ * copy is needed. */
+pkv_status pkv_alloc_append(pkv_allocator* alloc, int32_t seq_id, int64_t* slot_out,
+                            int32_t* cow_src, int32_t* cow_dst);
+/* One decode step: append one token to each of seq_ids[0..n-1] (distinct), in
+ * order.  slots_out: host int64 [n]; pairs_out: host int64 [n, 2] receives the
+ * copy pairs, *num_pairs_out their count.  All-or-nothing on PKV_ENOMEM. */
+pkv_status pkv_alloc_append_batch(pkv_allocator* alloc, const int32_t* seq_ids, int32_t n,
+                                  int64_t* slots_out, int64_t* pairs_out, int32_t* num_pairs_out);
+pkv_status pkv_alloc_free_seq(pkv_allocator* alloc, int32_t seq_id);
+/* Block tables of seq_ids as host int32 [n, max_blocks] padded with -1, and
+ * their lengths (lens_out may be NULL).  PKV_ERANGE if a table is longer than
+ * max_blocks. */
+pkv_status pkv_alloc_block_table(const pkv_allocator* alloc, const int32_t* seq_ids, int32_t n,
+                                 int32_t max_blocks, int32_t* table_out, int32_t* lens_out);
+pkv_status pkv_alloc_refcount(const pkv_allocator* alloc, int32_t block, int32_t* count_out);
+pkv_status pkv_alloc_stats(const pkv_allocator* alloc, pkv_alloc_stats_t* out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,305 @@
+// C ABI entry points (include/pkv.h): argument checks on the host, then launch.
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "cache_ops.cuh"
+#include "decode.cuh"
+#include "pkv.h"
+
+namespace pkv {
+
+// Sticky error flags of the kernels on each device (PKV_DEVERR_*).
+static __device__ unsigned int g_device_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kDefaultPartition = 512;
+
+struct DeviceInfo {
+  bool ready = false;
+  unsigned int* err = nullptr;  // device address of g_device_error
+  int num_sms = 0;
+};
+DeviceInfo g_devices[kMaxDevices];
+
+// Per-device set-up with that device current: the device address of the error
+// flag and the SM count.
+pkv_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ECUDA;
+  DeviceInfo& d = g_devices[dev];
+  if (!d.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return PKV_ECUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return PKV_ECUDA;
+    d.err = static_cast<unsigned int*>(p);
+    d.num_sms = sms;
+    d.ready = true;
+  }
+  *out = &d;
+  return PKV_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool validate_env() {
+  const char* v = getenv("PKV_VALIDATE");
+  return v && v[0] && strcmp(v, "0") != 0;
+}
+
+pkv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ECUDA; }
+
+bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+int resolve_partition(int32_t partition_size) {
+  return partition_size == 0 ? kDefaultPartition : partition_size;
+}
+
+bool valid_partition(int p) { return p >= 32 && p <= kMaxPartTokens && p % 32 == 0; }
+
+size_t workspace_bytes(int64_t S, int64_t Hq, int64_t D, int64_t max_ctx, int64_t part) {
+  const int64_t P = (max_ctx + part - 1) / part;
+  if (P <= 1) return 0;
+  const int64_t cells = S * Hq * P;
+  const int64_t bytes = cells * (D + 2) * 4;
+  return static_cast<size_t>((bytes + 255) / 256 * 256);
+}
+
+// Shared checks and launch of the paged and contiguous decode.
+pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pkv_dtype dtype,
+                         int32_t partition_size, void* workspace, size_t ws_bytes, bool paged,
+                         float scale, cudaStream_t stream) {
+  if (a.num_seqs == 0) return PKV_OK;
+  const int part = resolve_partition(partition_size);
+  if (!valid_partition(part)) return PKV_EINVAL;
+  const int group = a.num_heads / a.num_kv_heads;
+  a.part_tokens = part;
+  a.max_parts = (a.max_ctx + part - 1) / part;
+  if (a.max_parts < 1) a.max_parts = 1;
+  if (a.max_parts > 65535 || a.num_kv_heads > 65535 || a.num_seqs > 65535) return PKV_EUNSUPPORTED;
+  const size_t need = workspace_bytes(a.num_seqs, a.num_heads, head_dim, a.max_ctx, part);
+  if (need > 0) {
+    if (!workspace || ws_bytes < need || !aligned16(workspace)) return PKV_EINVAL;
+    const int64_t cells = static_cast<int64_t>(a.num_seqs) * a.num_heads * a.max_parts;
+    a.tmp_out = static_cast<float*>(workspace);
+    a.tmp_m = a.tmp_out + cells * head_dim;
+    a.tmp_l = a.tmp_m + cells;
+  } else {
+    a.tmp_out = a.tmp_m = a.tmp_l = nullptr;
+  }
+  a.scale_log2 = scale * 1.4426950408889634f;
+  DeviceInfo* dev = nullptr;
+  pkv_status st = device_info(&dev);
+  if (st != PKV_OK) return st;
+  a.err = dev->err;
+  cudaError_t e;
+  if (dtype == PKV_F16)
+    e = head_dim == 64 ? launch_decode<__half, 64>(a, group, block_size, paged, stream)
+                       : launch_decode<__half, 128>(a, group, block_size, paged, stream);
+  else
+    e = head_dim == 64 ? launch_decode<__nv_bfloat16, 64>(a, group, block_size, paged, stream)
+                       : launch_decode<__nv_bfloat16, 128>(a, group, block_size, paged, stream);
+  return from_cuda(e);
+}
+
+pkv_status check_heads(int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, pkv_dtype dtype) {
+  if (num_heads <= 0 || num_kv_heads <= 0) return PKV_EINVAL;
+  if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EUNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PKV_EUNSUPPORTED;
+  if (num_heads % num_kv_heads != 0 || !supported_group(num_heads / num_kv_heads))
+    return PKV_EUNSUPPORTED;
+  return PKV_OK;
+}
+
+// PKV_VALIDATE=1: copy the tables and lengths back and check every entry the
+// kernel would read.
+pkv_status validate_decode_tables(const int32_t* tables, const int32_t* lens, int32_t S,
+                                  int32_t MB, int32_t N, int32_t B, cudaStream_t stream) {
+  std::vector<int32_t> h_lens(S), h_tab(static_cast<size_t>(S) * MB);
+  if (cudaMemcpyAsync(h_lens.data(), lens, sizeof(int32_t) * S, cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(h_tab.data(), tables, sizeof(int32_t) * h_tab.size(), cudaMemcpyDeviceToHost,
+                      stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return PKV_ECUDA;
+  for (int32_t s = 0; s < S; ++s) {
+    const int64_t L = h_lens[s];
+    if (L < 0 || L > static_cast<int64_t>(MB) * B) return PKV_ERANGE;
+    for (int64_t j = 0; j < (L + B - 1) / B; ++j) {
+      const int32_t p = h_tab[static_cast<size_t>(s) * MB + j];
+      if (p < 0 || p >= N) return PKV_ERANGE;
+    }
+  }
+  return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+const char* pkv_status_string(pkv_status status) {
+  switch (status) {
+    case PKV_OK: return "PKV_OK";
+    case PKV_EINVAL: return "PKV_EINVAL: invalid argument";
+    case PKV_EUNSUPPORTED: return "PKV_EUNSUPPORTED: unsupported shape or dtype";
+    case PKV_ECUDA: return "PKV_ECUDA: CUDA runtime error";
+    case PKV_ENOMEM: return "PKV_ENOMEM: block pool exhausted";
+    case PKV_ERANGE: return "PKV_ERANGE: index out of range";
+  }
+  return "unknown pkv_status";
+}
+
+pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t stream) {
+  if (!flags_out) return PKV_EINVAL;
+  DeviceInfo* dev = nullptr;
+  pkv_status st = device_info(&dev);
+  if (st != PKV_OK) return st;
+  unsigned int h = 0;
+  if (cudaMemcpyAsync(&h, dev->err, sizeof h, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return PKV_ECUDA;
+  if (clear && cudaMemsetAsync(dev->err, 0, sizeof h, stream) != cudaSuccess) return PKV_ECUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return PKV_ECUDA;
+  *flags_out = h;
+  return PKV_OK;
+}
+
+size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
+                                  int32_t max_context_len, int32_t partition_size) {
+  const int part = resolve_partition(partition_size);
+  if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+      !valid_partition(part))
+    return 0;
+  return workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, part);
+}
+
+pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* block_tables,
+                                      const int32_t* context_lens, int32_t num_seqs,
+                                      int32_t max_blocks_per_seq, int32_t num_blocks, float scale,
+                                      int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t block_size, pkv_dtype dtype, int32_t partition_size,
+                                      void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream) {
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || num_blocks <= 0) return PKV_EINVAL;
+  pkv_status st = check_heads(num_heads, num_kv_heads, head_dim, dtype);
+  if (st != PKV_OK) return st;
+  if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_EUNSUPPORTED;
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_EINVAL;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_EINVAL;
+  const int64_t max_ctx = static_cast<int64_t>(max_blocks_per_seq) * block_size;
+  if (max_ctx > (1 << 30)) return PKV_EUNSUPPORTED;
+  if (validate_env()) {
+    st = validate_decode_tables(block_tables, context_lens, num_seqs, max_blocks_per_seq,
+                                num_blocks, block_size, stream);
+    if (st != PKV_OK) return st;
+  }
+  DecodeArgs a{};
+  a.out = out;
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.tables = block_tables;
+  a.lens = context_lens;
+  a.num_seqs = num_seqs;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.max_ctx = static_cast<int32_t>(max_ctx);
+  return decode_common(a, head_dim, block_size, dtype, partition_size, workspace, workspace_bytes,
+                       true, scale, stream);
+}
+
+pkv_status pkv_contiguous_attention_decode(void* out, const void* q, const void* k, const void* v,
+                                           const int32_t* context_lens, int32_t num_seqs,
+                                           int32_t max_context_len, float scale, int32_t num_heads,
+                                           int32_t num_kv_heads, int32_t head_dim, pkv_dtype dtype,
+                                           int32_t partition_size, void* workspace,
+                                           size_t workspace_bytes, cudaStream_t stream) {
+  if (num_seqs < 0 || max_context_len < 0) return PKV_EINVAL;
+  pkv_status st = check_heads(num_heads, num_kv_heads, head_dim, dtype);
+  if (st != PKV_OK) return st;
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !q || !k || !v || !context_lens) return PKV_EINVAL;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return PKV_EINVAL;
+  if (max_context_len > (1 << 30)) return PKV_EUNSUPPORTED;
+  if (validate_env()) {
+    std::vector<int32_t> h(num_seqs);
+    if (cudaMemcpyAsync(h.data(), context_lens, sizeof(int32_t) * num_seqs,
+                        cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return PKV_ECUDA;
+    for (int32_t L : h)
+      if (L < 0 || L > max_context_len) return PKV_ERANGE;
+  }
+  DecodeArgs a{};
+  a.out = out;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.lens = context_lens;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.max_ctx = max_context_len;
+  return decode_common(a, head_dim, 32, dtype, partition_size, workspace, workspace_bytes, false,
+                       scale, stream);
+}
+
+pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                                 const int64_t* slot_mapping, int32_t num_tokens,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int32_t num_blocks, pkv_dtype dtype, cudaStream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PKV_EINVAL;
+  if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EUNSUPPORTED;
+  const int32_t row_bytes = head_dim * 2;
+  if (row_bytes % 16 != 0) return PKV_EUNSUPPORTED;
+  if (num_tokens == 0) return PKV_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PKV_EINVAL;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_EINVAL;
+  if (validate_env()) {
+    std::vector<int64_t> h(num_tokens);
+    if (cudaMemcpyAsync(h.data(), slot_mapping, sizeof(int64_t) * num_tokens,
+                        cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return PKV_ECUDA;
+    for (int64_t s : h)
+      if (s >= static_cast<int64_t>(num_blocks) * block_size) return PKV_ERANGE;
+  }
+  DeviceInfo* dev = nullptr;
+  pkv_status st = device_info(&dev);
+  if (st != PKV_OK) return st;
+  return from_cuda(launch_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, num_tokens,
+                                            num_kv_heads, row_bytes, block_size, num_blocks,
+                                            dev->num_sms, dev->err, stream));
+}
+
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_pairs,
+                           int32_t num_pairs, int64_t block_bytes, int32_t num_blocks,
+                           cudaStream_t stream) {
+  if (num_pairs < 0 || block_bytes <= 0 || num_blocks <= 0) return PKV_EINVAL;
+  if (block_bytes % 16 != 0) return PKV_EINVAL;
+  if (num_pairs > 65535) return PKV_EUNSUPPORTED;
+  if (num_pairs == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !src_dst_pairs) return PKV_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
+  DeviceInfo* dev = nullptr;
+  pkv_status st = device_info(&dev);
+  if (st != PKV_OK) return st;
+  return from_cuda(launch_copy_blocks(k_cache, v_cache, src_dst_pairs, num_pairs, block_bytes,
+                                      num_blocks, dev->err, stream));
+}
+
+}  // extern "C"

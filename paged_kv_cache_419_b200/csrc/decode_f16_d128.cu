@@ -1,0 +1,6 @@
+// Decode kernels for f16 caches with head_dim 128.
+#include "decode_launch.cuh"
+
+namespace pkv {
+template cudaError_t launch_decode<__half, 128>(const DecodeArgs&, int, int, bool, cudaStream_t);
+}  // namespace pkv

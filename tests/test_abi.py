@@ -1,0 +1,110 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function
+include/pkv.h declares, and rejects bad arguments on the host before any CUDA
+call.  No test here launches or allocates anything on a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_419_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"^[A-Za-z_][\w \*]*?\b(pkv_\w+)\s*\(", text, flags=re.M))
+
+
+def test_header_declares_the_binding_export_list():
+    assert declared_functions() == set(B.EXPORTS)
+
+
+def test_library_exports_every_declared_function():
+    lib = B.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    for code in (B.PKV_OK, B.PKV_EINVAL, B.PKV_EUNSUPPORTED, B.PKV_ECUDA, B.PKV_ENOMEM, B.PKV_ERANGE):
+        assert B.status_string(code).startswith("PKV_")
+
+
+def test_workspace_bytes_formula():
+    # no partitioning needed -> no workspace
+    assert B.decode_workspace_bytes(256, 32, 128, 512) == 0
+    # 4096 tokens in 512-token partitions: P = 8 cells of (D + 2) floats
+    S, Hq, D, ctx = 256, 32, 128, 4096
+    need = S * Hq * 8 * (D + 2) * 4
+    assert B.decode_workspace_bytes(S, Hq, D, ctx) == (need + 255) // 256 * 256
+    assert B.decode_workspace_bytes(4, 32, 128, 32768, 1024) == ((4 * 32 * 32 * 130 * 4 + 255) // 256) * 256
+    # invalid partition sizes give 0
+    assert B.decode_workspace_bytes(4, 32, 128, 32768, 48) == 0
+    assert B.decode_workspace_bytes(4, 32, 128, 32768, 16384) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: every call below fails first
+
+
+def _paged(**kw):
+    args = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, tables=FAKE, lens=FAKE, S=4, MB=8, N=64,
+                scale=0.1, Hq=8, Hkv=8, D=64, Bs=16, dt=B.PKV_F16, part=0, ws=None, wsb=0)
+    args.update(kw)
+    a = args
+    return B.lib().pkv_paged_attention_decode(a["out"], a["q"], a["k"], a["v"], a["tables"],
+                                              a["lens"], a["S"], a["MB"], a["N"], a["scale"],
+                                              a["Hq"], a["Hkv"], a["D"], a["Bs"], a["dt"],
+                                              a["part"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), B.PKV_EUNSUPPORTED),
+    (dict(D=256), B.PKV_EUNSUPPORTED),
+    (dict(Bs=12), B.PKV_EUNSUPPORTED),
+    (dict(Bs=64), B.PKV_EUNSUPPORTED),
+    (dict(Hq=12, Hkv=8), B.PKV_EUNSUPPORTED),     # Hq % Hkv != 0
+    (dict(Hq=48, Hkv=3), B.PKV_EUNSUPPORTED),     # group of 16
+    (dict(dt=7), B.PKV_EUNSUPPORTED),
+    (dict(S=-1), B.PKV_EINVAL),
+    (dict(MB=0), B.PKV_EINVAL),
+    (dict(N=0), B.PKV_EINVAL),
+    (dict(Hkv=0), B.PKV_EINVAL),
+    (dict(q=None), B.PKV_EINVAL),
+    (dict(out=None), B.PKV_EINVAL),
+    (dict(tables=None), B.PKV_EINVAL),
+    (dict(k=ctypes.c_void_p((1 << 20) + 8)), B.PKV_EINVAL),   # misaligned
+    (dict(part=48), B.PKV_EINVAL),                # not a multiple of 32
+    (dict(part=16384), B.PKV_EINVAL),             # above 8192
+    (dict(MB=64), B.PKV_EINVAL),                  # 1024 tokens > 512: workspace required
+])
+def test_paged_decode_rejects_bad_arguments_before_launch(kw, status):
+    assert _paged(**kw) == status
+
+
+def test_zero_sequences_is_a_no_op():
+    assert _paged(S=0, q=None, out=None) == B.PKV_OK
+
+
+def test_cache_ops_reject_bad_arguments_before_launch():
+    L = B.lib()
+    # head_dim 4 (8 bytes per row) cannot be moved in 16-byte vectors
+    assert L.pkv_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 4, 16, 8, 0, None) == B.PKV_EUNSUPPORTED
+    assert L.pkv_reshape_and_cache(None, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 0, None) == B.PKV_EINVAL
+    assert L.pkv_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 64, 16, 8, 0, None) == B.PKV_EINVAL
+    assert L.pkv_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 64, 16, 8, 0, None) == B.PKV_OK
+    assert L.pkv_copy_blocks(FAKE, FAKE, FAKE, 3, 24, 8, None) == B.PKV_EINVAL      # not 16-byte multiple
+    assert L.pkv_copy_blocks(FAKE, FAKE, None, 3, 4096, 8, None) == B.PKV_EINVAL
+    assert L.pkv_copy_blocks(FAKE, FAKE, FAKE, 70000, 4096, 8, None) == B.PKV_EUNSUPPORTED
+    assert L.pkv_copy_blocks(FAKE, FAKE, FAKE, 0, 4096, 8, None) == B.PKV_OK
+
+
+def test_contiguous_decode_rejects_bad_arguments_before_launch():
+    L = B.lib()
+    f = L.pkv_contiguous_attention_decode
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 512, 0.1, 8, 8, 80, 0, 0, None, 0, None) == B.PKV_EUNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 4, 512, 0.1, 8, 8, 64, 0, 0, None, 0, None) == B.PKV_EINVAL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2048, 0.1, 8, 8, 64, 0, 0, None, 0, None) == B.PKV_EINVAL

@@ -1,0 +1,146 @@
+"""The C++ block allocator in libpkv agrees with the Python reference model:
+same slots, tables, copy pairs, reference counts, statistics and errors, on the
+pages' traces and on long random operation scripts.  Host code only."""
+import numpy as np
+import pytest
+
+from oracle.allocator_model import AllocatorModel, AllocatorError
+from paged_kv_cache_419_b200.binding import BlockAllocator, PkvError, PKV_ENOMEM, PKV_EINVAL
+import workloads as wl
+
+
+def same_state(native, model, seqs, max_blocks):
+    if seqs:
+        table, lens = native.block_table(seqs, max_blocks)
+        mt, ml = model.block_table(seqs, max_blocks)
+        assert table.tolist() == mt and lens.tolist() == ml
+    for b in range(model.N):
+        assert native.refcount(b) == model.ref[b]
+    st = native.stats()
+    for k, v in model.stats().items():
+        assert st[k] == v, k
+
+
+def test_pages_trace_new_frame_only_when_last_fills():
+    n = BlockAllocator(8, 16)
+    assert n.add_seq(0, 15).tolist() == list(range(15))
+    assert n.append(0) == (15, -1, -1)
+    assert n.append(0) == (16, -1, -1)
+
+
+def test_cow_batch_step_emits_one_pair_per_writer_while_shared():
+    order = np.random.default_rng(0).permutation(256).astype(np.int32)
+    n, m = BlockAllocator(256, 16, order), AllocatorModel(256, 16, order)
+    for a in (n, m):
+        a.add_seq(0, 1000)
+        for c in (1, 2, 3):
+            a.fork(0, c)
+    slots, pairs = n.append_batch([0, 1, 2, 3])
+    exp_slots, exp_pairs = [], []
+    for s in range(4):
+        slot, src, dst = m.append(s)
+        exp_slots.append(slot)
+        if src >= 0:
+            exp_pairs.append([src, dst])
+    assert slots.tolist() == exp_slots and pairs.tolist() == exp_pairs and len(exp_pairs) == 3
+    same_state(n, m, [0, 1, 2, 3], 80)
+
+
+def test_enomem_changes_nothing():
+    n = BlockAllocator(4, 16)
+    n.add_seq(0, 40)
+    before = n.stats()
+    with pytest.raises(PkvError) as e:
+        n.add_seq(1, 17)
+    assert e.value.status == PKV_ENOMEM and n.stats() == before
+    n.add_seq(1, 16)
+    n.fork(1, 2)
+    # the step needs 2 frames (seq 1 and seq 2 both start a new block), 0 free
+    with pytest.raises(PkvError) as e:
+        n.append_batch([1, 2])
+    assert e.value.status == PKV_ENOMEM and n.stats()["tokens"] == 40 + 16 + 16
+
+
+def test_bad_ids_are_rejected():
+    n = BlockAllocator(8, 4)
+    n.add_seq(0, 3)
+    for call in (lambda: n.add_seq(0, 1), lambda: n.fork(5, 6), lambda: n.fork(0, 0),
+                 lambda: n.append(9), lambda: n.free_seq(9), lambda: n.append_batch([0, 0])):
+        with pytest.raises(PkvError) as e:
+            call()
+        assert e.value.status == PKV_EINVAL
+    with pytest.raises(PkvError):
+        BlockAllocator(4, 4, frame_order=[0, 1, 1, 2])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_scripts_match_the_model(seed):
+    rng = np.random.default_rng(100 + seed)
+    N, Bsz = int(rng.integers(16, 200)), int(rng.choice([8, 16, 32]))
+    order = rng.permutation(N).astype(np.int32)
+    n, m = BlockAllocator(N, Bsz, order), AllocatorModel(N, Bsz, order)
+    live, next_id = [], 0
+    for step in range(400):
+        op = rng.choice(["add", "fork", "append", "batch", "free"], p=[0.2, 0.15, 0.3, 0.2, 0.15])
+        if op == "add" or not live:
+            L = int(rng.integers(0, 3 * Bsz))
+            try:
+                exp = m.add_seq(next_id, L)
+            except AllocatorError:
+                with pytest.raises(PkvError):
+                    n.add_seq(next_id, L)
+            else:
+                assert n.add_seq(next_id, L).tolist() == exp
+                live.append(next_id)
+            next_id += 1
+        elif op == "fork":
+            p = int(rng.choice(live))
+            m.fork(p, next_id)
+            n.fork(p, next_id)
+            live.append(next_id)
+            next_id += 1
+        elif op == "append":
+            s = int(rng.choice(live))
+            try:
+                exp = m.append(s)
+            except AllocatorError:
+                with pytest.raises(PkvError):
+                    n.append(s)
+            else:
+                assert n.append(s) == exp
+        elif op == "batch":
+            k = int(rng.integers(1, len(live) + 1))
+            ids = [int(x) for x in rng.choice(live, size=k, replace=False)]
+            snapshot = (list(m.free), list(m.ref), {s: list(t) for s, t in m.tables.items()},
+                        dict(m.lens))
+            try:
+                exp = [m.append(s) for s in ids]
+            except AllocatorError:
+                m.free, m.ref = type(m.free)(snapshot[0]), snapshot[1]
+                m.tables, m.lens = snapshot[2], snapshot[3]
+                with pytest.raises(PkvError):
+                    n.append_batch(ids)
+            else:
+                slots, pairs = n.append_batch(ids)
+                assert slots.tolist() == [e[0] for e in exp]
+                assert pairs.tolist() == [[e[1], e[2]] for e in exp if e[1] >= 0]
+        else:
+            s = int(rng.choice(live))
+            live.remove(s)
+            m.free_seq(s)
+            n.free_seq(s)
+        if step % 25 == 0:
+            same_state(n, m, live, 64)
+    same_state(n, m, live, 64)
+
+
+def test_decode_workload_tables_follow_the_frame_order():
+    w = wl.WORKLOADS["gqa8b"]
+    inp = wl.make_decode_inputs(w, num_seqs=16)
+    n = BlockAllocator(w.num_blocks, w.block_size, inp.frame_order)
+    for s, L in enumerate(inp.context_lens):
+        n.add_seq(s, int(L))
+    table, lens = n.block_table(list(range(16)), w.max_blocks_per_seq)
+    used = np.concatenate([table[s][table[s] >= 0] for s in range(16)])
+    assert used.tolist() == inp.frame_order[: used.size].tolist()
+    assert lens.tolist() == inp.context_lens.tolist()

@@ -1,0 +1,322 @@
+"""Parity of the CUDA path with the CPU oracle (run on a B200).
+
+Tolerances are the stated bar: max-abs error <= 2e-3 for fp16 and <= 1e-2 for
+bf16 attention outputs against the fp64 oracle; cache writes and block copies
+bit-exact.  The pool is filled with NaN before use, so a read of any byte that
+no table entry / context length covers shows up as NaN in the output.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.allocator_model import AllocatorModel
+import workloads as wl
+from flow import (TOL, POISON, gpu_step_inputs, gpu_decode_step, oracle_step_inputs, oracle_decode,
+                  max_abs_err, to_dev, from_dev, torch_dtype)
+
+pytestmark = pytest.mark.gpu
+
+
+def _bin():
+    from paged_kv_cache_419_b200 import binding
+    return binding
+
+
+def run_and_compare(inp, partition_size=0, seqs=None, check_cache=True, poison=True):
+    B = _bin()
+    b = gpu_step_inputs(inp, poison=poison)
+    out = gpu_decode_step(inp, b, partition_size)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    ob = oracle_step_inputs(inp)
+    assert np.array_equal(b.tables_host, ob.tables)
+    ref = oracle_decode(inp, ob, seqs=seqs)
+    rows = slice(None) if seqs is None else slice(*seqs)
+    out_np = out.float().cpu().numpy()
+    assert np.isfinite(out_np[rows]).all()
+    err = max_abs_err(out, ref, rows)
+    assert err <= TOL[inp.w.dtype], f"max-abs error {err}"
+    if check_cache:
+        used = np.unique(ob.tables[ob.tables >= 0])
+        assert np.array_equal(from_dev(b.k_cache)[used], ob.k_cache[used])
+        assert np.array_equal(from_dev(b.v_cache)[used], ob.v_cache[used])
+    return out, ref, err, b, ob
+
+
+# ------------------------------------------------------------ the workloads
+def test_tiny_full():
+    inp = wl.make_decode_inputs("tiny")
+    run_and_compare(inp)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_mha13b_block_sizes(bs):
+    w = wl.WORKLOADS["mha13b"]
+    w = w if bs == 16 else w.with_block_size(bs)
+    inp = wl.make_decode_inputs(w)
+    run_and_compare(inp)
+
+
+def test_mha13b_contiguous_matches_oracle_and_paged():
+    B = _bin()
+    inp = wl.make_decode_inputs("mha13b")
+    w = inp.w
+    out_paged, ref, _, b, ob = run_and_compare(inp, check_cache=False)
+    max_ctx = 2048
+    k = torch.zeros(w.num_seqs, w.num_kv_heads, max_ctx, w.head_dim, dtype=torch_dtype(w.dtype), device="cuda")
+    v = torch.zeros_like(k)
+    ks, vs = to_dev(inp.k_stream, w.dtype), to_dev(inp.v_stream, w.dtype)
+    for s in range(w.num_seqs):
+        a, e = int(inp.offsets[s]), int(inp.offsets[s + 1])
+        k[s, :, : e - a] = ks[a:e].transpose(0, 1)
+        v[s, :, : e - a] = vs[a:e].transpose(0, 1)
+    out = torch.empty_like(b.q)
+    B.contiguous_attention_decode(out, b.q, k, v, b.lens, w.scale)
+    torch.cuda.synchronize()
+    assert max_abs_err(out, ref) <= TOL[w.dtype]
+    # same partitions, same arithmetic order: the paged and contiguous kernels agree exactly
+    assert torch.equal(out, out_paged)
+
+
+def test_gqa8b_full_size_sampled_sequences():
+    """The benchmark's batch and launch configuration (partition 512), all 256
+    sequences run on the GPU; the oracle checks 40 of them spread over the batch,
+    including the shortest and the longest."""
+    inp = wl.make_decode_inputs("gqa8b")
+    B = _bin()
+    b = gpu_step_inputs(inp)
+    out = gpu_decode_step(inp, b, 512)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    ob = oracle_step_inputs(inp)
+    assert np.array_equal(b.tables_host, ob.tables)
+    lens = inp.context_lens
+    picks = sorted(set([int(np.argmin(lens)), int(np.argmax(lens))] +
+                       list(np.random.default_rng(5).choice(len(lens), 38, replace=False))))
+    out_np = out.float().cpu().numpy().astype(np.float64)
+    assert np.isfinite(out_np).all()
+    worst = 0.0
+    for s in picks:
+        ref = oracle_decode(inp, ob, seqs=(s, s + 1))
+        worst = max(worst, float(np.abs(out_np[s] - ref[s]).max()))
+    assert worst <= TOL[wl.BF16], worst
+    # sampled frames of the cache are bit-identical to the oracle's scatter
+    used = np.unique(ob.tables[ob.tables >= 0])
+    sample = np.random.default_rng(6).choice(used, 512, replace=False)
+    got = b.k_cache[torch.from_numpy(sample).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, ob.k_cache[sample])
+    got = b.v_cache[torch.from_numpy(sample).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, ob.v_cache[sample])
+
+
+@pytest.mark.parametrize("part", [512, 2048, 8192])
+def test_long_context_partitions(part):
+    inp = wl.make_decode_inputs("long")
+    run_and_compare(inp, partition_size=part, check_cache=False)
+
+
+# ------------------------------------------------------------ edge cases
+EDGE_LENGTHS = [0, 1, 2, 7, 8, 9, 15, 16, 17, 31, 32, 33, 511, 512, 513, 1023, 1024, 1025, 2047]
+
+
+@pytest.mark.parametrize("dtype", [wl.F16, wl.BF16])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_shapes_and_ragged_lengths(dtype, D, G, bs):
+    Hkv = 2
+    lens = np.array([1, 2, 7, 8, 9, 15, 16, 17, 31, 32, 33, 63, 64, 65, 511, 512, 513, 1030],
+                    np.int32)
+    max_blocks = -(-int(lens.max()) // bs) + 1
+    w = wl.Workload("edge", 7, len(lens), G * Hkv, Hkv, D, bs, max_blocks * len(lens) + 5, dtype,
+                    max_blocks, 1.0 / np.sqrt(D), lengths=("uniform", 1, 2))
+    inp = wl.make_decode_inputs(w, lengths=lens)
+    run_and_compare(inp, partition_size=512)
+
+
+def test_zero_length_context_writes_zeros():
+    lens = np.array([0, 5, 0, 40], np.int32)
+    w = wl.Workload("zero", 8, 4, 8, 2, 128, 16, 64, wl.BF16, 4, 0.088, lengths=("uniform", 1, 2))
+    inp_full = wl.make_decode_inputs(w, lengths=np.maximum(lens, 1))
+    # build the batch with lengths >= 1, then set two lengths to 0 on both sides
+    B = _bin()
+    b = gpu_step_inputs(inp_full)
+    out = gpu_decode_step(inp_full, b)
+    lens_dev = torch.from_numpy(lens).cuda()
+    out0 = torch.full_like(out, 3.0)
+    B.paged_attention_decode(out0, b.q, b.k_cache, b.v_cache, b.tables, lens_dev, w.scale)
+    torch.cuda.synchronize()
+    assert torch.all(out0[0] == 0) and torch.all(out0[2] == 0)
+    assert torch.equal(out0[1], out[1]) and torch.equal(out0[3], out[3])
+
+
+def test_many_short_sequences():
+    lens = np.random.default_rng(9).integers(1, 40, size=4096).astype(np.int32)
+    w = wl.Workload("many", 9, 4096, 8, 2, 64, 16, 4096 * 3 + 8, wl.F16, 3, 0.125,
+                    lengths=("uniform", 1, 2))
+    inp = wl.make_decode_inputs(w, lengths=lens)
+    run_and_compare(inp, check_cache=False)
+
+
+def test_permutation_of_physical_frames_is_bit_identical():
+    B = _bin()
+    inp = wl.make_decode_inputs("mha13b")
+    w = inp.w
+    b = gpu_step_inputs(inp)
+    out = gpu_decode_step(inp, b)
+    pi = torch.from_numpy(np.random.default_rng(3).permutation(w.num_blocks)).cuda()
+    k2 = torch.empty_like(b.k_cache)
+    v2 = torch.empty_like(b.v_cache)
+    k2[pi] = b.k_cache
+    v2[pi] = b.v_cache
+    t2 = torch.where(b.tables >= 0, pi[b.tables.clamp(min=0).long()].int(), b.tables)
+    out2 = torch.empty_like(out)
+    B.paged_attention_decode(out2, b.q, k2, v2, t2, b.lens, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
+def test_partition_size_changes_stay_within_tolerance():
+    inp = wl.make_decode_inputs("mha13b")
+    outs = [run_and_compare(inp, partition_size=p, check_cache=False)[0] for p in (64, 512, 8192)]
+    assert (outs[0].float() - outs[2].float()).abs().max().item() <= 2 * TOL[inp.w.dtype]
+
+
+# ------------------------------------------------------------ cache write / copy
+@pytest.mark.parametrize("dtype", [wl.F16, wl.BF16])
+@pytest.mark.parametrize("D", [64, 128])
+def test_reshape_and_cache_bit_exact(dtype, D):
+    B = _bin()
+    N, Hkv, bs, T = 96, 4, 16, 300
+    kc, vc = wl.random_pool(30 + D, N, Hkv, bs, D, dtype)
+    key, value = wl.make_token_rows(31 + D, T, Hkv, D, dtype)
+    slots = wl.random_slots(32 + D, T, N * bs, num_skipped=17)
+    gk, gv = to_dev(kc, dtype), to_dev(vc, dtype)
+    B.reshape_and_cache(to_dev(key, dtype), to_dev(value, dtype), gk, gv, torch.from_numpy(slots).cuda())
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    oracle.reshape_and_cache(kc, vc, key, value, slots, bs)
+    assert np.array_equal(from_dev(gk), kc) and np.array_equal(from_dev(gv), vc)
+
+
+def test_copy_blocks_bit_exact():
+    B = _bin()
+    N, Hkv, bs, D = 64, 8, 16, 128
+    kc, vc = wl.random_pool(40, N, Hkv, bs, D, wl.BF16)
+    rng = np.random.default_rng(41)
+    frames = rng.permutation(N)
+    pairs = np.stack([frames[:20], frames[20:40]], axis=1).astype(np.int64)
+    pairs = np.concatenate([pairs, [[frames[50], frames[50]]]])   # src == dst is a no-op
+    gk, gv = to_dev(kc, wl.BF16), to_dev(vc, wl.BF16)
+    B.copy_blocks(gk, gv, torch.from_numpy(pairs).cuda())
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    oracle.copy_blocks(kc, vc, pairs)
+    assert np.array_equal(from_dev(gk), kc) and np.array_equal(from_dev(gv), vc)
+
+
+# ------------------------------------------------------------ shared prefix + CoW
+def test_shared_prefix_parallel_sampling_with_copy_on_write():
+    """16 prompts x 4 samples: the prompt is written once, forked 3 times; every
+    generated token goes through allocator append -> copy_blocks (CoW pairs) ->
+    cache write, step by step; then decode over the mixed shared/private tables.
+    The oracle replays the same script with the allocator model."""
+    Bn = _bin()
+    inp = wl.make_shared_inputs()
+    w = inp.w
+    n = w.samples_per_prompt
+    S = w.num_seqs
+    shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+    td = torch_dtype(w.dtype)
+    gk = torch.full(shape, POISON[w.dtype], dtype=torch.int16, device="cuda").view(td)
+    gv = torch.full(shape, POISON[w.dtype], dtype=torch.int16, device="cuda").view(td)
+    ok = np.zeros(shape, np.uint16)
+    ov = np.zeros(shape, np.uint16)
+    na = Bn.BlockAllocator(w.num_blocks, w.block_size, inp.frame_order)
+    ma = AllocatorModel(w.num_blocks, w.block_size, inp.frame_order)
+    for p in range(w.num_prompts):
+        slots = na.add_seq(p * n, inp.prompt_len)
+        assert slots.tolist() == ma.add_seq(p * n, inp.prompt_len)
+        Bn.reshape_and_cache(to_dev(inp.prompt_k[p], w.dtype), to_dev(inp.prompt_v[p], w.dtype), gk, gv,
+                             torch.from_numpy(slots).cuda())
+        oracle.reshape_and_cache(ok, ov, inp.prompt_k[p], inp.prompt_v[p], slots, w.block_size)
+        for c in range(1, n):
+            na.fork(p * n, p * n + c)
+            ma.fork(p * n, p * n + c)
+    total_pairs = 0
+    for step in range(int(inp.gen_lens.max())):
+        ids = [s for s in range(S) if inp.gen_lens[s] > step]
+        slots, pairs = na.append_batch(ids)
+        exp = [ma.append(s) for s in ids]
+        assert slots.tolist() == [e[0] for e in exp]
+        assert pairs.tolist() == [[e[1], e[2]] for e in exp if e[1] >= 0]
+        rows = np.array([inp.gen_offsets[s] + step for s in ids])
+        if len(pairs):
+            Bn.copy_blocks(gk, gv, torch.from_numpy(pairs).cuda())
+            oracle.copy_blocks(ok, ov, pairs)
+            total_pairs += len(pairs)
+        Bn.reshape_and_cache(to_dev(inp.gen_k[rows], w.dtype), to_dev(inp.gen_v[rows], w.dtype), gk, gv,
+                             torch.from_numpy(slots).cuda())
+        oracle.reshape_and_cache(ok, ov, inp.gen_k[rows], inp.gen_v[rows], slots, w.block_size)
+    writers = (inp.gen_lens.reshape(w.num_prompts, n) > 0).sum(axis=1)
+    assert total_pairs == int(np.minimum(writers, n - 1).sum())
+    table, lens = na.block_table(np.arange(S, dtype=np.int32), w.max_blocks_per_seq)
+    mt, ml = ma.block_table(range(S), w.max_blocks_per_seq)
+    assert table.tolist() == mt and lens.tolist() == ml
+    q = to_dev(inp.q, w.dtype)
+    out = torch.empty_like(q)
+    Bn.paged_attention_decode(out, q, gk, gv, torch.from_numpy(table).cuda(),
+                              torch.from_numpy(lens).cuda(), w.scale)
+    torch.cuda.synchronize()
+    assert Bn.device_error() == 0
+    used = np.unique(table[table >= 0])
+    assert np.array_equal(from_dev(gk)[used], ok[used]) and np.array_equal(from_dev(gv)[used], ov[used])
+    ref = oracle.paged_decode(inp.q, ok, ov, np.array(mt, np.int32), np.array(ml, np.int32), w.scale,
+                              w.num_kv_heads, w.block_size, w.dtype)
+    assert max_abs_err(out, ref) <= TOL[w.dtype]
+
+
+# ------------------------------------------------------------ bad device data
+def test_bad_indices_set_device_flags_without_faulting():
+    B = _bin()
+    inp = wl.make_decode_inputs("tiny")
+    w = inp.w
+    b = gpu_step_inputs(inp)
+    gpu_decode_step(inp, b)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    out = torch.empty_like(b.q)
+    bad = b.tables.clone()
+    bad[0, 0] = w.num_blocks + 5
+    B.paged_attention_decode(out, b.q, b.k_cache, b.v_cache, bad, b.lens, w.scale)
+    assert B.device_error() & B.DEVERR_TABLE_ENTRY
+    lens = b.lens.clone()
+    lens[1] = w.max_blocks_per_seq * w.block_size + 3
+    B.paged_attention_decode(out, b.q, b.k_cache, b.v_cache, b.tables, lens, w.scale)
+    assert B.device_error() & B.DEVERR_CONTEXT_LEN
+    slots = torch.tensor([w.num_blocks * w.block_size + 1, -1, 3, 4], dtype=torch.int64, device="cuda")
+    B.reshape_and_cache(b.new_k, b.new_v, b.k_cache, b.v_cache, slots)
+    assert B.device_error() == B.DEVERR_SLOT
+    B.copy_blocks(b.k_cache, b.v_cache, torch.tensor([[0, w.num_blocks]], dtype=torch.int64, device="cuda"))
+    assert B.device_error() == B.DEVERR_COPY_PAIR
+    assert B.device_error() == 0
+
+
+def test_validate_env_rejects_bad_tables_before_launch(monkeypatch):
+    B = _bin()
+    inp = wl.make_decode_inputs("tiny")
+    w = inp.w
+    b = gpu_step_inputs(inp)
+    monkeypatch.setenv("PKV_VALIDATE", "1")
+    bad = b.tables.clone()
+    bad[2, 0] = -1
+    out = torch.zeros_like(b.q)
+    with pytest.raises(B.PkvError) as e:
+        B.paged_attention_decode(out, b.q, b.k_cache, b.v_cache, bad, b.lens, w.scale)
+    assert e.value.status == B.PKV_ERANGE
+    B.paged_attention_decode(out, b.q, b.k_cache, b.v_cache, b.tables, b.lens, w.scale)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
