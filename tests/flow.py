@@ -110,9 +110,10 @@ class OracleBatch:
     lens: np.ndarray
 
 
-def oracle_step_inputs(inp: wl.DecodeInputs) -> OracleBatch:
+def oracle_step_inputs(inp: wl.DecodeInputs, poison: bool = True) -> OracleBatch:
     """The same step on the CPU: allocator model, oracle scatter of the context and
-    of the appended token."""
+    of the appended token.  The pool starts with the same fill as the GPU pool
+    (NaN bit patterns, or zeros), so whole frames can be compared byte for byte."""
     w = inp.w
     S = w.num_seqs
     m = AllocatorModel(w.num_blocks, w.block_size, inp.frame_order)
@@ -121,8 +122,9 @@ def oracle_step_inputs(inp: wl.DecodeInputs) -> OracleBatch:
         pre += m.add_seq(s, int(inp.context_lens[s]) - 1)
     new = [m.append(s)[0] for s in range(S)]
     shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
-    kc = np.zeros(shape, np.uint16)
-    vc = np.zeros(shape, np.uint16)
+    fill = POISON[w.dtype] if poison else 0
+    kc = np.full(shape, fill, np.uint16)
+    vc = np.full(shape, fill, np.uint16)
     pk, pv, nk, nv = split_stream(inp)
     oracle.reshape_and_cache(kc, vc, pk, pv, np.array(pre, np.int64), w.block_size)
     oracle.reshape_and_cache(kc, vc, nk, nv, np.array(new, np.int64), w.block_size)

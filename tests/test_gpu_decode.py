@@ -31,7 +31,7 @@ def run_and_compare(inp, partition_size=0, seqs=None, check_cache=True, poison=T
     out = gpu_decode_step(inp, b, partition_size)
     torch.cuda.synchronize()
     assert B.device_error() == 0
-    ob = oracle_step_inputs(inp)
+    ob = oracle_step_inputs(inp, poison=poison)
     assert np.array_equal(b.tables_host, ob.tables)
     ref = oracle_decode(inp, ob, seqs=seqs)
     rows = slice(None) if seqs is None else slice(*seqs)
@@ -233,8 +233,8 @@ def test_shared_prefix_parallel_sampling_with_copy_on_write():
     td = torch_dtype(w.dtype)
     gk = torch.full(shape, POISON[w.dtype], dtype=torch.int16, device="cuda").view(td)
     gv = torch.full(shape, POISON[w.dtype], dtype=torch.int16, device="cuda").view(td)
-    ok = np.zeros(shape, np.uint16)
-    ov = np.zeros(shape, np.uint16)
+    ok = np.full(shape, POISON[w.dtype], np.uint16)
+    ov = np.full(shape, POISON[w.dtype], np.uint16)
     na = Bn.BlockAllocator(w.num_blocks, w.block_size, inp.frame_order)
     ma = AllocatorModel(w.num_blocks, w.block_size, inp.frame_order)
     for p in range(w.num_prompts):
