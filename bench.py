@@ -24,6 +24,7 @@ time.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -58,6 +59,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="gqa8b", choices=["tiny", "mha13b", "gqa8b", "long"])
     ap.add_argument("--block-size", type=int, default=0, help="override the workload's block size")
     ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="smaller batch of the same length law, pool sized to fit (profiling)")
     ap.add_argument("--no-contiguous", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -179,6 +182,9 @@ def workload(args):
     w = wl.WORKLOADS[args.workload]
     if args.block_size and args.block_size != w.block_size:
         w = w.with_block_size(args.block_size)
+    if args.num_seqs:
+        w = dataclasses.replace(w, num_seqs=args.num_seqs,
+                                num_blocks=min(w.num_blocks, args.num_seqs * w.max_blocks_per_seq))
     return w
 
 
