@@ -117,6 +117,38 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
                                       cudaStream_t stream);
 
 /*
+ * Allocation-free variant of pkv_paged_attention_decode.  The pages describe no
+ * counterpart; it exists for callers that cannot allocate device memory when
+ * they run decode (an engine that fixes its whole device-memory plan up front,
+ * a plugin hook that must not allocate, code whose allocator belongs to someone
+ * else), so it takes no workspace argument.
+ *
+ * Its scratch is one array of PKV_STATIC_WORKSPACE_BYTES inside the library's
+ * device memory, held by every GPU that loads the library until the process
+ * exits.  The call allocates and frees nothing.  Limits and behaviour:
+ *  - Shapes whose workspace (pkv_decode_workspace_bytes with max_context_len =
+ *    max_blocks_per_seq * block_size) exceeds PKV_STATIC_WORKSPACE_BYTES return
+ *    PKV_EUNSUPPORTED and launch nothing; use pkv_paged_attention_decode then.
+ *  - The first call on a device that needs scratch looks up the array's device
+ *    address (cudaGetSymbolAddress, with that device current); make that first
+ *    call before any stream capture.
+ *  - All calls share the one array per device: calls that may overlap on the GPU
+ *    (different streams, no ordering between them) race on it.  Calls ordered on
+ *    one stream are fine.  The array keeps the last call's contents; nothing in it
+ *    needs to start at zero.
+ * Arguments, results and errors are otherwise those of pkv_paged_attention_decode.
+ */
+#define PKV_STATIC_WORKSPACE_BYTES (16u << 20)
+
+pkv_status pkv_paged_attention_decode_static(void* out, const void* q, const void* k_cache,
+                                             const void* v_cache, const int32_t* block_tables,
+                                             const int32_t* context_lens, int32_t num_seqs,
+                                             int32_t max_blocks_per_seq, int32_t num_blocks,
+                                             float scale, int32_t num_heads, int32_t num_kv_heads,
+                                             int32_t head_dim, int32_t block_size, pkv_dtype dtype,
+                                             int32_t partition_size, cudaStream_t stream);
+
+/*
  * The same attention over a contiguous cache, one max-length reservation per
  * sequence (the layout of slides 6-7 and the dataarena note section 1 that
  * paging replaces).  Kept as the measurement baseline for the cost of the

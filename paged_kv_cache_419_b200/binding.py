@@ -24,7 +24,8 @@ DEVERR_TABLE_ENTRY, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_COPY_PAIR, DEVERR_WA
 # Every function include/pkv.h declares.
 EXPORTS = (
     "pkv_status_string", "pkv_device_error", "pkv_decode_workspace_bytes",
-    "pkv_paged_attention_decode", "pkv_contiguous_attention_decode", "pkv_reshape_and_cache",
+    "pkv_paged_attention_decode", "pkv_paged_attention_decode_static",
+    "pkv_contiguous_attention_decode", "pkv_reshape_and_cache",
     "pkv_copy_blocks", "pkv_alloc_create", "pkv_alloc_destroy", "pkv_alloc_add_seq",
     "pkv_alloc_fork", "pkv_alloc_append", "pkv_alloc_append_batch", "pkv_alloc_free_seq",
     "pkv_alloc_block_table", "pkv_alloc_refcount", "pkv_alloc_stats",
@@ -64,6 +65,9 @@ def lib() -> ctypes.CDLL:
             "pkv_paged_attention_decode": (
                 [P, P, P, P, P, P, i32, i32, i32, f32, i32, i32, i32, i32, ctypes.c_int, i32, P, sz,
                  P], ctypes.c_int),
+            "pkv_paged_attention_decode_static": (
+                [P, P, P, P, P, P, i32, i32, i32, f32, i32, i32, i32, i32, ctypes.c_int, i32, P],
+                ctypes.c_int),
             "pkv_contiguous_attention_decode": (
                 [P, P, P, P, P, i32, i32, f32, i32, i32, i32, ctypes.c_int, i32, P, sz, P],
                 ctypes.c_int),
