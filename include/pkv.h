@@ -72,11 +72,13 @@ pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t str
 /* ------------------------------------------------------------------------ */
 
 /*
- * Bytes of workspace the decode calls need: 0 when every sequence fits in one
- * context partition (max_context_len <= partition_size), else
- * num_seqs * num_heads * P * (head_dim + 2) * 4 rounded up to 256, with
- * P = ceil(max_context_len / partition_size).  partition_size 0 = default (512).
- * Returns 0 for invalid arguments as well; the decode call then rejects them.
+ * Bytes of workspace the decode calls need (always > 0 for valid arguments):
+ * 256 bytes of work counters, 4 * num_seqs * num_heads bytes of merge counters,
+ * 8 * num_seqs * P bytes of work list, and, when P > 1, the partition results
+ * num_seqs * num_heads * P * (head_dim + 2) * 4 bytes; each piece rounded up to
+ * 256 bytes, with P = ceil(max_context_len / partition_size).  partition_size
+ * 0 = default (512).  Returns 0 for invalid arguments; the decode call then
+ * rejects them.
  */
 size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
                                   int32_t max_context_len, int32_t partition_size);
@@ -99,13 +101,17 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t h
  *   block_tables device int32 [num_seqs, max_blocks_per_seq]; only the first
  *                ceil(context_lens[s] / block_size) entries of row s are read
  *   context_lens device int32 [num_seqs], 0 <= context_lens[s] <= max_blocks_per_seq * block_size
- *   partition_size tokens per context partition (0 = 512); a multiple of 32 in [32, 8192].
- *                Contexts longer than one partition are split across CTAs and merged
- *                in a second pass (log-sum-exp), which needs the workspace.
+ *   partition_size maximum tokens per context partition (0 = 512); a multiple of 32
+ *                in [32, 4096].  A context of L tokens is split into ceil(L / partition_size)
+ *                near-equal partitions (multiples of 32 tokens) that run on different
+ *                CTAs and are merged with a log-sum-exp in the same launch sequence.
  *   workspace    device scratch of pkv_decode_workspace_bytes(num_seqs, num_heads,
- *                head_dim, max_blocks_per_seq * block_size, partition_size) bytes
- *                (may be NULL when that is 0); 16-byte aligned; contents need no
- *                initialisation and are garbage afterwards.
+ *                head_dim, max_blocks_per_seq * block_size, partition_size) bytes,
+ *                16-byte aligned; contents need no initialisation and are garbage
+ *                afterwards.  Calls that may overlap on the GPU need separate workspaces.
+ *
+ * Launches: a one-CTA planning kernel (work list, counters) and the persistent
+ * decode kernel (programmatic dependent launch), in that order on `stream`.
  */
 pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
                                       const void* v_cache, const int32_t* block_tables,

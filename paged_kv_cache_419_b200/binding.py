@@ -134,7 +134,7 @@ def decode_workspace_bytes(num_seqs: int, num_heads: int, head_dim: int, max_con
 
 def _workspace(workspace, need: int, device):
     if need == 0:
-        return None, 0
+        raise ValueError("invalid decode arguments (no workspace size)")
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
     if workspace.numel() * workspace.element_size() < need:

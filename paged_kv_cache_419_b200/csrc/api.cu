@@ -62,12 +62,28 @@ int resolve_partition(int32_t partition_size) {
 
 bool valid_partition(int p) { return p >= 32 && p <= kMaxPartTokens && p % 32 == 0; }
 
+int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
+
+// Workspace layout: [work counters | merge counters (S x Hq >= S x Hkv) |
+// item list (S x P) | partition results (only when P > 1)].
+struct WorkspaceLayout {
+  int64_t counters, merge, items, tmp, total;
+};
+
+WorkspaceLayout workspace_layout(int64_t S, int64_t Hq, int64_t D, int64_t max_ctx, int64_t part) {
+  int64_t P = (max_ctx + part - 1) / part;
+  if (P < 1) P = 1;
+  WorkspaceLayout w;
+  w.counters = 0;
+  w.merge = 256;
+  w.items = w.merge + round256(4 * S * Hq);
+  w.tmp = w.items + round256(8 * S * P);
+  w.total = w.tmp + (P > 1 ? round256(S * Hq * P * (D + 2) * 4) : 0);
+  return w;
+}
+
 size_t workspace_bytes(int64_t S, int64_t Hq, int64_t D, int64_t max_ctx, int64_t part) {
-  const int64_t P = (max_ctx + part - 1) / part;
-  if (P <= 1) return 0;
-  const int64_t cells = S * Hq * P;
-  const int64_t bytes = cells * (D + 2) * 4;
-  return static_cast<size_t>((bytes + 255) / 256 * 256);
+  return static_cast<size_t>(workspace_layout(S, Hq, D, max_ctx, part).total);
 }
 
 // Shared checks and launch of the paged and contiguous decode.
@@ -81,12 +97,16 @@ pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pk
   a.part_tokens = part;
   a.max_parts = (a.max_ctx + part - 1) / part;
   if (a.max_parts < 1) a.max_parts = 1;
-  if (a.max_parts > 65535 || a.num_kv_heads > 65535 || a.num_seqs > 65535) return PKV_EUNSUPPORTED;
-  const size_t need = workspace_bytes(a.num_seqs, a.num_heads, head_dim, a.max_ctx, part);
-  if (need > 0) {
-    if (!workspace || ws_bytes < need || !aligned16(workspace)) return PKV_EINVAL;
+  const WorkspaceLayout lay = workspace_layout(a.num_seqs, a.num_heads, head_dim, a.max_ctx, part);
+  if (!workspace || ws_bytes < static_cast<size_t>(lay.total) || !aligned16(workspace))
+    return PKV_EINVAL;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.work = reinterpret_cast<uint32_t*>(ws + lay.counters);
+  a.merge_cnt = reinterpret_cast<uint32_t*>(ws + lay.merge);
+  a.items = reinterpret_cast<int2*>(ws + lay.items);
+  if (a.max_parts > 1) {
     const int64_t cells = static_cast<int64_t>(a.num_seqs) * a.num_heads * a.max_parts;
-    a.tmp_out = static_cast<float*>(workspace);
+    a.tmp_out = reinterpret_cast<float*>(ws + lay.tmp);
     a.tmp_m = a.tmp_out + cells * head_dim;
     a.tmp_l = a.tmp_m + cells;
   } else {
@@ -97,13 +117,14 @@ pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pk
   pkv_status st = device_info(&dev);
   if (st != PKV_OK) return st;
   a.err = dev->err;
+  const int sms = dev->num_sms;
   cudaError_t e;
   if (dtype == PKV_F16)
-    e = head_dim == 64 ? launch_decode<__half, 64>(a, group, block_size, paged, stream)
-                       : launch_decode<__half, 128>(a, group, block_size, paged, stream);
+    e = head_dim == 64 ? launch_decode<__half, 64>(a, group, block_size, paged, sms, stream)
+                       : launch_decode<__half, 128>(a, group, block_size, paged, sms, stream);
   else
-    e = head_dim == 64 ? launch_decode<__nv_bfloat16, 64>(a, group, block_size, paged, stream)
-                       : launch_decode<__nv_bfloat16, 128>(a, group, block_size, paged, stream);
+    e = head_dim == 64 ? launch_decode<__nv_bfloat16, 64>(a, group, block_size, paged, sms, stream)
+                       : launch_decode<__nv_bfloat16, 128>(a, group, block_size, paged, sms, stream);
   return from_cuda(e);
 }
 

@@ -5,54 +5,76 @@
 
 namespace pkv {
 
+// Persistent grid size of one decode instantiation on the current device:
+// SM count x resident CTAs per SM (set up once per device).
 template <typename T, int D, int G, int B, bool PAGED>
-cudaError_t launch_decode_one(const DecodeArgs& a, cudaStream_t stream) {
+cudaError_t decode_grid(int num_sms, int* grid) {
   using Tr = DecodeTraits<T, D, G, B, PAGED>;
-  auto kern = decode_kernel<T, D, G, B, PAGED>;
-  // The opt-in shared-memory size is a per-device function attribute; set it
-  // once per device.
-  static bool configured[64] = {};
+  static int blocks_per_sm[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
+  if (blocks_per_sm[dev] == 0) {
+    auto kern = decode_kernel<T, D, G, B, PAGED>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    configured[dev] = true;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecodeThreads, Tr::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    blocks_per_sm[dev] = n > 0 ? n : 1;
   }
-  const dim3 grid(a.max_parts, a.num_kv_heads, a.num_seqs);
-  kern<<<grid, kDecodeThreads, Tr::SMEM_BYTES, stream>>>(a);
+  *grid = num_sms * blocks_per_sm[dev];
+  return cudaSuccess;
+}
+
+template <typename T, int D, int G, int B, bool PAGED>
+cudaError_t launch_decode_one(const DecodeArgs& a, int num_sms, cudaStream_t stream) {
+  using Tr = DecodeTraits<T, D, G, B, PAGED>;
+  int grid = 0;
+  cudaError_t e = decode_grid<T, D, G, B, PAGED>(num_sms, &grid);
+  if (e != cudaSuccess) return e;
+  plan_kernel<<<1, kPlanThreads, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (a.max_parts > 1) {
-    merge_partitions_kernel<T, D><<<dim3(a.num_heads, a.num_seqs), D, 0, stream>>>(a);
-    e = cudaGetLastError();
-  }
-  return e;
+  // Programmatic dependent launch: the decode CTAs may start (and set up their
+  // barriers) while the plan kernel finishes; they wait for it in-kernel.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<T, D, G, B, PAGED>, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 template <typename T, int D, int B, bool PAGED>
-cudaError_t launch_decode_group(const DecodeArgs& a, int group, cudaStream_t stream) {
+cudaError_t launch_decode_group(const DecodeArgs& a, int group, int num_sms, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_decode_one<T, D, 1, B, PAGED>(a, stream);
-    case 2: return launch_decode_one<T, D, 2, B, PAGED>(a, stream);
-    case 4: return launch_decode_one<T, D, 4, B, PAGED>(a, stream);
-    case 8: return launch_decode_one<T, D, 8, B, PAGED>(a, stream);
+    case 1: return launch_decode_one<T, D, 1, B, PAGED>(a, num_sms, stream);
+    case 2: return launch_decode_one<T, D, 2, B, PAGED>(a, num_sms, stream);
+    case 4: return launch_decode_one<T, D, 4, B, PAGED>(a, num_sms, stream);
+    case 8: return launch_decode_one<T, D, 8, B, PAGED>(a, num_sms, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <typename T, int D>
-cudaError_t launch_decode(const DecodeArgs& a, int group, int block_size, bool paged,
+cudaError_t launch_decode(const DecodeArgs& a, int group, int block_size, bool paged, int num_sms,
                           cudaStream_t stream) {
-  if (!paged) return launch_decode_group<T, D, 32, false>(a, group, stream);
+  if (!paged) return launch_decode_group<T, D, 32, false>(a, group, num_sms, stream);
   switch (block_size) {
-    case 8: return launch_decode_group<T, D, 8, true>(a, group, stream);
-    case 16: return launch_decode_group<T, D, 16, true>(a, group, stream);
-    case 32: return launch_decode_group<T, D, 32, true>(a, group, stream);
+    case 8: return launch_decode_group<T, D, 8, true>(a, group, num_sms, stream);
+    case 16: return launch_decode_group<T, D, 16, true>(a, group, num_sms, stream);
+    case 32: return launch_decode_group<T, D, 32, true>(a, group, num_sms, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -58,8 +58,9 @@ extern "C" pkv_status pkv_paged_attention_decode_static(
     const pkv_status st = scratch_address(&scratch);
     if (st != PKV_OK) return st;
   }
-  // The partition results in the scratch need no clearing: the merge reads only
-  // cells that the first pass of the same call has written.
+  // Nothing in the scratch needs clearing: every call's planning kernel writes the
+  // work list and zeroes the counters it uses, and the partition merge reads only
+  // results written earlier in the same call.
   return pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
                                     max_blocks_per_seq, num_blocks, scale, num_heads, num_kv_heads,
                                     head_dim, block_size, dtype, partition_size, scratch,

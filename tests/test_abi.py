@@ -34,17 +34,23 @@ def test_status_strings():
         assert B.status_string(code).startswith("PKV_")
 
 
+def _layout_bytes(S, Hq, D, ctx, part=512):
+    r = lambda x: (x + 255) // 256 * 256
+    P = max(1, -(-ctx // part))
+    return 256 + r(4 * S * Hq) + r(8 * S * P) + (r(S * Hq * P * (D + 2) * 4) if P > 1 else 0)
+
+
 def test_workspace_bytes_formula():
-    # no partitioning needed -> no workspace
-    assert B.decode_workspace_bytes(256, 32, 128, 512) == 0
+    # one partition per context: counters and the work list only
+    assert B.decode_workspace_bytes(256, 32, 128, 512) == _layout_bytes(256, 32, 128, 512)
+    assert B.decode_workspace_bytes(256, 32, 128, 512) < 1 << 20
     # 4096 tokens in 512-token partitions: P = 8 cells of (D + 2) floats
-    S, Hq, D, ctx = 256, 32, 128, 4096
-    need = S * Hq * 8 * (D + 2) * 4
-    assert B.decode_workspace_bytes(S, Hq, D, ctx) == (need + 255) // 256 * 256
-    assert B.decode_workspace_bytes(4, 32, 128, 32768, 1024) == ((4 * 32 * 32 * 130 * 4 + 255) // 256) * 256
+    assert B.decode_workspace_bytes(256, 32, 128, 4096) == _layout_bytes(256, 32, 128, 4096)
+    assert B.decode_workspace_bytes(256, 32, 128, 4096) > 256 * 32 * 8 * 130 * 4
+    assert B.decode_workspace_bytes(4, 32, 128, 32768, 1024) == _layout_bytes(4, 32, 128, 32768, 1024)
     # invalid partition sizes give 0
     assert B.decode_workspace_bytes(4, 32, 128, 32768, 48) == 0
-    assert B.decode_workspace_bytes(4, 32, 128, 32768, 16384) == 0
+    assert B.decode_workspace_bytes(4, 32, 128, 32768, 8192) == 0
 
 
 FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: every call below fails first
@@ -78,8 +84,8 @@ def _paged(**kw):
     (dict(tables=None), B.PKV_EINVAL),
     (dict(k=ctypes.c_void_p((1 << 20) + 8)), B.PKV_EINVAL),   # misaligned
     (dict(part=48), B.PKV_EINVAL),                # not a multiple of 32
-    (dict(part=16384), B.PKV_EINVAL),             # above 8192
-    (dict(MB=64), B.PKV_EINVAL),                  # 1024 tokens > 512: workspace required
+    (dict(part=8192), B.PKV_EINVAL),              # above 4096
+    (dict(MB=64), B.PKV_EINVAL),                  # no workspace given
 ])
 def test_paged_decode_rejects_bad_arguments_before_launch(kw, status):
     assert _paged(**kw) == status
@@ -108,3 +114,4 @@ def test_contiguous_decode_rejects_bad_arguments_before_launch():
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 512, 0.1, 8, 8, 80, 0, 0, None, 0, None) == B.PKV_EUNSUPPORTED
     assert f(FAKE, FAKE, FAKE, FAKE, None, 4, 512, 0.1, 8, 8, 64, 0, 0, None, 0, None) == B.PKV_EINVAL
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2048, 0.1, 8, 8, 64, 0, 0, None, 0, None) == B.PKV_EINVAL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 0.1, 8, 8, 64, 0, 0, None, 0, None) == B.PKV_EINVAL
