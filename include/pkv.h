@@ -73,12 +73,12 @@ pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t str
 
 /*
  * Bytes of workspace the decode calls need (always > 0 for valid arguments):
- * 256 bytes of work counters, 4 * num_seqs * num_heads bytes of merge counters,
- * 8 * num_seqs * P bytes of work list, and, when P > 1, the partition results
- * num_seqs * num_heads * P * (head_dim + 2) * 4 bytes; each piece rounded up to
- * 256 bytes, with P = ceil(max_context_len / partition_size).  partition_size
- * 0 = default (512).  Returns 0 for invalid arguments; the decode call then
- * rejects them.
+ * 256 bytes of work counters, 4 * num_seqs bytes of sequence list,
+ * 32 * num_seqs * P bytes of work records (one per context partition), and, when
+ * P > 1, the partition results num_seqs * num_heads * P * (head_dim + 2) * 4
+ * bytes; each piece rounded up to 256 bytes, with
+ * P = ceil(max_context_len / partition_size).  partition_size 0 = default (512).
+ * Returns 0 for invalid arguments; the decode call then rejects them.
  */
 size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
                                   int32_t max_context_len, int32_t partition_size);
@@ -110,8 +110,9 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t h
  *                16-byte aligned; contents need no initialisation and are garbage
  *                afterwards.  Calls that may overlap on the GPU need separate workspaces.
  *
- * Launches: a one-CTA planning kernel (work list, counters) and the persistent
- * decode kernel (programmatic dependent launch), in that order on `stream`.
+ * Launches, in this order on `stream`: a one-CTA planning kernel (work list),
+ * the persistent decode kernel and, when a context can span more than one
+ * partition, the partition merge kernel (both with programmatic dependent launch).
  */
 pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
                                       const void* v_cache, const int32_t* block_tables,

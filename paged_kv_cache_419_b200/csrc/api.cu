@@ -64,10 +64,10 @@ bool valid_partition(int p) { return p >= 32 && p <= kMaxPartTokens && p % 32 ==
 
 int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace layout: [work counters | merge counters (S x Hq >= S x Hkv) |
-// item list (S x P) | partition results (only when P > 1)].
+// Workspace layout: [work counters | list of multi-partition sequences (S) |
+// work records (S x P) | partition results (only when P > 1)].
 struct WorkspaceLayout {
-  int64_t counters, merge, items, tmp, total;
+  int64_t counters, merge, records, tmp, total;
 };
 
 WorkspaceLayout workspace_layout(int64_t S, int64_t Hq, int64_t D, int64_t max_ctx, int64_t part) {
@@ -76,8 +76,8 @@ WorkspaceLayout workspace_layout(int64_t S, int64_t Hq, int64_t D, int64_t max_c
   WorkspaceLayout w;
   w.counters = 0;
   w.merge = 256;
-  w.items = w.merge + round256(4 * S * Hq);
-  w.tmp = w.items + round256(8 * S * P);
+  w.records = w.merge + round256(4 * S);
+  w.tmp = w.records + round256(S * P * kRecordBytes);
   w.total = w.tmp + (P > 1 ? round256(S * Hq * P * (D + 2) * 4) : 0);
   return w;
 }
@@ -102,8 +102,9 @@ pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pk
     return PKV_EINVAL;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.work = reinterpret_cast<uint32_t*>(ws + lay.counters);
-  a.merge_cnt = reinterpret_cast<uint32_t*>(ws + lay.merge);
-  a.items = reinterpret_cast<int2*>(ws + lay.items);
+  a.merge_seqs = reinterpret_cast<int32_t*>(ws + lay.merge);
+  a.records = ws + lay.records;
+  a.block_size = block_size;
   if (a.max_parts > 1) {
     const int64_t cells = static_cast<int64_t>(a.num_seqs) * a.num_heads * a.max_parts;
     a.tmp_out = reinterpret_cast<float*>(ws + lay.tmp);

@@ -12,8 +12,8 @@
 //    is cut into n = ceil(L / part_tokens) near-equal partitions whose sizes are
 //    multiples of 32 tokens.  All G = Hq/Hkv query heads of the kv head share one
 //    K/V fetch.
-//  * plan_kernel (one CTA) lists the items, largest first, and zeroes the work
-//    counter and the per-(sequence, kv head) merge counters in the workspace.
+//  * plan_kernel (one CTA) lists the items, largest first, lists the contexts
+//    that span several partitions, and resets the work counter.
 //  * decode_kernel is persistent: (SM count x occupancy) CTAs, launched with
 //    programmatic dependent launch so that their set-up overlaps the plan.  Each
 //    CTA takes items from the list with an atomic counter until it runs dry.
@@ -30,13 +30,15 @@
 //    each lane owns D/32 output dims of all G heads.
 //  * Epilogue per item: the four warps merge in shared memory.  A one-partition
 //    context writes `out`; otherwise the partition's normalised output, max and
-//    sum go to the workspace, and the CTA that completes the last partition of a
-//    (sequence, kv head) merges them (log-sum-exp) and writes `out`.
+//    sum go to the workspace, and merge_kernel (launched behind the decode grid)
+//    merges the partitions of each such context (log-sum-exp) into `out`.
 //  * Scores are kept in base-2 units (q is pre-scaled by scale * log2 e), so the
 //    exponentials are single ex2 instructions.
 #pragma once
 
 #include <math_constants.h>
+
+#include <type_traits>
 
 #include "device.cuh"
 
@@ -52,15 +54,16 @@ struct DecodeArgs {
   int32_t num_seqs;
   int32_t max_blocks;     // paged: MB
   int32_t num_blocks;     // paged: N
+  int32_t block_size;     // paged: B
   int32_t num_heads;
   int32_t num_kv_heads;
   int32_t max_ctx;        // capacity in tokens: MB * B (paged) or the contiguous stride
   int32_t part_tokens;    // maximum tokens per partition (multiple of 32)
   int32_t max_parts;      // ceil(max_ctx / part_tokens): upper bound of partitions per context
   float scale_log2;       // scale * log2(e)
-  uint32_t* work;         // [0] next item, [1] item count
-  uint32_t* merge_cnt;    // [S * Hkv] partitions finished
-  int2* items;            // [S * max_parts] (sequence, partition), largest first
+  uint32_t* work;         // [0] next item, [1] item count, [2] multi-partition sequences
+  int32_t* merge_seqs;    // [S] sequences whose context spans more than one partition
+  uint8_t* records;       // [S * max_parts] work records, largest partition first (32 B each)
   float* tmp_out;         // [S, Hq, max_parts, D]
   float* tmp_m;           // [S, Hq, max_parts]
   float* tmp_l;           // [S, Hq, max_parts]
@@ -72,6 +75,9 @@ constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxPartTokens = 4096;
 constexpr int kPlanThreads = 1024;
 constexpr int kItemSlots = 2;
+// Work record of one (sequence, partition): int32 s, part, n_parts, t_begin,
+// n_tok, L, 0, 0.
+constexpr int kRecordBytes = 32;
 
 // Partitioning of a context of L tokens (L already clamped to [0, max_ctx]):
 // n partitions of `size` tokens (a multiple of 32), the last one shorter.
@@ -112,16 +118,17 @@ struct DecodeTraits {
   static constexpr int TILE_BYTES = TS * ROW_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int Q_BYTES = G * D * 2;
-  static constexpr int MAX_TABLE = PAGED ? kMaxPartTokens / B : 4;
+  static constexpr int MAX_TABLE = PAGED ? kMaxPartTokens / B : 4;  // table entries of one item
   // shared memory carve-up (bytes, 16-byte aligned pieces)
   static constexpr int OFF_Q = STAGES * STAGE_BYTES;
   static constexpr int OFF_ACC = OFF_Q + kItemSlots * Q_BYTES;          // [warps][G][D] f32
   static constexpr int OFF_P = OFF_ACC + kConsumerWarps * G * D * 4;    // [warps][TPW][G] (p, p)
-  static constexpr int OFF_TABLE = OFF_P + kConsumerWarps * TPW * G * 8;
-  static constexpr int OFF_STAT = OFF_TABLE + MAX_TABLE * 4;            // m, l per warp and head
+  static constexpr int OFF_REC = OFF_P + kConsumerWarps * TPW * G * 8;  // 2 record slots
+  static constexpr int OFF_TAB = OFF_REC + 2 * kRecordBytes;            // 2 table buffers
+  static constexpr int OFF_STAT = OFF_TAB + 2 * MAX_TABLE * 4;          // m, l per warp and head
   static constexpr int OFF_ITEM = OFF_STAT + 2 * kConsumerWarps * G * 4 + 16;
   static constexpr int OFF_BARS = OFF_ITEM + kItemSlots * 32;
-  static constexpr int SMEM_BYTES = OFF_BARS + (2 * STAGES + 2 * kItemSlots) * 8;
+  static constexpr int SMEM_BYTES = OFF_BARS + (2 * STAGES + 2 * kItemSlots + 2) * 8;
 
   static_assert(D % 64 == 0, "head_dim must be 64 or 128");
   static_assert(EPL % 8 == 0 && VPL >= 1, "score vectors are 16 bytes");
@@ -129,7 +136,7 @@ struct DecodeTraits {
   static_assert(TPW % TPR == 0, "whole rounds per stage");
   static_assert(TS % CH == 0 && NCH <= 32, "whole copies per stage, one lane each");
   static_assert(DPL == 2 || DPL == 4, "PV reads 4 or 8 bytes per lane");
-  static_assert(OFF_BARS % 8 == 0, "mbarriers are 8-byte aligned");
+  static_assert(OFF_BARS % 8 == 0 && OFF_STAT % 16 == 0, "alignment");
 };
 
 // Item slot handed from the producer to the consumers.
@@ -146,62 +153,91 @@ __device__ __forceinline__ void allow_dependent_launch() {
 }
 
 // ---------------------------------------------------------------- plan
-// One CTA: clamp the context lengths, list every (sequence, partition) in
-// decreasing order of size (counting sort on 32-token size classes), and zero
-// the work counter and the merge counters.
+// One CTA: clamp the context lengths, write one work record per (sequence,
+// partition) in decreasing order of partition size (counting sort on 32-token
+// size classes), list the sequences that span several partitions (for the
+// merge kernel), and reset the work counter.  Every global read is issued by
+// all threads at once (one round trip); the lengths are kept in shared memory
+// for the second pass.
+constexpr int kPlanSmemSeqs = 8192;
+
 static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeArgs a) {
+  // The decode grid may start its set-up now; it waits for this grid to finish
+  // before it reads anything written here.  This grid itself starts behind its
+  // predecessor on the stream and waits for it before reading any input.
+  allow_dependent_launch();
+  grid_dependency_wait();
   constexpr int kMaxClasses = kMaxPartTokens / 32 + 2;
   __shared__ uint32_t count[kMaxClasses];
   __shared__ uint32_t cursor[kMaxClasses];
-  __shared__ uint32_t total;
+  __shared__ uint32_t total, n_multi;
+  __shared__ int s_len[kPlanSmemSeqs];
   const int classes = a.part_tokens / 32 + 2;  // class c: size in (part - 32(c+1), part - 32c]; last: empty
+  const bool cached = a.num_seqs <= kPlanSmemSeqs;
   for (int c = threadIdx.x; c < classes; c += blockDim.x) count[c] = 0;
-  if (threadIdx.x == 0) total = 0;
-  const int cnt_len = a.num_seqs * a.num_kv_heads;
-  for (int i = threadIdx.x; i < cnt_len; i += blockDim.x) a.merge_cnt[i] = 0;
+  if (threadIdx.x == 0) total = n_multi = 0;
   __syncthreads();
-  auto size_class = [&](int sz) {
-    return sz == 0 ? classes - 1 : (a.part_tokens - sz) / 32;
-  };
+  auto size_class = [&](int sz) { return sz == 0 ? classes - 1 : (a.part_tokens - sz) / 32; };
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int raw = a.lens[s];
     if (raw < 0 || raw > a.max_ctx) set_error(a.err, PKV_DEVERR_CONTEXT_LEN);
     const int L = clamp_len(raw, a.max_ctx);
+    if (cached) s_len[s] = L;
     int n, size;
     partition_of(L, a.part_tokens, n, size);
     for (int p = 0; p < n; ++p) atomicAdd(&count[size_class(min(size, L - p * size))], 1u);
     atomicAdd(&total, static_cast<uint32_t>(n));
+    if (n > 1) a.merge_seqs[atomicAdd(&n_multi, 1u)] = s;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t run = 0;
-    for (int c = 0; c < classes; ++c) {
-      cursor[c] = run;
-      run += count[c];
+  if (threadIdx.x < 32) {  // exclusive scan of the class counts, one warp
+    const int lane = threadIdx.x;
+    constexpr int kPerLane = (kMaxClasses + 31) / 32;
+    uint32_t v[kPerLane], run = 0;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+      const int c = lane * kPerLane + i;
+      v[i] = c < classes ? count[c] : 0u;
+      run += v[i];
+    }
+    uint32_t incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    uint32_t base = incl - run;
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+      const int c = lane * kPerLane + i;
+      if (c < classes) cursor[c] = base;
+      base += v[i];
     }
   }
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
-    const int L = clamp_len(a.lens[s], a.max_ctx);
+    const int L = cached ? s_len[s] : clamp_len(a.lens[s], a.max_ctx);
     int n, size;
     partition_of(L, a.part_tokens, n, size);
     for (int p = 0; p < n; ++p) {
-      const uint32_t pos = atomicAdd(&cursor[size_class(min(size, L - p * size))], 1u);
-      a.items[pos] = make_int2(s, p);
+      const int t_begin = p * size;
+      const int n_tok = min(size, L - t_begin);
+      const uint32_t pos = atomicAdd(&cursor[size_class(n_tok)], 1u);
+      int4* rec = reinterpret_cast<int4*>(a.records + static_cast<int64_t>(pos) * kRecordBytes);
+      rec[0] = make_int4(s, p, n, t_begin);
+      rec[1] = make_int4(n_tok, L, 0, 0);
     }
   }
   if (threadIdx.x == 0) {
     a.work[0] = 0;
     a.work[1] = total * static_cast<uint32_t>(a.num_kv_heads);
+    a.work[2] = n_multi;
   }
-  __threadfence();
-  __syncthreads();
-  allow_dependent_launch();
 }
 
 // ---------------------------------------------------------------- decode
 template <typename T, int D, int G, int B, bool PAGED>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kernel(const DecodeArgs a) {
   using Tr = DecodeTraits<T, D, G, B, PAGED>;
   constexpr int STAGES = Tr::STAGES, TS = Tr::TS, LPT = Tr::LPT, LPH = Tr::LPH, TPR = Tr::TPR;
   constexpr int TPW = Tr::TPW, ROUNDS = Tr::ROUNDS, VPL = Tr::VPL, DPL = Tr::DPL;
@@ -212,13 +248,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
   uint64_t* empty = full + STAGES;
   uint64_t* item_full = empty + STAGES;
   uint64_t* item_empty = item_full + kItemSlots;
+  uint64_t* rec_bar = item_empty + kItemSlots;
   ItemInfo* items = reinterpret_cast<ItemInfo*>(smem + Tr::OFF_ITEM);
-  int32_t* s_table = reinterpret_cast<int32_t*>(smem + Tr::OFF_TABLE);
   float* s_acc = reinterpret_cast<float*>(smem + Tr::OFF_ACC);
   float2* s_p = reinterpret_cast<float2*>(smem + Tr::OFF_P);
   float* s_m = reinterpret_cast<float*>(smem + Tr::OFF_STAT);
   float* s_l = s_m + NW * G;
-  int* s_flag = reinterpret_cast<int*>(s_l + NW * G);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -232,6 +267,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
       mbar_init(&item_full[i], 1);
       mbar_init(&item_empty[i], NW);
     }
+    mbar_init(&rec_bar[0], 1);
+    mbar_init(&rec_bar[1], 1);
     fence_barrier_init();
   }
   __syncthreads();
@@ -239,52 +276,93 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
   grid_dependency_wait();
 
   // ================================================================ producer
+  // Per item k: the record (32-byte header) of item k + 1 is copied in while
+  // item k's stages are issued; the table entries of item k + 1 are loaded right
+  // after, while the ring is full of item k's data, so no round trip sits between
+  // two items.  Item indices are taken two ahead for the same reason.
   if (warp == NW) {
     const uint8_t* kbase = static_cast<const uint8_t*>(a.k);
     const uint8_t* vbase = static_cast<const uint8_t*>(a.v);
     const uint32_t n_items = *reinterpret_cast<volatile uint32_t*>(a.work + 1);
-    uint32_t stage_iter = 0;
+    const uint32_t Hkv = static_cast<uint32_t>(a.num_kv_heads);
+    int32_t* s_tab = reinterpret_cast<int32_t*>(smem + Tr::OFF_TAB);
+    auto rec_slot = [&](int r) { return reinterpret_cast<const int32_t*>(smem + Tr::OFF_REC + r * kRecordBytes); };
+    auto copy_record = [&](int r, uint32_t idx) {
+      mbar_arrive_expect_tx(&rec_bar[r], kRecordBytes);
+      bulk_load(smem + Tr::OFF_REC + r * kRecordBytes,
+                a.records + static_cast<int64_t>(idx / Hkv) * kRecordBytes, kRecordBytes, &rec_bar[r]);
+    };
+    // Table entries of the item described by record r into table buffer r.
+    auto load_table = [&](int r) {
+      if constexpr (PAGED) {
+        const int32_t* rec = rec_slot(r);
+        const int s = rec[0], t_begin = rec[3], n_tok = rec[4];
+        const int nb = (n_tok + B - 1) / B;
+        const int32_t* row = a.tables + static_cast<int64_t>(s) * a.max_blocks + t_begin / B;
+        for (int j = lane; j < nb; j += 32) {
+          int32_t f = __ldg(row + j);
+          if (f < 0 || f >= a.num_blocks) {
+            set_error(a.err, PKV_DEVERR_TABLE_ENTRY);
+            f = 0;
+          }
+          s_tab[r * Tr::MAX_TABLE + j] = f;
+        }
+      }
+    };
+    // record slot r holds items r, r + 2, ...: item j's copy completes phase j / 2
+    uint32_t rec_pending = 0, rec_parity = 0;  // bit r: unwaited copy in slot r / its parity
+    uint32_t idx_cur = 0, idx_nxt = 0;
     bool ok = true;
-    for (uint32_t item_iter = 0;; ++item_iter) {
-      uint32_t idx = 0;
-      if (lane == 0) idx = atomicAdd(a.work, 1u);
-      idx = __shfl_sync(0xffffffffu, idx, 0);
-      const int slot = item_iter % kItemSlots;
-      if (item_iter >= kItemSlots && lane == 0 &&
-          !mbar_wait_bounded(&item_empty[slot], ((item_iter / kItemSlots) - 1) & 1)) {
+    if (lane == 0) {
+      idx_cur = atomicAdd(a.work, 1u);
+      if (idx_cur < n_items) {
+        copy_record(0, idx_cur);
+        rec_pending = 1u;
+      }
+      idx_nxt = atomicAdd(a.work, 1u);
+    }
+    if (__shfl_sync(0xffffffffu, idx_cur, 0) < n_items) {
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&rec_bar[0], 0));
+      if (lane == 0) {
+        if (!ok) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+        rec_pending = 0;
+      }
+      if (ok) load_table(0);
+      __syncwarp();
+    }
+    uint32_t issued = 0, st = 0, ph = 0;  // stages issued; ring slot and use parity of the next
+    for (uint32_t k = 0; ok; ++k) {
+      const int slot = k & (kItemSlots - 1);
+      const int rs = k & 1;
+      const uint32_t cur = __shfl_sync(0xffffffffu, idx_cur, 0);
+      const uint32_t nxt = __shfl_sync(0xffffffffu, idx_nxt, 0);
+      if (lane == 0 && k >= kItemSlots &&
+          !mbar_wait_bounded(&item_empty[slot], ((k / kItemSlots) - 1) & 1)) {
         set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
         ok = false;
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      if (idx >= n_items) {
+      if (cur >= n_items) {
         if (lane == 0) {
           items[slot].s = -1;  // no more work
           mbar_arrive(&item_full[slot]);
         }
         break;
       }
-      const int2 it = __ldcg(a.items + idx / a.num_kv_heads);
-      const int kvh = idx % a.num_kv_heads;
-      const int s = it.x, part = it.y;
-      const int L = clamp_len(__ldg(a.lens + s), a.max_ctx);
-      int n_parts, psize;
-      partition_of(L, a.part_tokens, n_parts, psize);
-      const int t_begin = part * psize;
-      const int n_tok = min(L - t_begin, psize);  // 0 only when L == 0
-      if constexpr (PAGED) {
-        const int first_blk = t_begin / B;
-        const int n_blk = (n_tok + B - 1) / B;
-        const int32_t* row = a.tables + static_cast<int64_t>(s) * a.max_blocks + first_blk;
-        for (int j = lane; j < n_blk; j += 32) {
-          int32_t p = __ldg(row + j);
-          if (p < 0 || p >= a.num_blocks) {
-            set_error(a.err, PKV_DEVERR_TABLE_ENTRY);
-            p = 0;
-          }
-          s_table[j] = p;
+      uint32_t after = 0;
+      if (lane == 0) {
+        if (nxt < n_items) {
+          fence_proxy_async_smem();  // this record slot was last read two items ago
+          copy_record(rs ^ 1, nxt);
+          rec_pending |= 1u << (rs ^ 1);
+          rec_parity = (rec_parity & ~(1u << (rs ^ 1))) | ((((k + 1) >> 1) & 1u) << (rs ^ 1));
         }
+        after = atomicAdd(a.work, 1u);
       }
+      const int32_t* rec = rec_slot(rs);
+      const int s = rec[0], part = rec[1], n_parts = rec[2], t_begin = rec[3], n_tok = rec[4];
+      const int kvh = static_cast<int>(cur % Hkv);
       if (lane == 0) {
         ItemInfo& info = items[slot];
         info.s = s;
@@ -298,30 +376,24 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
                               (static_cast<int64_t>(s) * a.num_heads + kvh * G) * Tr::ROW_BYTES;
         bulk_load(smem + Tr::OFF_Q + slot * Tr::Q_BYTES, qsrc, Tr::Q_BYTES, &item_full[slot]);
       }
-      __syncwarp();
+      const int32_t* tab = s_tab + rs * Tr::MAX_TABLE;
       const int n_stages = (n_tok + TS - 1) / TS;
-      for (int i = 0; i < n_stages; ++i, ++stage_iter) {
-        const int st = stage_iter % STAGES;
-        if (lane == 0 && stage_iter >= STAGES &&
-            !mbar_wait_bounded(&empty[st], ((stage_iter / STAGES) - 1) & 1)) {
+      for (int i = 0; i < n_stages; ++i) {
+        if (lane == 0 && issued >= STAGES && !mbar_wait_bounded(&empty[st], ph ^ 1)) {
           set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
           ok = false;
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         const int t0 = i * TS;  // relative to the partition start (block aligned)
-        if (lane == 0) {
-          const int rows = min(TS, n_tok - t0);
-          mbar_arrive_expect_tx(&full[st], 2u * rows * Tr::ROW_BYTES);
-        }
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2u * min(TS, n_tok - t0) * Tr::ROW_BYTES);
         __syncwarp();
         const int tc = t0 + lane * Tr::CH;
         if (lane < Tr::NCH && tc < n_tok) {
           const uint32_t nbytes = min(Tr::CH, n_tok - tc) * Tr::ROW_BYTES;
           int64_t row;
           if constexpr (PAGED) {
-            const int64_t frame = s_table[tc / B];
-            row = (frame * a.num_kv_heads + kvh) * B + (t_begin + tc) % B;
+            row = (static_cast<int64_t>(tab[tc / B]) * a.num_kv_heads + kvh) * B + tc % B;
           } else {
             row = (static_cast<int64_t>(s) * a.num_kv_heads + kvh) * a.max_ctx + t_begin + tc;
           }
@@ -330,15 +402,37 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
           bulk_load(sk + Tr::TILE_BYTES, vbase + row * Tr::ROW_BYTES, nbytes, &full[st]);
         }
         __syncwarp();
+        ++issued;
+        if (++st == STAGES) {
+          st = 0;
+          ph ^= 1;
+        }
       }
       if (!ok) break;  // the consumers time out on their next wait and stop too
+      if (nxt < n_items) {
+        // next item's record has had all of this item to arrive; its table load
+        // overlaps the stages just issued
+        const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&rec_bar[rs ^ 1], ((k + 1) >> 1) & 1));
+        if (lane == 0) {
+          if (!got) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+          rec_pending &= ~(1u << (rs ^ 1));
+        }
+        if (!got) break;
+        load_table(rs ^ 1);
+        __syncwarp();
+      }
+      idx_cur = idx_nxt;
+      idx_nxt = after;
     }
     // Never leave the CTA with copies in flight: wait (bounded) until the last
-    // use of every stage has landed.
+    // use of every stage and any prefetched record have landed.
     if (lane == 0) {
-      const uint32_t first = stage_iter > STAGES ? stage_iter - STAGES : 0;
-      for (uint32_t i = first; i < stage_iter; ++i)
+      const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+      for (uint32_t i = first; i < issued; ++i)
         if (!mbar_wait_bounded(&full[i % STAGES], (i / STAGES) & 1))
+          set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+      for (int r = 0; r < 2; ++r)
+        if (((rec_pending >> r) & 1u) && !mbar_wait_bounded(&rec_bar[r], (rec_parity >> r) & 1u))
           set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
     }
     return;
@@ -353,11 +447,11 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
   const bool p_writer = (li % LPH) == 0;
   const int w_tok0 = warp * TPW;
   float2* p_warp = s_p + warp * TPW * G;
-  uint32_t stage_iter = 0;
+  uint32_t st = 0, ph = 0;  // ring slot and use parity of the next stage
 
-  for (uint32_t item_iter = 0;; ++item_iter) {
-    const int slot = item_iter % kItemSlots;
-    const bool arrived = mbar_wait_bounded(&item_full[slot], (item_iter / kItemSlots) & 1);
+  for (uint32_t k = 0;; ++k) {
+    const int slot = k & (kItemSlots - 1);
+    const bool arrived = mbar_wait_bounded(&item_full[slot], (k / kItemSlots) & 1);
     if (!arrived && lane == 0) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
     const ItemInfo info = items[slot];
     if (named_barrier_or(1, NW * 32, !arrived || info.s < 0)) break;
@@ -391,22 +485,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
-      for (int k = 0; k < DPL / 2; ++k) acc[g][k] = make_float2(0.f, 0.f);
+      for (int kk = 0; kk < DPL / 2; ++kk) acc[g][kk] = make_float2(0.f, 0.f);
 
-    const int n_stages = (info.n_tok + TS - 1) / TS;
-    bool ok = true;
-    for (int i = 0; i < n_stages; ++i, ++stage_iter) {
-      const int st = stage_iter % STAGES;
-      if (!mbar_wait_bounded(&full[st], (stage_iter / STAGES) & 1)) {
-        if (lane == 0) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
-        ok = false;
-        break;
-      }
-      const T* sK = reinterpret_cast<const T*>(smem + st * Tr::STAGE_BYTES);
-      const T* sV = sK + TS * D;
-      const int nv = min(TS, info.n_tok - i * TS);
-
-      // ---- scores: every lane ends with the score of head my_h of its token
+    // One stage: scores of this warp's TPW tokens, online softmax, PV.  FULL
+    // stages (all TS tokens valid) skip the masking and the early exits.
+    auto stage = [&](const T* sK, const T* sV, int nv, auto full_tag) {
+      constexpr bool FULL = decltype(full_tag)::value;
       float sc[ROUNDS];
 #pragma unroll
       for (int r = 0; r < ROUNDS; ++r) {
@@ -443,10 +527,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
         // the lanes of one head's group finish with a plain reduction
 #pragma unroll
         for (int m = LPH / 2; m > 0; m >>= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], m);
-        sc[r] = tok < nv ? x[0] : -CUDART_INF_F;
+        if constexpr (FULL)
+          sc[r] = x[0];
+        else
+          sc[r] = tok < nv ? x[0] : -CUDART_INF_F;
       }
 
-      // ---- online softmax for head my_h
+      // online softmax for head my_h
       float mx = sc[0];
 #pragma unroll
       for (int r = 1; r < ROUNDS; ++r) mx = fmaxf(mx, sc[r]);
@@ -461,13 +548,17 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
           const float ag = __shfl_sync(0xffffffffu, alpha, g * LPH);
           const float2 a2 = make_float2(ag, ag);
 #pragma unroll
-          for (int k = 0; k < DPL / 2; ++k) acc[g][k] = fmul2(acc[g][k], a2);
+          for (int kk = 0; kk < DPL / 2; ++kk) acc[g][kk] = fmul2(acc[g][kk], a2);
         }
         m_run = m_new;
       }
 #pragma unroll
       for (int r = 0; r < ROUNDS; ++r) {
-        const float p = sc[r] == -CUDART_INF_F ? 0.f : fast_exp2(sc[r] - m_run);
+        float p;
+        if constexpr (FULL)
+          p = fast_exp2(sc[r] - m_run);
+        else
+          p = sc[r] == -CUDART_INF_F ? 0.f : fast_exp2(sc[r] - m_run);
         if (p_writer) {
           p_warp[(r * TPR + tg) * G + my_h] = make_float2(p, p);
           l_lane += p;
@@ -475,10 +566,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
       }
       __syncwarp();
 
-      // ---- PV over this warp's valid tokens
+      // PV over this warp's valid tokens
 #pragma unroll
       for (int j = 0; j < TPW; ++j) {
-        if (w_tok0 + j >= nv) break;
+        if constexpr (!FULL) {
+          if (w_tok0 + j >= nv) break;
+        }
         float2 pj[G];
         if constexpr (G % 2 == 0) {
 #pragma unroll
@@ -502,10 +595,31 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-          for (int k = 0; k < DPL / 2; ++k) acc[g][k] = ffma2(pj[g], vf[k], acc[g][k]);
+          for (int kk = 0; kk < DPL / 2; ++kk) acc[g][kk] = ffma2(pj[g], vf[kk], acc[g][kk]);
       }
+    };
+
+    const int n_stages = (info.n_tok + TS - 1) / TS;
+    bool ok = true;
+    for (int i = 0; i < n_stages; ++i) {
+      if (!mbar_wait_bounded(&full[st], ph)) {
+        if (lane == 0) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+        ok = false;
+        break;
+      }
+      const T* sK = reinterpret_cast<const T*>(smem + st * Tr::STAGE_BYTES);
+      const T* sV = sK + TS * D;
+      const int nv = info.n_tok - i * TS;
+      if (nv >= TS)
+        stage(sK, sV, TS, std::true_type{});
+      else
+        stage(sK, sV, nv, std::false_type{});
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
+      if (++st == STAGES) {
+        st = 0;
+        ph ^= 1;
+      }
     }
 
     // ---- merge the four warps of this item
@@ -542,70 +656,116 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeArgs
             from_float<T>(lsum > 0.f ? o / lsum : 0.f);
       } else {
         const int64_t cell = (static_cast<int64_t>(s) * a.num_heads + h0 + g) * a.max_parts + info.part;
-        __stcg(a.tmp_out + cell * D + d, o / lsum);
+        a.tmp_out[cell * D + d] = o / lsum;
         if (d == 0) {
-          __stcg(a.tmp_m + cell, M);
-          __stcg(a.tmp_l + cell, lsum);
+          a.tmp_m[cell] = M;
+          a.tmp_l[cell] = lsum;
         }
       }
     }
-    if (!single) __threadfence();
     named_barrier_sync(1, NW * 32);  // s_acc, s_m, s_l are free again
-    if (single) continue;
+  }
+}
 
-    if (threadIdx.x == 0) {
-      const uint32_t done = atomicAdd(a.merge_cnt + s * a.num_kv_heads + info.kvh, 1u);
-      *s_flag = (done == static_cast<uint32_t>(info.n_parts - 1));
+// ---------------------------------------------------------------- merge
+// Contexts that span several partitions: out = sum_p w_p o_p with
+// w_p = l_p 2^(m_p - M) / sum_q l_q 2^(m_q - M), M = max_p m_p, summed in
+// partition order.  One CTA of 128 threads per (sequence, kv head) pair listed
+// by the plan kernel (grid-stride when there are more pairs than CTAs).  The
+// outputs of the first kPre partitions are loaded into registers up front, so
+// with up to kPre partitions a pair costs about one memory round trip.
+// Launched behind the decode grid (programmatic dependent launch): it waits for
+// the whole decode grid before reading its results.
+constexpr int kMergeThreads = 128;
+constexpr int kMergeStat = 64;  // partitions per statistics round
+constexpr int kPre = 8;         // partitions per output round
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a) {
+  __shared__ float s_m[G][kMergeStat], s_l[G][kMergeStat], s_w[G][kPre];
+  __shared__ float s_M[G], s_L[G];
+  grid_dependency_wait();
+  constexpr int kPer = (G * D + kMergeThreads - 1) / kMergeThreads;
+  const uint32_t Hkv = static_cast<uint32_t>(a.num_kv_heads);
+  const uint32_t n_tasks = a.work[2] * Hkv;
+  for (uint32_t t = blockIdx.x; t < n_tasks; t += gridDim.x) {
+    const int s = a.merge_seqs[t / Hkv];
+    const int h0 = static_cast<int>(t % Hkv) * G;
+    int np, psize;
+    partition_of(clamp_len(a.lens[s], a.max_ctx), a.part_tokens, np, psize);
+    const int64_t base0 = (static_cast<int64_t>(s) * a.num_heads + h0) * a.max_parts;
+    auto cell = [&](int g, int p) { return base0 + static_cast<int64_t>(g) * a.max_parts + p; };
+
+    float pre[kPre][kPer];  // outputs of partitions 0 .. kPre-1
+#pragma unroll
+    for (int p = 0; p < kPre; ++p)
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int idx = threadIdx.x + k * kMergeThreads;
+        pre[p][k] = (p < np && idx < G * D) ? a.tmp_out[cell(idx / D, p) * D + idx % D] : 0.f;
+      }
+
+    // M and the normaliser per head, online over rounds of kMergeStat partitions
+    if (threadIdx.x < G) {
+      s_M[threadIdx.x] = -CUDART_INF_F;
+      s_L[threadIdx.x] = 0.f;
     }
-    named_barrier_sync(1, NW * 32);
-    if (!*s_flag) continue;
+    for (int c0 = 0; c0 < np; c0 += kMergeStat) {
+      const int cn = min(kMergeStat, np - c0);
+      for (int i = threadIdx.x; i < G * cn; i += kMergeThreads) {
+        const int g = i / cn, p = i % cn;
+        s_m[g][p] = a.tmp_m[cell(g, c0 + p)];
+        s_l[g][p] = a.tmp_l[cell(g, c0 + p)];
+      }
+      __syncthreads();
+      if (threadIdx.x < G) {
+        const int g = threadIdx.x;
+        float M = s_M[g];
+        for (int p = 0; p < cn; ++p) M = fmaxf(M, s_m[g][p]);
+        float L = s_L[g] * fast_exp2(s_M[g] - M);  // 0 on the first round
+        for (int p = 0; p < cn; ++p) L += s_l[g][p] * fast_exp2(s_m[g][p] - M);
+        s_M[g] = M;
+        s_L[g] = L;
+      }
+      __syncthreads();
+    }
 
-    // Last partition of this (sequence, kv head) to finish: merge all partitions,
-    // out = sum_p w_p o_p with w_p = l_p 2^(m_p - M) / sum_q l_q 2^(m_q - M), in
-    // partition order.
-    __threadfence();
-    constexpr int kChunk = NW * D;  // partitions per pass; s_acc holds G * kChunk weights
-    constexpr int kPer = (G * D + NW * 32 - 1) / (NW * 32);
-    const int np = info.n_parts;
     float o_reg[kPer];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) o_reg[k] = 0.f;
-    float* s_w = s_acc;
-    for (int p0 = 0; p0 < np; p0 += kChunk) {
-      const int pc = min(kChunk, np - p0);
-      for (int g = warp; g < G; g += NW) {
-        const int64_t base = (static_cast<int64_t>(s) * a.num_heads + h0 + g) * a.max_parts;
-        float M = -CUDART_INF_F;
-        for (int p = lane; p < np; p += 32) M = fmaxf(M, __ldcg(a.tmp_m + base + p));
-#pragma unroll
-        for (int m = 16; m > 0; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-        float lsum = 0.f;
-        for (int p = lane; p < np; p += 32)
-          lsum += __ldcg(a.tmp_l + base + p) * fast_exp2(__ldcg(a.tmp_m + base + p) - M);
-#pragma unroll
-        for (int m = 16; m > 0; m >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, m);
-        const float inv = 1.f / lsum;
-        for (int p = lane; p < pc; p += 32)
-          s_w[g * kChunk + p] =
-              __ldcg(a.tmp_l + base + p0 + p) * fast_exp2(__ldcg(a.tmp_m + base + p0 + p) - M) * inv;
+    for (int p0 = 0; p0 < np; p0 += kPre) {
+      const int pc = min(kPre, np - p0);
+      if (threadIdx.x < G * pc) {
+        const int g = threadIdx.x / pc, p = threadIdx.x % pc;
+        s_w[g][p] = a.tmp_l[cell(g, p0 + p)] * fast_exp2(a.tmp_m[cell(g, p0 + p)] - s_M[g]) / s_L[g];
       }
-      named_barrier_sync(1, NW * 32);
+      if (p0 > 0) {
+#pragma unroll
+        for (int p = 0; p < kPre; ++p)
+#pragma unroll
+          for (int k = 0; k < kPer; ++k) {
+            const int idx = threadIdx.x + k * kMergeThreads;
+            pre[p][k] = (p < pc && idx < G * D) ? a.tmp_out[cell(idx / D, p0 + p) * D + idx % D] : 0.f;
+          }
+      }
+      __syncthreads();
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
-        const int idx = threadIdx.x + k * NW * 32;
+        const int idx = threadIdx.x + k * kMergeThreads;
         if (idx < G * D) {
-          const int g = idx / D, d = idx % D;
-          const int64_t base = (static_cast<int64_t>(s) * a.num_heads + h0 + g) * a.max_parts + p0;
+          const int g = idx / D;
           float o = o_reg[k];
-          for (int p = 0; p < pc; ++p) o += s_w[g * kChunk + p] * __ldcg(a.tmp_out + (base + p) * D + d);
+#pragma unroll
+          for (int p = 0; p < kPre; ++p)
+            if (p < pc) o += s_w[g][p] * pre[p][k];
           o_reg[k] = o;
         }
       }
-      named_barrier_sync(1, NW * 32);
+      __syncthreads();
     }
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
-      const int idx = threadIdx.x + k * NW * 32;
+      const int idx = threadIdx.x + k * kMergeThreads;
       if (idx < G * D) {
         const int g = idx / D, d = idx % D;
         static_cast<T*>(a.out)[(static_cast<int64_t>(s) * a.num_heads + h0 + g) * D + d] =

@@ -36,22 +36,36 @@ cudaError_t launch_decode_one(const DecodeArgs& a, int num_sms, cudaStream_t str
   int grid = 0;
   cudaError_t e = decode_grid<T, D, G, B, PAGED>(num_sms, &grid);
   if (e != cudaSuccess) return e;
-  plan_kernel<<<1, kPlanThreads, 0, stream>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // Programmatic dependent launch: the decode CTAs may start (and set up their
-  // barriers) while the plan kernel finishes; they wait for it in-kernel.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kDecodeThreads);
-  cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
-  cfg.stream = stream;
+  // Programmatic dependent launch for all three kernels: each may start (and
+  // set up) while its predecessor finishes, and waits for it in-kernel before
+  // touching anything the predecessor writes.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kPlanThreads);
+  cfg.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&cfg, plan_kernel, a);
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
   e = cudaLaunchKernelEx(&cfg, decode_kernel<T, D, G, B, PAGED>, a);
+  if (e != cudaSuccess) return e;
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.max_parts <= 1) return e;
+  // Partition merge, also behind its predecessor: its CTAs start as decode CTAs
+  // retire and wait in-kernel for the whole decode grid.
+  const int64_t pairs = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
+  const int64_t want = static_cast<int64_t>(num_sms) * 16;  // one wave of 128-thread CTAs
+  cfg.gridDim = dim3(static_cast<unsigned>(pairs < want ? pairs : want));
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&cfg, merge_kernel<T, D, G>, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

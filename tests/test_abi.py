@@ -37,7 +37,8 @@ def test_status_strings():
 def _layout_bytes(S, Hq, D, ctx, part=512):
     r = lambda x: (x + 255) // 256 * 256
     P = max(1, -(-ctx // part))
-    return 256 + r(4 * S * Hq) + r(8 * S * P) + (r(S * Hq * P * (D + 2) * 4) if P > 1 else 0)
+    rec = 32
+    return 256 + r(4 * S) + r(S * P * rec) + (r(S * Hq * P * (D + 2) * 4) if P > 1 else 0)
 
 
 def test_workspace_bytes_formula():
