@@ -101,9 +101,9 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t h
  *   block_tables device int32 [num_seqs, max_blocks_per_seq]; only the first
  *                ceil(context_lens[s] / block_size) entries of row s are read
  *   context_lens device int32 [num_seqs], 0 <= context_lens[s] <= max_blocks_per_seq * block_size
- *   partition_size maximum tokens per context partition (0 = 512); a multiple of 32
- *                in [32, 4096].  A context of L tokens is split into ceil(L / partition_size)
- *                near-equal partitions (multiples of 32 tokens) that run on different
+ *   partition_size maximum tokens per context partition (0 = 512); a multiple of 64
+ *                in [64, 2048].  A context of L tokens is split into ceil(L / partition_size)
+ *                near-equal partitions (multiples of 64 tokens) that run on different
  *                CTAs and are merged with a log-sum-exp in the same launch sequence.
  *   workspace    device scratch of pkv_decode_workspace_bytes(num_seqs, num_heads,
  *                head_dim, max_blocks_per_seq * block_size, partition_size) bytes,

@@ -60,7 +60,7 @@ int resolve_partition(int32_t partition_size) {
   return partition_size == 0 ? kDefaultPartition : partition_size;
 }
 
-bool valid_partition(int p) { return p >= 32 && p <= kMaxPartTokens && p % 32 == 0; }
+bool valid_partition(int p) { return p >= kStageTokens && p <= kMaxPartTokens && p % kStageTokens == 0; }
 
 int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
 

@@ -72,15 +72,18 @@ struct DecodeArgs {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
-constexpr int kMaxPartTokens = 4096;
+constexpr int kMaxPartTokens = 2048;
 constexpr int kPlanThreads = 1024;
 constexpr int kItemSlots = 2;
+constexpr int kRecSlots = 4;   // records of items k .. k+3 (copied two items ahead)
+constexpr int kStageTokens = 64;
 // Work record of one (sequence, partition): int32 s, part, n_parts, t_begin,
 // n_tok, L, 0, 0.
 constexpr int kRecordBytes = 32;
 
 // Partitioning of a context of L tokens (L already clamped to [0, max_ctx]):
-// n partitions of `size` tokens (a multiple of 32), the last one shorter.
+// n partitions of `size` tokens (a multiple of the 64-token stage), the last
+// one shorter.  part_tokens is a multiple of 64, so size <= part_tokens.
 __device__ __forceinline__ void partition_of(int L, int part_tokens, int& n, int& size) {
   if (L <= 0) {
     n = 1;
@@ -88,7 +91,7 @@ __device__ __forceinline__ void partition_of(int L, int part_tokens, int& n, int
     return;
   }
   const int n0 = (L + part_tokens - 1) / part_tokens;
-  size = ((L + n0 - 1) / n0 + 31) & ~31;
+  size = ((L + n0 - 1) / n0 + kStageTokens - 1) & ~(kStageTokens - 1);
   n = (L + size - 1) / size;
 }
 
@@ -107,12 +110,12 @@ struct DecodeTraits {
   static constexpr int EPL = D / LPT;                     // row elements per lane (scores)
   static constexpr int VPL = EPL / 8;                     // 16-byte vectors per lane (scores)
   static constexpr int TPR = 32 / LPT;                    // tokens per warp round
-  static constexpr int TPW = 8;                           // tokens per warp per stage
+  static constexpr int TPW = kStageTokens / kConsumerWarps;  // tokens per warp per stage
   static constexpr int ROUNDS = TPW / TPR;
   static constexpr int TS = kConsumerWarps * TPW;         // tokens per stage
   static constexpr int CH = PAGED ? (B < TS ? B : TS) : TS;  // tokens per bulk copy
   static constexpr int NCH = TS / CH;
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = 2;
   static constexpr int DPL = D / 32;                      // output dims per lane (PV)
   static constexpr int ROW_BYTES = D * 2;
   static constexpr int TILE_BYTES = TS * ROW_BYTES;
@@ -121,22 +124,26 @@ struct DecodeTraits {
   static constexpr int MAX_TABLE = PAGED ? kMaxPartTokens / B : 4;  // table entries of one item
   // shared memory carve-up (bytes, 16-byte aligned pieces)
   static constexpr int OFF_Q = STAGES * STAGE_BYTES;
-  static constexpr int OFF_ACC = OFF_Q + kItemSlots * Q_BYTES;          // [warps][G][D] f32
-  static constexpr int OFF_P = OFF_ACC + kConsumerWarps * G * D * 4;    // [warps][TPW][G] (p, p)
-  static constexpr int OFF_REC = OFF_P + kConsumerWarps * TPW * G * 8;  // 2 record slots
-  static constexpr int OFF_TAB = OFF_REC + 2 * kRecordBytes;            // 2 table buffers
+  static constexpr int HG = G > 1 ? G / 2 : 1;                          // heads per merge round
+  static constexpr int OFF_ACC = OFF_Q + kItemSlots * Q_BYTES;          // [warps][HG][D] f32
+  static constexpr int OFF_P = OFF_ACC + kConsumerWarps * HG * D * 4;   // [warps][TPW][G] (p, p)
+  static constexpr int OFF_REC = OFF_P + kConsumerWarps * TPW * G * 8;  // record slots
+  static constexpr int OFF_TAB = OFF_REC + kRecSlots * kRecordBytes;    // 2 table buffers
   static constexpr int OFF_STAT = OFF_TAB + 2 * MAX_TABLE * 4;          // m, l per warp and head
   static constexpr int OFF_ITEM = OFF_STAT + 2 * kConsumerWarps * G * 4 + 16;
   static constexpr int OFF_BARS = OFF_ITEM + kItemSlots * 32;
-  static constexpr int SMEM_BYTES = OFF_BARS + (2 * STAGES + 2 * kItemSlots + 2) * 8;
+  static constexpr int SMEM_BYTES = OFF_BARS + (2 * STAGES + 2 * kItemSlots + kRecSlots + 2) * 8;
 
   static_assert(D % 64 == 0, "head_dim must be 64 or 128");
   static_assert(EPL % 8 == 0 && VPL >= 1, "score vectors are 16 bytes");
   static_assert(G <= LPT && LPT % G == 0, "reduce-scatter leaves one head per lane group");
   static_assert(TPW % TPR == 0, "whole rounds per stage");
+  static_assert(TS == kStageTokens, "stage = partition granule");
   static_assert(TS % CH == 0 && NCH <= 32, "whole copies per stage, one lane each");
   static_assert(DPL == 2 || DPL == 4, "PV reads 4 or 8 bytes per lane");
   static_assert(OFF_BARS % 8 == 0 && OFF_STAT % 16 == 0, "alignment");
+  // three CTAs per SM (228 KB of shared memory, 1 KB reserved per CTA) up to G = 4
+  static_assert(G > 4 || 3 * (SMEM_BYTES + 1024) <= 228 * 1024, "3 CTAs per SM");
 };
 
 // Item slot handed from the producer to the consumers.
@@ -248,7 +255,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
   uint64_t* empty = full + STAGES;
   uint64_t* item_full = empty + STAGES;
   uint64_t* item_empty = item_full + kItemSlots;
-  uint64_t* rec_bar = item_empty + kItemSlots;
+  uint64_t* rec_bar = item_empty + kItemSlots;  // [kRecSlots]
+  uint64_t* tab_bar = rec_bar + kRecSlots;       // [2]
   ItemInfo* items = reinterpret_cast<ItemInfo*>(smem + Tr::OFF_ITEM);
   float* s_acc = reinterpret_cast<float*>(smem + Tr::OFF_ACC);
   float2* s_p = reinterpret_cast<float2*>(smem + Tr::OFF_P);
@@ -267,8 +275,9 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
       mbar_init(&item_full[i], 1);
       mbar_init(&item_empty[i], NW);
     }
-    mbar_init(&rec_bar[0], 1);
-    mbar_init(&rec_bar[1], 1);
+    for (int i = 0; i < kRecSlots; ++i) mbar_init(&rec_bar[i], 1);
+    mbar_init(&tab_bar[0], 32);  // one asynchronous arrival per producer lane
+    mbar_init(&tab_bar[1], 32);
     fence_barrier_init();
   }
   __syncthreads();
@@ -276,66 +285,83 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
   grid_dependency_wait();
 
   // ================================================================ producer
-  // Per item k: the record (32-byte header) of item k + 1 is copied in while
-  // item k's stages are issued; the table entries of item k + 1 are loaded right
-  // after, while the ring is full of item k's data, so no round trip sits between
-  // two items.  Item indices are taken two ahead for the same reason.
+  // Item j (the j-th item this CTA takes): its index is taken three items ahead,
+  // its 32-byte record is bulk-copied two items ahead into record slot j % 4, and
+  // its block-table entries are fetched one item ahead with cp.async into table
+  // buffer j % 2.  So while item k's stages are issued, nothing the producer
+  // waits for was requested less than one item ago.
   if (warp == NW) {
     const uint8_t* kbase = static_cast<const uint8_t*>(a.k);
     const uint8_t* vbase = static_cast<const uint8_t*>(a.v);
     const uint32_t n_items = *reinterpret_cast<volatile uint32_t*>(a.work + 1);
     const uint32_t Hkv = static_cast<uint32_t>(a.num_kv_heads);
     int32_t* s_tab = reinterpret_cast<int32_t*>(smem + Tr::OFF_TAB);
-    auto rec_slot = [&](int r) { return reinterpret_cast<const int32_t*>(smem + Tr::OFF_REC + r * kRecordBytes); };
-    auto copy_record = [&](int r, uint32_t idx) {
+    auto rec_slot = [&](uint32_t j) {
+      return reinterpret_cast<const int32_t*>(smem + Tr::OFF_REC + (j % kRecSlots) * kRecordBytes);
+    };
+    // Outstanding copies nobody waited for yet (error exits drain them): bit r of
+    // rec_pending / rec_parity = record slot r and the parity of its open phase;
+    // likewise for the two table buffers.
+    uint32_t rec_pending = 0, rec_parity = 0, tab_pending = 0, tab_parity = 0;
+    auto copy_record = [&](uint32_t j, uint32_t idx) {  // lane 0
+      const uint32_t r = j % kRecSlots;
       mbar_arrive_expect_tx(&rec_bar[r], kRecordBytes);
       bulk_load(smem + Tr::OFF_REC + r * kRecordBytes,
                 a.records + static_cast<int64_t>(idx / Hkv) * kRecordBytes, kRecordBytes, &rec_bar[r]);
+      rec_pending |= 1u << r;
+      rec_parity = (rec_parity & ~(1u << r)) | (((j / kRecSlots) & 1u) << r);
     };
-    // Table entries of the item described by record r into table buffer r.
-    auto load_table = [&](int r) {
+    // Every lane waits for record j (all lanes read it).
+    auto wait_record = [&](uint32_t j) {
+      const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&rec_bar[j % kRecSlots], (j / kRecSlots) & 1));
+      if (lane == 0) {
+        if (!got) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+        rec_pending &= ~(1u << (j % kRecSlots));
+      }
+      return got;
+    };
+    // Block-table entries of item j (its record has landed) into buffer j % 2.
+    auto fetch_table = [&](uint32_t j) {
       if constexpr (PAGED) {
-        const int32_t* rec = rec_slot(r);
+        const int32_t* rec = rec_slot(j);
         const int s = rec[0], t_begin = rec[3], n_tok = rec[4];
         const int nb = (n_tok + B - 1) / B;
         const int32_t* row = a.tables + static_cast<int64_t>(s) * a.max_blocks + t_begin / B;
-        for (int j = lane; j < nb; j += 32) {
-          int32_t f = __ldg(row + j);
-          if (f < 0 || f >= a.num_blocks) {
-            set_error(a.err, PKV_DEVERR_TABLE_ENTRY);
-            f = 0;
-          }
-          s_tab[r * Tr::MAX_TABLE + j] = f;
-        }
+        int32_t* dst = s_tab + (j & 1) * Tr::MAX_TABLE;
+        for (int e = lane; e < nb; e += 32) cp_async_4(dst + e, row + e);
+        cp_async_arrive_noinc(&tab_bar[j & 1]);
+        tab_pending |= 1u << (j & 1);
+        tab_parity = (tab_parity & ~(1u << (j & 1))) | (((j >> 1) & 1u) << (j & 1));
       }
     };
-    // record slot r holds items r, r + 2, ...: item j's copy completes phase j / 2
-    uint32_t rec_pending = 0, rec_parity = 0;  // bit r: unwaited copy in slot r / its parity
-    uint32_t idx_cur = 0, idx_nxt = 0;
+    auto wait_table = [&](uint32_t j) {
+      if constexpr (PAGED) {
+        const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&tab_bar[j & 1], (j >> 1) & 1));
+        if (!got && lane == 0) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+        tab_pending &= ~(1u << (j & 1));
+        return got;
+      }
+      return true;
+    };
+
+    uint32_t idx0 = 0, idx1 = 0, idx2 = 0;  // items k, k + 1, k + 2 (lane 0)
     bool ok = true;
     if (lane == 0) {
-      idx_cur = atomicAdd(a.work, 1u);
-      if (idx_cur < n_items) {
-        copy_record(0, idx_cur);
-        rec_pending = 1u;
-      }
-      idx_nxt = atomicAdd(a.work, 1u);
+      idx0 = atomicAdd(a.work, 1u);
+      idx1 = atomicAdd(a.work, 1u);
+      idx2 = atomicAdd(a.work, 1u);
+      if (idx0 < n_items) copy_record(0, idx0);
+      if (idx1 < n_items) copy_record(1, idx1);
     }
-    if (__shfl_sync(0xffffffffu, idx_cur, 0) < n_items) {
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&rec_bar[0], 0));
-      if (lane == 0) {
-        if (!ok) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
-        rec_pending = 0;
-      }
-      if (ok) load_table(0);
-      __syncwarp();
+    if (__shfl_sync(0xffffffffu, idx0, 0) < n_items) {
+      ok = wait_record(0);
+      if (ok) fetch_table(0);
     }
     uint32_t issued = 0, st = 0, ph = 0;  // stages issued; ring slot and use parity of the next
     for (uint32_t k = 0; ok; ++k) {
       const int slot = k & (kItemSlots - 1);
-      const int rs = k & 1;
-      const uint32_t cur = __shfl_sync(0xffffffffu, idx_cur, 0);
-      const uint32_t nxt = __shfl_sync(0xffffffffu, idx_nxt, 0);
+      const uint32_t cur = __shfl_sync(0xffffffffu, idx0, 0);
+      const uint32_t nx1 = __shfl_sync(0xffffffffu, idx1, 0);
       if (lane == 0 && k >= kItemSlots &&
           !mbar_wait_bounded(&item_empty[slot], ((k / kItemSlots) - 1) & 1)) {
         set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
@@ -350,17 +376,21 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
         }
         break;
       }
-      uint32_t after = 0;
+      uint32_t idx3 = 0;
       if (lane == 0) {
-        if (nxt < n_items) {
+        if (idx2 < n_items) {
           fence_proxy_async_smem();  // this record slot was last read two items ago
-          copy_record(rs ^ 1, nxt);
-          rec_pending |= 1u << (rs ^ 1);
-          rec_parity = (rec_parity & ~(1u << (rs ^ 1))) | ((((k + 1) >> 1) & 1u) << (rs ^ 1));
+          copy_record(k + 2, idx2);
         }
-        after = atomicAdd(a.work, 1u);
+        idx3 = atomicAdd(a.work, 1u);
       }
-      const int32_t* rec = rec_slot(rs);
+      if (nx1 < n_items) {
+        // record k + 1 was requested one item ago; fetch its table now
+        if (!wait_record(k + 1)) break;
+        fetch_table(k + 1);
+      }
+      if (!wait_table(k)) break;  // requested one item ago
+      const int32_t* rec = rec_slot(k);
       const int s = rec[0], part = rec[1], n_parts = rec[2], t_begin = rec[3], n_tok = rec[4];
       const int kvh = static_cast<int>(cur % Hkv);
       if (lane == 0) {
@@ -376,7 +406,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
                               (static_cast<int64_t>(s) * a.num_heads + kvh * G) * Tr::ROW_BYTES;
         bulk_load(smem + Tr::OFF_Q + slot * Tr::Q_BYTES, qsrc, Tr::Q_BYTES, &item_full[slot]);
       }
-      const int32_t* tab = s_tab + rs * Tr::MAX_TABLE;
+      const int32_t* tab = s_tab + (k & 1) * Tr::MAX_TABLE;
       const int n_stages = (n_tok + TS - 1) / TS;
       for (int i = 0; i < n_stages; ++i) {
         if (lane == 0 && issued >= STAGES && !mbar_wait_bounded(&empty[st], ph ^ 1)) {
@@ -393,7 +423,12 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
           const uint32_t nbytes = min(Tr::CH, n_tok - tc) * Tr::ROW_BYTES;
           int64_t row;
           if constexpr (PAGED) {
-            row = (static_cast<int64_t>(tab[tc / B]) * a.num_kv_heads + kvh) * B + tc % B;
+            int32_t f = tab[tc / B];
+            if (f < 0 || f >= a.num_blocks) {
+              set_error(a.err, PKV_DEVERR_TABLE_ENTRY);
+              f = 0;
+            }
+            row = (static_cast<int64_t>(f) * a.num_kv_heads + kvh) * B + tc % B;
           } else {
             row = (static_cast<int64_t>(s) * a.num_kv_heads + kvh) * a.max_ctx + t_begin + tc;
           }
@@ -409,32 +444,26 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
         }
       }
       if (!ok) break;  // the consumers time out on their next wait and stop too
-      if (nxt < n_items) {
-        // next item's record has had all of this item to arrive; its table load
-        // overlaps the stages just issued
-        const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&rec_bar[rs ^ 1], ((k + 1) >> 1) & 1));
-        if (lane == 0) {
-          if (!got) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
-          rec_pending &= ~(1u << (rs ^ 1));
-        }
-        if (!got) break;
-        load_table(rs ^ 1);
-        __syncwarp();
-      }
-      idx_cur = idx_nxt;
-      idx_nxt = after;
+      idx0 = idx1;
+      idx1 = idx2;
+      idx2 = idx3;
     }
     // Never leave the CTA with copies in flight: wait (bounded) until the last
-    // use of every stage and any prefetched record have landed.
+    // use of every stage, and every record and table copy, have landed.
     if (lane == 0) {
       const uint32_t first = issued > STAGES ? issued - STAGES : 0;
       for (uint32_t i = first; i < issued; ++i)
         if (!mbar_wait_bounded(&full[i % STAGES], (i / STAGES) & 1))
           set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
-      for (int r = 0; r < 2; ++r)
-        if (((rec_pending >> r) & 1u) && !mbar_wait_bounded(&rec_bar[r], (rec_parity >> r) & 1u))
-          set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
     }
+    for (int r = 0; r < kRecSlots; ++r)
+      if (lane == 0 && ((rec_pending >> r) & 1u) &&
+          !mbar_wait_bounded(&rec_bar[r], (rec_parity >> r) & 1u))
+        set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+    for (int b = 0; b < 2; ++b)
+      if (((tab_pending >> b) & 1u) && !mbar_wait_bounded(&tab_bar[b], (tab_parity >> b) & 1u) &&
+          lane == 0)
+        set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
     return;
   }
 
@@ -622,14 +651,9 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
       }
     }
 
-    // ---- merge the four warps of this item
+    // ---- merge the four warps of this item, HG heads per round
 #pragma unroll
     for (int m = LPT; m < 32; m <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, m);
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int k = 0; k < DPL / 2; ++k)
-        *reinterpret_cast<float2*>(s_acc + (warp * G + g) * D + lane * DPL + 2 * k) = acc[g][k];
     if (tg == 0 && p_writer) {
       s_m[warp * G + my_h] = m_run;
       s_l[warp * G + my_h] = l_lane;
@@ -638,28 +662,40 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
 
     const int s = info.s;
     const bool single = info.n_parts == 1;
-    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
-      const int g = idx / D, d = idx % D;
-      float M = -CUDART_INF_F;
+    constexpr int HG = Tr::HG;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * G + g]);
-      float lsum = 0.f, o = 0.f;
+    for (int r = 0; r < G / HG; ++r) {
+      if (r > 0) named_barrier_sync(1, NW * 32);  // previous round's reads are done
 #pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        const float mw = s_m[w * G + g];
-        const float f = mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M);
-        lsum += f * s_l[w * G + g];
-        o += f * s_acc[(w * G + g) * D + d];
-      }
-      if (single) {
-        static_cast<T*>(a.out)[(static_cast<int64_t>(s) * a.num_heads + h0 + g) * D + d] =
-            from_float<T>(lsum > 0.f ? o / lsum : 0.f);
-      } else {
-        const int64_t cell = (static_cast<int64_t>(s) * a.num_heads + h0 + g) * a.max_parts + info.part;
-        a.tmp_out[cell * D + d] = o / lsum;
-        if (d == 0) {
-          a.tmp_m[cell] = M;
-          a.tmp_l[cell] = lsum;
+      for (int gg = 0; gg < HG; ++gg)
+#pragma unroll
+        for (int kk = 0; kk < DPL / 2; ++kk)
+          *reinterpret_cast<float2*>(s_acc + (warp * HG + gg) * D + lane * DPL + 2 * kk) = acc[r * HG + gg][kk];
+      named_barrier_sync(1, NW * 32);
+      for (int idx = threadIdx.x; idx < HG * D; idx += NW * 32) {
+        const int gg = idx / D, d = idx % D;
+        const int g = r * HG + gg;
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * G + g]);
+        float lsum = 0.f, o = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const float mw = s_m[w * G + g];
+          const float f = mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M);
+          lsum += f * s_l[w * G + g];
+          o += f * s_acc[(w * HG + gg) * D + d];
+        }
+        if (single) {
+          static_cast<T*>(a.out)[(static_cast<int64_t>(s) * a.num_heads + h0 + g) * D + d] =
+              from_float<T>(lsum > 0.f ? o / lsum : 0.f);
+        } else {
+          const int64_t cell = (static_cast<int64_t>(s) * a.num_heads + h0 + g) * a.max_parts + info.part;
+          a.tmp_out[cell * D + d] = o / lsum;
+          if (d == 0) {
+            a.tmp_m[cell] = M;
+            a.tmp_l[cell] = lsum;
+          }
         }
       }
     }

@@ -51,7 +51,7 @@ def test_workspace_bytes_formula():
     assert B.decode_workspace_bytes(4, 32, 128, 32768, 1024) == _layout_bytes(4, 32, 128, 32768, 1024)
     # invalid partition sizes give 0
     assert B.decode_workspace_bytes(4, 32, 128, 32768, 48) == 0
-    assert B.decode_workspace_bytes(4, 32, 128, 32768, 8192) == 0
+    assert B.decode_workspace_bytes(4, 32, 128, 32768, 4096) == 0
 
 
 FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: every call below fails first
@@ -84,8 +84,9 @@ def _paged(**kw):
     (dict(out=None), B.PKV_EINVAL),
     (dict(tables=None), B.PKV_EINVAL),
     (dict(k=ctypes.c_void_p((1 << 20) + 8)), B.PKV_EINVAL),   # misaligned
-    (dict(part=48), B.PKV_EINVAL),                # not a multiple of 32
-    (dict(part=8192), B.PKV_EINVAL),              # above 4096
+    (dict(part=48), B.PKV_EINVAL),                # not a multiple of 64
+    (dict(part=96), B.PKV_EINVAL),
+    (dict(part=4096), B.PKV_EINVAL),              # above 2048
     (dict(MB=64), B.PKV_EINVAL),                  # no workspace given
 ])
 def test_paged_decode_rejects_bad_arguments_before_launch(kw, status):
