@@ -65,6 +65,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU baseline sample budget")
+    ap.add_argument("--eager", action="store_true",
+                    help="time eager launches instead of CUDA-graph replays of the step")
     return ap.parse_args(argv)
 
 
@@ -276,45 +278,67 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     n_pairs = int(b["pairs"].shape[0])
     max_parts = math.ceil(w.max_blocks_per_seq * w.block_size / part)
-    launches_per_step = 1 + 1 + (1 if max_parts > 1 else 0) + (1 if n_pairs else 0)
+    # cache write; plan + decode (+ partition merge when contexts can span partitions)
+    launches_per_step = 1 + 2 + (1 if max_parts > 1 else 0) + (1 if n_pairs else 0)
 
-    def step():
+    def write_step():
         if n_pairs:
             pkv.copy_blocks(b["k_cache"], b["v_cache"], b["pairs"])
         pkv.reshape_and_cache(b["new_k"], b["new_v"], b["k_cache"], b["v_cache"], b["slots"])
+
+    def decode_step():
         pkv.paged_attention_decode(b["out"], b["q"], b["k_cache"], b["v_cache"], b["tables"], b["lens"],
                                    w.scale, partition_size=part, workspace=ws)
 
+    def timed_steps(run_write, run_decode, K):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        barrier()
+        torch.cuda.synchronize()
+        for k in range(K):
+            flush.zero_()
+            evs[k][0].record()
+            run_write()
+            evs[k][1].record()
+            run_decode()
+            evs[k][2].record()
+        torch.cuda.synchronize()
+        barrier()
+        return ([e[0].elapsed_time(e[2]) for e in evs], [e[1].elapsed_time(e[2]) for e in evs])
+
     for _ in range(max(args.warmup, 0)):
         flush.zero_()
-        step()
+        write_step()
+        decode_step()
     torch.cuda.synchronize()
     if pkv.device_error():
         raise RuntimeError("device error flags set during warm-up")
 
+    eager_step_ms, _ = timed_steps(write_step, decode_step, min(args.steps, 5))
+    if args.eager:
+        run_write, run_decode, mode = write_step, decode_step, "eager launches"
+    else:
+        # A serving engine replays the decode step as a CUDA graph; so does the bench.
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        g_write, g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_write, stream=side):
+            write_step()
+        with torch.cuda.graph(g_decode, stream=side):
+            decode_step()
+        torch.cuda.current_stream().wait_stream(side)
+        for _ in range(2):
+            flush.zero_()
+            g_write.replay()
+            g_decode.replay()
+        torch.cuda.synchronize()
+        run_write, run_decode, mode = g_write.replay, g_decode.replay, "CUDA graph replay"
+
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     sampler = ClockSampler(local) if rank == 0 else None
     if sampler:
         sampler.start()
-    barrier()
-    torch.cuda.synchronize()
-    for k in range(K):
-        flush.zero_()
-        e0, e1, e2 = ev[k]
-        e0.record()
-        if n_pairs:
-            pkv.copy_blocks(b["k_cache"], b["v_cache"], b["pairs"])
-        pkv.reshape_and_cache(b["new_k"], b["new_v"], b["k_cache"], b["v_cache"], b["slots"])
-        e1.record()
-        pkv.paged_attention_decode(b["out"], b["q"], b["k_cache"], b["v_cache"], b["tables"], b["lens"],
-                                   w.scale, partition_size=part, workspace=ws)
-        e2.record()
-    torch.cuda.synchronize()
-    barrier()
+    step_ms, decode_ms = timed_steps(run_write, run_decode, K)
     clocks = sampler.stop() if sampler else None
-    step_ms = [ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]
-    decode_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
     if pkv.device_error():
         raise RuntimeError("device error flags set during the timed steps")
 
@@ -338,14 +362,16 @@ def run_ours(args, world, rank, local):
             "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
             "context_tokens_per_gpu": int(inp.context_lens.sum()), "partition_size": part,
             "l2": "flushed before every timed step (256 MiB write); K/V read per step > L2",
+            "execution": mode,
             "parallelism": f"dp{world} (sequences sharded, no collective)",
         },
         "seqs_per_s": round(total_seqs / (total_ms * 1e-3), 1),
         "pct_of_nominal_8tbs": round(100 * value / NOMINAL_HBM_GBS, 2),
         "bytes_per_step": nbytes,
+        "eager_ms_per_step": round(statistics.mean(eager_step_ms), 5),
         "gpu_launches": launches_per_step * K,
         "roofline": {
-            "bound": "hbm", "kernel": "paged_attention_decode (pass 1 + partition merge)",
+            "bound": "hbm", "kernel": "paged_attention_decode call (plan + decode + partition merge kernels)",
             "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "traffic": (traffic or {}).get("bytes_per_launch") if traffic else None,
@@ -377,6 +403,17 @@ def contiguous_compare(args, inp, b, ws, flush, part, device):
 
     def time_it(fn):
         for _ in range(3):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        if not args.eager:
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                fn()
+            torch.cuda.current_stream().wait_stream(side)
+            fn = g.replay
             flush.zero_()
             fn()
         evs = []

@@ -61,6 +61,7 @@ struct DecodeArgs {
   int32_t part_tokens;    // maximum tokens per partition (multiple of 32)
   int32_t max_parts;      // ceil(max_ctx / part_tokens): upper bound of partitions per context
   float scale_log2;       // scale * log2(e)
+  int32_t grid_ctas;      // decode CTAs; the first 3 * grid_ctas items are assigned statically
   uint32_t* work;         // [0] next item, [1] item count, [2] multi-partition sequences
   int32_t* merge_seqs;    // [S] sequences whose context spans more than one partition
   uint8_t* records;       // [S * max_parts] work records, largest partition first (32 B each)
@@ -236,7 +237,7 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
     }
   }
   if (threadIdx.x == 0) {
-    a.work[0] = 0;
+    a.work[0] = 3u * static_cast<uint32_t>(a.grid_ctas);  // items below are pre-assigned
     a.work[1] = total * static_cast<uint32_t>(a.num_kv_heads);
     a.work[2] = n_multi;
   }
@@ -347,9 +348,11 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
     uint32_t idx0 = 0, idx1 = 0, idx2 = 0;  // items k, k + 1, k + 2 (lane 0)
     bool ok = true;
     if (lane == 0) {
-      idx0 = atomicAdd(a.work, 1u);
-      idx1 = atomicAdd(a.work, 1u);
-      idx2 = atomicAdd(a.work, 1u);
+      // CTA c starts with items c, c + G, c + 2G (G = grid size) of the
+      // largest-first list, then takes more from the counter.
+      idx0 = blockIdx.x;
+      idx1 = blockIdx.x + gridDim.x;
+      idx2 = blockIdx.x + 2 * gridDim.x;
       if (idx0 < n_items) copy_record(0, idx0);
       if (idx1 < n_items) copy_record(1, idx1);
     }

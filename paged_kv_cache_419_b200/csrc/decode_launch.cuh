@@ -31,11 +31,13 @@ cudaError_t decode_grid(int num_sms, int* grid) {
 }
 
 template <typename T, int D, int G, int B, bool PAGED>
-cudaError_t launch_decode_one(const DecodeArgs& a, int num_sms, cudaStream_t stream) {
+cudaError_t launch_decode_one(const DecodeArgs& args, int num_sms, cudaStream_t stream) {
   using Tr = DecodeTraits<T, D, G, B, PAGED>;
   int grid = 0;
   cudaError_t e = decode_grid<T, D, G, B, PAGED>(num_sms, &grid);
   if (e != cudaSuccess) return e;
+  DecodeArgs a = args;
+  a.grid_ctas = grid;
   // Programmatic dependent launch for all three kernels: each may start (and
   // set up) while its predecessor finishes, and waits for it in-kernel before
   // touching anything the predecessor writes.
