@@ -109,13 +109,32 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profile_traffic():
-    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary,
-    with the kernel revision they were taken on; null when absent."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+DECODE_SOURCES = ("decode.cuh", "decode_launch.cuh", "device.cuh")
+
+
+def decode_sources_sha256() -> str:
+    """Hash of the decode kernel's sources: the revision an ncu capture describes."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_419_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profile_traffic(algorithmic_bytes_per_launch: int):
+    """DRAM bytes per decode launch from the committed ncu summary
+    (profiles/decode_gqa8b64_traffic.json: read + write bytes over algorithmic bytes of the
+    captured case, scaled to this launch).  None when there is no summary or when
+    the decode sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "decode_gqa8b64_traffic.json")
     try:
         with open(path) as f:
-            return json.load(f)
+            t = json.load(f)
+        if t.get("sources_sha256") != decode_sources_sha256():
+            return None
+        return int(round(t["traffic_over_algorithmic"] * algorithmic_bytes_per_launch))
     except Exception:
         return None
 
@@ -349,7 +368,7 @@ def run_ours(args, world, rank, local):
     peak, peak_kind = measured_hbm_peak()
     dec_ms = statistics.mean(decode_ms)
     achieved = nbytes["decode"] / (dec_ms * 1e-3) / 1e9
-    traffic = profile_traffic()
+    traffic = profile_traffic(nbytes["decode"])
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
@@ -374,7 +393,7 @@ def run_ours(args, world, rank, local):
             "bound": "hbm", "kernel": "paged_attention_decode call (plan + decode + partition merge kernels)",
             "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
             "frac": round(achieved / peak, 4),
-            "traffic": (traffic or {}).get("bytes_per_launch") if traffic else None,
+            "traffic": traffic,
             "decode_ms": round(dec_ms, 5),
         },
         "clocks": clocks,
