@@ -2,6 +2,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
 #include <vector>
 
 #include "cache_ops.cuh"
@@ -86,6 +87,64 @@ size_t workspace_bytes(int64_t S, int64_t Hq, int64_t D, int64_t max_ctx, int64_
   return static_cast<size_t>(workspace_layout(S, Hq, D, max_ctx, part).total);
 }
 
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link against
+// the driver library).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Map of a cache viewed as [planes][rows][head_dim] 16-bit elements: boxes of
+// one 128-byte panel x box_rows rows x 1 plane, 128-byte swizzle, zero fill
+// outside the tensor, 256-byte L2 promotion (a box reads half of each
+// 256-byte row; the other half is the next box).
+pkv_status encode_cache_map(CUtensorMap* m, const void* base, pkv_dtype dtype, int head_dim,
+                            int64_t rows, int64_t planes, int box_rows) {
+  const EncodeTiledFn fn = encode_tiled();
+  if (!fn) return PKV_ECUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim),
+                              static_cast<cuuint64_t>(rows > 0 ? rows : 1),
+                              static_cast<cuuint64_t>(planes > 0 ? planes : 1)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                 static_cast<cuuint64_t>(dims[1]) * head_dim * 2};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t elem_strides[3] = {1u, 1u, 1u};
+  const CUresult r =
+      fn(m, dtype == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+         const_cast<void*>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_EINVAL;
+}
+
+// The four maps of one call (full-chunk and 8-row boxes of K and V).
+pkv_status encode_decode_maps(DecodeMaps* m, const DecodeArgs& a, pkv_dtype dtype, int head_dim,
+                              int block_size, bool paged) {
+  const int64_t rows = paged ? static_cast<int64_t>(a.num_kv_heads) * block_size : a.max_ctx;
+  const int64_t planes =
+      paged ? a.num_blocks : static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
+  const int ch = chunk_rows(paged, block_size);
+  pkv_status st;
+  if ((st = encode_cache_map(&m->k, a.k, dtype, head_dim, rows, planes, ch)) != PKV_OK) return st;
+  if ((st = encode_cache_map(&m->v, a.v, dtype, head_dim, rows, planes, ch)) != PKV_OK) return st;
+  if ((st = encode_cache_map(&m->k_tail, a.k, dtype, head_dim, rows, planes, 8)) != PKV_OK) return st;
+  return encode_cache_map(&m->v_tail, a.v, dtype, head_dim, rows, planes, 8);
+}
+
 // Shared checks and launch of the paged and contiguous decode.
 pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pkv_dtype dtype,
                          int32_t partition_size, void* workspace, size_t ws_bytes, bool paged,
@@ -119,13 +178,17 @@ pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pk
   if (st != PKV_OK) return st;
   a.err = dev->err;
   const int sms = dev->num_sms;
+  DecodeMaps maps;
+  st = encode_decode_maps(&maps, a, dtype, head_dim, block_size, paged);
+  if (st != PKV_OK) return st;
   cudaError_t e;
   if (dtype == PKV_F16)
-    e = head_dim == 64 ? launch_decode<__half, 64>(a, group, block_size, paged, sms, stream)
-                       : launch_decode<__half, 128>(a, group, block_size, paged, sms, stream);
+    e = head_dim == 64 ? launch_decode<__half, 64>(a, maps, group, block_size, paged, sms, stream)
+                       : launch_decode<__half, 128>(a, maps, group, block_size, paged, sms, stream);
   else
-    e = head_dim == 64 ? launch_decode<__nv_bfloat16, 64>(a, group, block_size, paged, sms, stream)
-                       : launch_decode<__nv_bfloat16, 128>(a, group, block_size, paged, sms, stream);
+    e = head_dim == 64
+            ? launch_decode<__nv_bfloat16, 64>(a, maps, group, block_size, paged, sms, stream)
+            : launch_decode<__nv_bfloat16, 128>(a, maps, group, block_size, paged, sms, stream);
   return from_cuda(e);
 }
 

@@ -36,6 +36,7 @@
 //    exponentials are single ex2 instructions.
 #pragma once
 
+#include <cuda.h>
 #include <math_constants.h>
 
 #include <type_traits>
@@ -61,7 +62,7 @@ struct DecodeArgs {
   int32_t part_tokens;    // maximum tokens per partition (multiple of 32)
   int32_t max_parts;      // ceil(max_ctx / part_tokens): upper bound of partitions per context
   float scale_log2;       // scale * log2(e)
-  int32_t grid_ctas;      // decode CTAs; the first 3 * grid_ctas items are assigned statically
+  int32_t grid_ctas;      // decode CTAs; item c (c < grid_ctas) is CTA c's first item
   uint32_t* work;         // [0] next item, [1] item count, [2] multi-partition sequences
   int32_t* merge_seqs;    // [S] sequences whose context spans more than one partition
   uint8_t* records;       // [S * max_parts] work records, largest partition first (32 B each)
@@ -76,7 +77,7 @@ constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxPartTokens = 2048;
 constexpr int kPlanThreads = 1024;
 constexpr int kItemSlots = 2;
-constexpr int kRecSlots = 4;   // records of items k .. k+3 (copied two items ahead)
+constexpr int kRecSlots = 2;   // records of items k and k+1
 constexpr int kStageTokens = 64;
 // Work record of one (sequence, partition): int32 s, part, n_parts, t_begin,
 // n_tok, L, 0, 0.
@@ -100,49 +101,61 @@ __device__ __forceinline__ int clamp_len(int L, int max_ctx) {
   return L < 0 ? 0 : (L > max_ctx ? max_ctx : L);
 }
 
+// Rows of a full box: one cache block (paged, blocks up to a stage long) or a
+// whole stage (contiguous).
+constexpr int chunk_rows(bool paged, int block_size) {
+  return paged ? (block_size < kStageTokens ? block_size : kStageTokens) : kStageTokens;
+}
+
+// Tensor maps of the K and V caches, built on the host for each call.  A cache
+// is viewed as [planes][rows][D] (paged: [N][Hkv * B][D]; contiguous:
+// [S * Hkv][max_ctx][D]).  A box is one 128-byte panel (64 elements) of D wide
+// and stored with the 128-byte swizzle: 16-byte chunk c of tile row r lands at
+// chunk c ^ (r % 8) of that row.  `k`, `v` copy a full chunk of CH rows;
+// `k_tail`, `v_tail` 8 rows, for the ragged end of a context.
+struct DecodeMaps {
+  CUtensorMap k, v, k_tail, v_tail;
+};
+
 template <typename T, int D_, int G_, int B_, bool PAGED_>
 struct DecodeTraits {
   static constexpr int D = D_;
   static constexpr int G = G_;
   static constexpr int B = B_;
   static constexpr bool PAGED = PAGED_;
-  static constexpr int LPT = (G * D / 8 <= 64) ? 8 : 16;  // lanes per token (scores)
-  static constexpr int LPH = LPT / G;                     // lanes holding one head's score
-  static constexpr int EPL = D / LPT;                     // row elements per lane (scores)
-  static constexpr int VPL = EPL / 8;                     // 16-byte vectors per lane (scores)
-  static constexpr int TPR = 32 / LPT;                    // tokens per warp round
-  static constexpr int TPW = kStageTokens / kConsumerWarps;  // tokens per warp per stage
-  static constexpr int ROUNDS = TPW / TPR;
-  static constexpr int TS = kConsumerWarps * TPW;         // tokens per stage
-  static constexpr int CH = PAGED ? (B < TS ? B : TS) : TS;  // tokens per bulk copy
+  static constexpr int TS = kStageTokens;                    // tokens per stage
+  static constexpr int TPW = TS / kConsumerWarps;            // tokens per warp per stage
+  static constexpr int KS = D / 16;                          // k-steps of the score tile
+  static constexpr int MT = D / 16;                          // 16-dim m-tiles of the output tile
+  static constexpr int ND = D / 64;                          // 128-byte panels per row
+  static constexpr int CH = chunk_rows(PAGED, B);            // rows per full box
   static constexpr int NCH = TS / CH;
   static constexpr int STAGES = 2;
-  static constexpr int DPL = D / 32;                      // output dims per lane (PV)
   static constexpr int ROW_BYTES = D * 2;
-  static constexpr int TILE_BYTES = TS * ROW_BYTES;
+  static constexpr int PANEL_BYTES = TS * 128;               // one panel of a stage tile
+  static constexpr int TILE_BYTES = ND * PANEL_BYTES;        // K (or V) of one stage
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int Q_BYTES = G * D * 2;
+  static constexpr int ACC_PITCH = D + 4;                    // floats per head row of a merge slot
+  static constexpr int HG = G <= 2 ? G : G / 2;              // heads per merge round
   static constexpr int MAX_TABLE = PAGED ? kMaxPartTokens / B : 4;  // table entries of one item
-  // shared memory carve-up (bytes, 16-byte aligned pieces)
+  // shared memory carve-up (bytes from a 1024-byte aligned base)
   static constexpr int OFF_Q = STAGES * STAGE_BYTES;
-  static constexpr int HG = G > 1 ? G / 2 : 1;                          // heads per merge round
-  static constexpr int OFF_ACC = OFF_Q + kItemSlots * Q_BYTES;          // [warps][HG][D] f32
-  static constexpr int OFF_P = OFF_ACC + kConsumerWarps * HG * D * 4;   // [warps][TPW][G] (p, p)
-  static constexpr int OFF_REC = OFF_P + kConsumerWarps * TPW * G * 8;  // record slots
+  static constexpr int OFF_ACC = OFF_Q + kItemSlots * Q_BYTES;          // [warps][HG][ACC_PITCH] f32
+  static constexpr int OFF_REC = OFF_ACC + kConsumerWarps * HG * ACC_PITCH * 4;  // record slots
   static constexpr int OFF_TAB = OFF_REC + kRecSlots * kRecordBytes;    // 2 table buffers
   static constexpr int OFF_STAT = OFF_TAB + 2 * MAX_TABLE * 4;          // m, l per warp and head
   static constexpr int OFF_ITEM = OFF_STAT + 2 * kConsumerWarps * G * 4 + 16;
   static constexpr int OFF_BARS = OFF_ITEM + kItemSlots * 32;
-  static constexpr int SMEM_BYTES = OFF_BARS + (2 * STAGES + 2 * kItemSlots + kRecSlots + 2) * 8;
+  static constexpr int SMEM_USED = OFF_BARS + (4 * STAGES + 2 * kItemSlots + kRecSlots + 2) * 8;
+  static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base
 
-  static_assert(D % 64 == 0, "head_dim must be 64 or 128");
-  static_assert(EPL % 8 == 0 && VPL >= 1, "score vectors are 16 bytes");
-  static_assert(G <= LPT && LPT % G == 0, "reduce-scatter leaves one head per lane group");
-  static_assert(TPW % TPR == 0, "whole rounds per stage");
-  static_assert(TS == kStageTokens, "stage = partition granule");
-  static_assert(TS % CH == 0 && NCH <= 32, "whole copies per stage, one lane each");
-  static_assert(DPL == 2 || DPL == 4, "PV reads 4 or 8 bytes per lane");
-  static_assert(OFF_BARS % 8 == 0 && OFF_STAT % 16 == 0, "alignment");
+  static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
+  static_assert(G <= 8, "one 8-column n-tile holds the heads of a group");
+  static_assert(TPW == 16, "a warp's tokens are one 16-deep k-step of the output tile");
+  static_assert(CH % 8 == 0 && TS % CH == 0 && NCH * ND <= 32, "one copier lane per box");
+  static_assert(STAGE_BYTES % 1024 == 0 && PANEL_BYTES % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(OFF_BARS % 8 == 0 && OFF_STAT % 16 == 0 && OFF_ACC % 16 == 0, "alignment");
   // three CTAs per SM (228 KB of shared memory, 1 KB reserved per CTA) up to G = 4
   static_assert(G > 4 || 3 * (SMEM_BYTES + 1024) <= 228 * 1024, "3 CTAs per SM");
 };
@@ -237,7 +250,7 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
     }
   }
   if (threadIdx.x == 0) {
-    a.work[0] = 3u * static_cast<uint32_t>(a.grid_ctas);  // items below are pre-assigned
+    a.work[0] = static_cast<uint32_t>(a.grid_ctas);  // item c is CTA c's first
     a.work[1] = total * static_cast<uint32_t>(a.num_kv_heads);
     a.work[2] = n_multi;
   }
@@ -245,22 +258,28 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
 
 // ---------------------------------------------------------------- decode
 template <typename T, int D, int G, int B, bool PAGED>
-__global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
+    decode_kernel(const DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
   using Tr = DecodeTraits<T, D, G, B, PAGED>;
-  constexpr int STAGES = Tr::STAGES, TS = Tr::TS, LPT = Tr::LPT, LPH = Tr::LPH, TPR = Tr::TPR;
-  constexpr int TPW = Tr::TPW, ROUNDS = Tr::ROUNDS, VPL = Tr::VPL, DPL = Tr::DPL;
+  constexpr int STAGES = Tr::STAGES, TS = Tr::TS, TPW = Tr::TPW, KS = Tr::KS, MT = Tr::MT;
+  constexpr int ND = Tr::ND;
   constexpr int NW = kConsumerWarps;
 
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BARS);
-  uint64_t* empty = full + STAGES;
-  uint64_t* item_full = empty + STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // Swizzled tiles need a 1024-byte aligned base; the launch reserves the slack.
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  // K and V halves of a stage have their own barriers: K is released after the
+  // scores, V after PV, so a half is refilled as soon as it is no longer read.
+  uint64_t* full_k = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BARS);
+  uint64_t* full_v = full_k + STAGES;
+  uint64_t* empty_k = full_v + STAGES;
+  uint64_t* empty_v = empty_k + STAGES;
+  uint64_t* item_full = empty_v + STAGES;
   uint64_t* item_empty = item_full + kItemSlots;
   uint64_t* rec_bar = item_empty + kItemSlots;  // [kRecSlots]
   uint64_t* tab_bar = rec_bar + kRecSlots;       // [2]
   ItemInfo* items = reinterpret_cast<ItemInfo*>(smem + Tr::OFF_ITEM);
   float* s_acc = reinterpret_cast<float*>(smem + Tr::OFF_ACC);
-  float2* s_p = reinterpret_cast<float2*>(smem + Tr::OFF_P);
   float* s_m = reinterpret_cast<float*>(smem + Tr::OFF_STAT);
   float* s_l = s_m + NW * G;
 
@@ -269,8 +288,10 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], NW);
+      mbar_init(&full_k[i], 1);
+      mbar_init(&full_v[i], 1);
+      mbar_init(&empty_k[i], NW);
+      mbar_init(&empty_v[i], NW);
     }
     for (int i = 0; i < kItemSlots; ++i) {
       mbar_init(&item_full[i], 1);
@@ -286,38 +307,40 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
   grid_dependency_wait();
 
   // ================================================================ producer
-  // Item j (the j-th item this CTA takes): its index is taken three items ahead,
-  // its 32-byte record is bulk-copied two items ahead into record slot j % 4, and
-  // its block-table entries are fetched one item ahead with cp.async into table
-  // buffer j % 2.  So while item k's stages are issued, nothing the producer
-  // waits for was requested less than one item ago.
+  // Item k (the k-th item this CTA takes).  The CTA's first item is item
+  // blockIdx.x of the largest-first list; each later one comes from the work
+  // counter, taken while the previous item streams: right after that item's
+  // first stage is issued (a stage is in flight while the atomic returns), its
+  // 32-byte record is bulk-copied; after the second stage (or at the end of a
+  // one-stage item) the record has landed and its block-table entries are
+  // fetched with cp.async.  Only one item is ever reserved ahead, so the end of
+  // the list stays dynamic.
   if (warp == NW) {
-    const uint8_t* kbase = static_cast<const uint8_t*>(a.k);
-    const uint8_t* vbase = static_cast<const uint8_t*>(a.v);
+    if (lane < 4) prefetch_tensor_map(&maps.k + lane);
     const uint32_t n_items = *reinterpret_cast<volatile uint32_t*>(a.work + 1);
     const uint32_t Hkv = static_cast<uint32_t>(a.num_kv_heads);
     int32_t* s_tab = reinterpret_cast<int32_t*>(smem + Tr::OFF_TAB);
     auto rec_slot = [&](uint32_t j) {
-      return reinterpret_cast<const int32_t*>(smem + Tr::OFF_REC + (j % kRecSlots) * kRecordBytes);
+      return reinterpret_cast<const int32_t*>(smem + Tr::OFF_REC + (j & 1) * kRecordBytes);
     };
     // Outstanding copies nobody waited for yet (error exits drain them): bit r of
     // rec_pending / rec_parity = record slot r and the parity of its open phase;
     // likewise for the two table buffers.
     uint32_t rec_pending = 0, rec_parity = 0, tab_pending = 0, tab_parity = 0;
-    auto copy_record = [&](uint32_t j, uint32_t idx) {  // lane 0
-      const uint32_t r = j % kRecSlots;
+    auto copy_record = [&](uint32_t j, uint32_t idx) {  // lane 0; record j -> slot j % 2
+      const uint32_t r = j & 1;
+      fence_proxy_async_smem();  // this slot was last read two items ago
       mbar_arrive_expect_tx(&rec_bar[r], kRecordBytes);
       bulk_load(smem + Tr::OFF_REC + r * kRecordBytes,
                 a.records + static_cast<int64_t>(idx / Hkv) * kRecordBytes, kRecordBytes, &rec_bar[r]);
       rec_pending |= 1u << r;
-      rec_parity = (rec_parity & ~(1u << r)) | (((j / kRecSlots) & 1u) << r);
+      rec_parity = (rec_parity & ~(1u << r)) | (((j >> 1) & 1u) << r);
     };
-    // Every lane waits for record j (all lanes read it).
-    auto wait_record = [&](uint32_t j) {
-      const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&rec_bar[j % kRecSlots], (j / kRecSlots) & 1));
+    auto wait_record = [&](uint32_t j) {  // every lane reads the record, so every lane waits
+      const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&rec_bar[j & 1], (j >> 1) & 1));
       if (lane == 0) {
         if (!got) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
-        rec_pending &= ~(1u << (j % kRecSlots));
+        rec_pending &= ~(1u << (j & 1));
       }
       return got;
     };
@@ -345,26 +368,16 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
       return true;
     };
 
-    uint32_t idx0 = 0, idx1 = 0, idx2 = 0;  // items k, k + 1, k + 2 (lane 0)
     bool ok = true;
-    if (lane == 0) {
-      // CTA c starts with items c, c + G, c + 2G (G = grid size) of the
-      // largest-first list, then takes more from the counter.
-      idx0 = blockIdx.x;
-      idx1 = blockIdx.x + gridDim.x;
-      idx2 = blockIdx.x + 2 * gridDim.x;
-      if (idx0 < n_items) copy_record(0, idx0);
-      if (idx1 < n_items) copy_record(1, idx1);
-    }
-    if (__shfl_sync(0xffffffffu, idx0, 0) < n_items) {
+    uint32_t cur = blockIdx.x;  // this CTA's first item
+    if (cur < n_items) {
+      if (lane == 0) copy_record(0, cur);
       ok = wait_record(0);
       if (ok) fetch_table(0);
     }
     uint32_t issued = 0, st = 0, ph = 0;  // stages issued; ring slot and use parity of the next
     for (uint32_t k = 0; ok; ++k) {
       const int slot = k & (kItemSlots - 1);
-      const uint32_t cur = __shfl_sync(0xffffffffu, idx0, 0);
-      const uint32_t nx1 = __shfl_sync(0xffffffffu, idx1, 0);
       if (lane == 0 && k >= kItemSlots &&
           !mbar_wait_bounded(&item_empty[slot], ((k / kItemSlots) - 1) & 1)) {
         set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
@@ -379,20 +392,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
         }
         break;
       }
-      uint32_t idx3 = 0;
-      if (lane == 0) {
-        if (idx2 < n_items) {
-          fence_proxy_async_smem();  // this record slot was last read two items ago
-          copy_record(k + 2, idx2);
-        }
-        idx3 = atomicAdd(a.work, 1u);
-      }
-      if (nx1 < n_items) {
-        // record k + 1 was requested one item ago; fetch its table now
-        if (!wait_record(k + 1)) break;
-        fetch_table(k + 1);
-      }
-      if (!wait_table(k)) break;  // requested one item ago
+      if (!wait_table(k)) break;  // fetched while the previous item streamed
       const int32_t* rec = rec_slot(k);
       const int s = rec[0], part = rec[1], n_parts = rec[2], t_begin = rec[3], n_tok = rec[4];
       const int kvh = static_cast<int>(cur % Hkv);
@@ -411,55 +411,105 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
       }
       const int32_t* tab = s_tab + (k & 1) * Tr::MAX_TABLE;
       const int n_stages = (n_tok + TS - 1) / TS;
-      for (int i = 0; i < n_stages; ++i) {
-        if (lane == 0 && issued >= STAGES && !mbar_wait_bounded(&empty[st], ph ^ 1)) {
-          set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
-          ok = false;
+      uint32_t nxt = n_items;     // next item (lane 0 knows it after the first stage)
+      bool next_ready = false;    // its record waited for and its table requested
+      auto prepare_next = [&](int step) {
+        if (step == 0) {
+          if (lane == 0) {
+            nxt = atomicAdd(a.work, 1u);
+            if (nxt < n_items) copy_record(k + 1, nxt);
+          }
+          nxt = __shfl_sync(0xffffffffu, nxt, 0);
+        } else if (!next_ready) {
+          next_ready = true;
+          if (nxt < n_items) {
+            if (!wait_record(k + 1)) return false;
+            fetch_table(k + 1);
+          }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
+        return true;
+      };
+      for (int i = 0; i < n_stages; ++i) {
         const int t0 = i * TS;  // relative to the partition start (block aligned)
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2u * min(TS, n_tok - t0) * Tr::ROW_BYTES);
-        __syncwarp();
-        const int tc = t0 + lane * Tr::CH;
-        if (lane < Tr::NCH && tc < n_tok) {
-          const uint32_t nbytes = min(Tr::CH, n_tok - tc) * Tr::ROW_BYTES;
-          int64_t row;
+        // Boxes: full chunks of CH rows, the ragged end in 8-row boxes, so a
+        // stage moves its valid rows rounded up to 8, per panel.
+        const int nvs = min(TS, n_tok - t0);
+        const uint32_t half_bytes = static_cast<uint32_t>((nvs + 7) & ~7) * Tr::ROW_BYTES;
+        const int c = lane / ND, h = lane % ND;  // copier lane: chunk and panel
+        const int tc = t0 + c * Tr::CH;
+        const bool copier = c < Tr::NCH && tc < n_tok;
+        int rows = 0, y = 0, z = 0;
+        if (copier) {
+          rows = min(Tr::CH, n_tok - tc);
           if constexpr (PAGED) {
             int32_t f = tab[tc / B];
             if (f < 0 || f >= a.num_blocks) {
               set_error(a.err, PKV_DEVERR_TABLE_ENTRY);
               f = 0;
             }
-            row = (static_cast<int64_t>(f) * a.num_kv_heads + kvh) * B + tc % B;
+            y = kvh * B + tc % B;
+            z = f;
           } else {
-            row = (static_cast<int64_t>(s) * a.num_kv_heads + kvh) * a.max_ctx + t_begin + tc;
+            y = t_begin + tc;
+            z = s * static_cast<int>(Hkv) + kvh;
           }
-          uint8_t* sk = smem + st * Tr::STAGE_BYTES + lane * Tr::CH * Tr::ROW_BYTES;
-          bulk_load(sk, kbase + row * Tr::ROW_BYTES, nbytes, &full[st]);
-          bulk_load(sk + Tr::TILE_BYTES, vbase + row * Tr::ROW_BYTES, nbytes, &full[st]);
         }
+        uint8_t* dst = smem + st * Tr::STAGE_BYTES + h * Tr::PANEL_BYTES + c * Tr::CH * 128;
+        auto issue = [&](uint8_t* d, const CUtensorMap* full, const CUtensorMap* tail, uint64_t* bar) {
+          if (!copier) return;
+          if (rows == Tr::CH) {
+            tma_load_3d(d, full, h * 64, y, z, bar);
+          } else {
+            for (int r = 0; r < rows; r += 8) tma_load_3d(d + r * 128, tail, h * 64, y + r, z, bar);
+          }
+        };
+        // K half: free once the consumers' scores of this slot's last use are done
+        if (lane == 0 && issued >= STAGES && !mbar_wait_bounded(&empty_k[st], ph ^ 1)) {
+          set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+          ok = false;
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full_k[st], half_bytes);
+        __syncwarp();
+        issue(dst, &maps.k, &maps.k_tail, &full_k[st]);
+        __syncwarp();
+        // V half: free once their PV is done
+        if (lane == 0 && issued >= STAGES && !mbar_wait_bounded(&empty_v[st], ph ^ 1)) {
+          set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+          ok = false;
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full_v[st], half_bytes);
+        __syncwarp();
+        issue(dst + Tr::TILE_BYTES, &maps.v, &maps.v_tail, &full_v[st]);
         __syncwarp();
         ++issued;
         if (++st == STAGES) {
           st = 0;
           ph ^= 1;
         }
+        if (i <= 1 && !prepare_next(i)) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) break;  // the consumers time out on their next wait and stop too
-      idx0 = idx1;
-      idx1 = idx2;
-      idx2 = idx3;
+      if (n_stages == 0 && !prepare_next(0)) break;
+      if (!prepare_next(1)) break;  // one-stage (or empty) items: finish preparing now
+      cur = nxt;
     }
     // Never leave the CTA with copies in flight: wait (bounded) until the last
     // use of every stage, and every record and table copy, have landed.
     if (lane == 0) {
       const uint32_t first = issued > STAGES ? issued - STAGES : 0;
       for (uint32_t i = first; i < issued; ++i)
-        if (!mbar_wait_bounded(&full[i % STAGES], (i / STAGES) & 1))
+        if (!mbar_wait_bounded(&full_k[i % STAGES], (i / STAGES) & 1) ||
+            !mbar_wait_bounded(&full_v[i % STAGES], (i / STAGES) & 1))
           set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
     }
-    for (int r = 0; r < kRecSlots; ++r)
+    for (int r = 0; r < 2; ++r)
       if (lane == 0 && ((rec_pending >> r) & 1u) &&
           !mbar_wait_bounded(&rec_bar[r], (rec_parity >> r) & 1u))
         set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
@@ -471,14 +521,30 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
   }
 
   // ================================================================ consumers
+  // Warp w owns tokens [16 w, 16 w + 16) of every stage, with its own online
+  // softmax state per head; the tiles run on the tensor cores (mma.sync
+  // m16n8k16, fp32 accumulation):
+  //   scores  S^T (16 x 16) = Q (16 x D, rows >= G zero) K^T: two 8-token
+  //           n-tiles, K read with ldmatrix straight from the swizzled stage;
+  //   output  O^T (D x 8) += V^T (D x 16) P^T (16 x 8): V read with transposing
+  //           ldmatrix, P^T taken from the score accumulators as they lie
+  //           (their C layout is the B layout of the next product).
   // Exits are decided together (barrier-OR over the consumer warps) so that no
   // warp is ever left waiting at a named barrier.
-  const int tg = lane / LPT;       // token group inside a round
-  const int li = lane % LPT;       // lane inside the token group
-  const int my_h = li / LPH;       // head whose score this lane holds after the reduce-scatter
-  const bool p_writer = (li % LPH) == 0;
+  const int quad = lane >> 2;  // score tile: head row; output tile: dim row
+  const int qc = lane & 3;     // score tile: token pair; output tile: head pair
   const int w_tok0 = warp * TPW;
-  float2* p_warp = s_p + warp * TPW * G;
+  // ldmatrix addressing: lane supplies row (lane & 7) of matrix (lane >> 3).
+  // Swizzled offset of 16-byte chunk j of tile row r: r * 128 + ((j ^ (r & 7)) << 4);
+  // the part of j that varies per call is applied with one xor.
+  const int mrow = lane & 7, mat = lane >> 3;
+  // K, matrix i of k-step pair kp: token w_tok0 + 8 nt + mrow, chunk 4 (kp & 1) + i
+  // of panel kp / 2.
+  const uint32_t k_lane = static_cast<uint32_t>((w_tok0 + mrow) * 128 + ((mat ^ mrow) << 4));
+  // V, matrix i of m-tile mt: token w_tok0 + 8 (i >> 1) + mrow, chunk
+  // 2 (mt & 3) + (i & 1) of panel mt / 4.
+  const uint32_t v_lane =
+      static_cast<uint32_t>((w_tok0 + 8 * (mat >> 1) + mrow) * 128 + (((mat & 1) ^ mrow) << 4));
   uint32_t st = 0, ph = 0;  // ring slot and use parity of the next stage
 
   for (uint32_t k = 0;; ++k) {
@@ -489,220 +555,231 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2)) decode_kerne
     if (named_barrier_or(1, NW * 32, !arrived || info.s < 0)) break;
     const int h0 = info.kvh * G;
 
-    // q of the G heads, scaled into base-2 score units, in the score-step layout:
-    // vector c of lane li covers row elements [(c * LPT + li) * 8, +8).
-    float2 qf[G][VPL][4];
+    // Q as the A operand: lane holds head `quad`, dims 16 ks + 2 qc (+1) and the
+    // same + 8 (zero for rows >= G).
+    uint32_t qa[KS][2];
     {
-      const T* sq = reinterpret_cast<const T*>(smem + Tr::OFF_Q + slot * Tr::Q_BYTES);
+      const uint8_t* sq = smem + Tr::OFF_Q + slot * Tr::Q_BYTES + (quad * D + 2 * qc) * 2;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-#pragma unroll
-        for (int c = 0; c < VPL; ++c) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(sq + g * D + (c * LPT + li) * 8);
-          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 f = unpack2<T>(w4[j]);
-            qf[g][c][j] = make_float2(f.x * a.scale_log2, f.y * a.scale_log2);
-          }
-        }
+      for (int ks = 0; ks < KS; ++ks) {
+        qa[ks][0] = quad < G ? *reinterpret_cast<const uint32_t*>(sq + ks * 32) : 0u;
+        qa[ks][1] = quad < G ? *reinterpret_cast<const uint32_t*>(sq + ks * 32 + 16) : 0u;
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&item_empty[slot]);
 
-    float m_run = -CUDART_INF_F;  // running max of head my_h
-    float l_lane = 0.f;           // partial softmax sum of head my_h (p_writer lanes)
-    float2 acc[G][DPL / 2];
+    float m_run = -CUDART_INF_F;  // running max of head `quad` over this warp's tokens (base 2)
+    float l_lane = 0.f;           // sum of this lane's probabilities of head `quad`
+    // O^T accumulators: acc[mt][0], [1] = dim 16 mt + quad of heads 2 qc, 2 qc + 1;
+    // acc[mt][2], [3] = the same for dim + 8.
+    float acc[MT][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int kk = 0; kk < DPL / 2; ++kk) acc[g][kk] = make_float2(0.f, 0.f);
+    for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 
-    // One stage: scores of this warp's TPW tokens, online softmax, PV.  FULL
-    // stages (all TS tokens valid) skip the masking and the early exits.
-    auto stage = [&](const T* sK, const T* sV, int nv, auto full_tag) {
+    // One stage.  FULL stages (all TS tokens valid) skip the masking.
+    auto stage = [&](uint32_t sK, uint8_t* pV, int nv, auto full_tag) -> bool {
       constexpr bool FULL = decltype(full_tag)::value;
-      float sc[ROUNDS];
+      const uint32_t sV = sK + Tr::TILE_BYTES;
+      // ---- scores; even and odd k-steps accumulate apart (shorter chains)
+      float sacc[2][2][4];
 #pragma unroll
-      for (int r = 0; r < ROUNDS; ++r) {
-        const int tok = w_tok0 + r * TPR + tg;
-        const T* krow = sK + tok * D;
-        float2 part2[G];
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int g = 0; g < G; ++g) part2[g] = make_float2(0.f, 0.f);
+        for (int c = 0; c < 2; ++c) sacc[nt][c][0] = sacc[nt][c][1] = sacc[nt][c][2] = sacc[nt][c][3] = 0.f;
 #pragma unroll
-        for (int c = 0; c < VPL; ++c) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(krow + (c * LPT + li) * 8);
-          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+      for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 kf = unpack2<T>(w4[j]);
-#pragma unroll
-            for (int g = 0; g < G; ++g) part2[g] = ffma2(qf[g][c][j], kf, part2[g]);
-          }
+        for (int kp = 0; kp < KS / 2; ++kp) {
+          uint32_t kb[4];
+          ldmatrix_x4(kb, sK + (kp >> 1) * Tr::PANEL_BYTES + nt * 1024 + (k_lane ^ ((kp & 1) << 6)));
+          const uint32_t a0[4] = {qa[2 * kp][0], 0u, qa[2 * kp][1], 0u};
+          const uint32_t a1[4] = {qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u};
+          mma_16816<T>(sacc[nt][0], a0, kb[0], kb[1]);
+          mma_16816<T>(sacc[nt][1], a1, kb[2], kb[3]);
         }
-        float x[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) x[g] = part2[g].x + part2[g].y;
-        // reduce-scatter: each halving step keeps half of the heads
-#pragma unroll
-        for (int cnt = G, m = LPT / 2; cnt > 1; cnt >>= 1, m >>= 1) {
-          const bool upper = (li & m) != 0;
-#pragma unroll
-          for (int j = 0; j < cnt / 2; ++j) {
-            const float send = upper ? x[j] : x[j + cnt / 2];
-            const float keep = upper ? x[j + cnt / 2] : x[j];
-            x[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-          }
-        }
-        // the lanes of one head's group finish with a plain reduction
-#pragma unroll
-        for (int m = LPH / 2; m > 0; m >>= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], m);
-        if constexpr (FULL)
-          sc[r] = x[0];
-        else
-          sc[r] = tok < nv ? x[0] : -CUDART_INF_F;
       }
+      // x[nt][e]: head quad, token w_tok0 + 8 nt + 2 qc + e, in base-2 units
+      float x[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          x[nt][e] = (sacc[nt][0][e] + sacc[nt][1][e]) * a.scale_log2;
+          if constexpr (!FULL) {
+            if (w_tok0 + 8 * nt + 2 * qc + e >= nv) x[nt][e] = -CUDART_INF_F;
+          }
+        }
+      // this warp is done reading the K half
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_k[st]);
 
-      // online softmax for head my_h
-      float mx = sc[0];
-#pragma unroll
-      for (int r = 1; r < ROUNDS; ++r) mx = fmaxf(mx, sc[r]);
-#pragma unroll
-      for (int m = LPT; m < 32; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+      // ---- online softmax, per head over the quad's lanes
+      float mx = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
       const float m_new = fmaxf(m_run, mx);
       if (__any_sync(0xffffffffu, m_new > m_run)) {
         const float alpha = m_new == m_run ? 1.f : fast_exp2(m_run - m_new);  // 0 when m_run = -inf
         l_lane *= alpha;
+        // this lane's output columns are heads 2 qc and 2 qc + 1
+        const float a_lo = __shfl_sync(0xffffffffu, alpha, 8 * qc);
+        const float a_hi = __shfl_sync(0xffffffffu, alpha, 8 * qc + 4);
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float ag = __shfl_sync(0xffffffffu, alpha, g * LPH);
-          const float2 a2 = make_float2(ag, ag);
-#pragma unroll
-          for (int kk = 0; kk < DPL / 2; ++kk) acc[g][kk] = fmul2(acc[g][kk], a2);
+        for (int mt = 0; mt < MT; ++mt) {
+          acc[mt][0] *= a_lo;
+          acc[mt][1] *= a_hi;
+          acc[mt][2] *= a_lo;
+          acc[mt][3] *= a_hi;
         }
         m_run = m_new;
       }
+      float p[2][2];
 #pragma unroll
-      for (int r = 0; r < ROUNDS; ++r) {
-        float p;
-        if constexpr (FULL)
-          p = fast_exp2(sc[r] - m_run);
-        else
-          p = sc[r] == -CUDART_INF_F ? 0.f : fast_exp2(sc[r] - m_run);
-        if (p_writer) {
-          p_warp[(r * TPR + tg) * G + my_h] = make_float2(p, p);
-          l_lane += p;
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          if constexpr (FULL)
+            p[nt][e] = fast_exp2(x[nt][e] - m_run);
+          else
+            p[nt][e] = x[nt][e] == -CUDART_INF_F ? 0.f : fast_exp2(x[nt][e] - m_run);
+          l_lane += p[nt][e];
         }
+      // P^T as the B operand: k = token, n = head (rounded to the input type)
+      const uint32_t pb0 = pack2<T>(p[0][0], p[0][1]);
+      const uint32_t pb1 = pack2<T>(p[1][0], p[1][1]);
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_v[st], ph))) return false;
+      if constexpr (!FULL) {
+        // V rows past the end of the context hold whatever the pool or an
+        // earlier stage left there; zero them so that 0 * row stays 0.
+        const int r0 = max(nv, w_tok0);
+        const int n_zero = (w_tok0 + TPW - r0) * ND * 8;  // 16-byte chunks
+        for (int e = lane; e < n_zero; e += 32) {
+          const int row = r0 + e / (ND * 8), rem = e % (ND * 8);
+          *reinterpret_cast<uint4*>(pV + (rem >> 3) * Tr::PANEL_BYTES + row * 128 + (rem & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
       }
-      __syncwarp();
-
-      // PV over this warp's valid tokens
+      // ---- O^T += V^T P^T over this warp's 16 tokens
 #pragma unroll
-      for (int j = 0; j < TPW; ++j) {
-        if constexpr (!FULL) {
-          if (w_tok0 + j >= nv) break;
-        }
-        float2 pj[G];
-        if constexpr (G % 2 == 0) {
-#pragma unroll
-          for (int g = 0; g < G; g += 2) {
-            const float4 p4 = *reinterpret_cast<const float4*>(p_warp + j * G + g);
-            pj[g] = make_float2(p4.x, p4.y);
-            pj[g + 1] = make_float2(p4.z, p4.w);
-          }
-        } else {
-          pj[0] = p_warp[j * G];
-        }
-        const T* vrow = sV + (w_tok0 + j) * D + lane * DPL;
-        float2 vf[DPL / 2];
-        if constexpr (DPL == 4) {
-          const uint2 raw = *reinterpret_cast<const uint2*>(vrow);
-          vf[0] = unpack2<T>(raw.x);
-          vf[1] = unpack2<T>(raw.y);
-        } else {
-          vf[0] = unpack2<T>(*reinterpret_cast<const uint32_t*>(vrow));
-        }
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-          for (int kk = 0; kk < DPL / 2; ++kk) acc[g][kk] = ffma2(pj[g], vf[kk], acc[g][kk]);
+      for (int mt = 0; mt < MT; ++mt) {
+        uint32_t va[4];
+        ldmatrix_x4_trans(va, sV + (mt >> 2) * Tr::PANEL_BYTES + (v_lane ^ ((mt & 3) << 5)));
+        mma_16816<T>(acc[mt], va, pb0, pb1);
       }
+      // the zeroing stores must be ordered before the next bulk copy into this half
+      if constexpr (!FULL) fence_proxy_async_smem();
+      return true;
     };
 
     const int n_stages = (info.n_tok + TS - 1) / TS;
     bool ok = true;
     for (int i = 0; i < n_stages; ++i) {
-      if (!mbar_wait_bounded(&full[st], ph)) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_k[st], ph))) {
         if (lane == 0) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
         ok = false;
         break;
       }
-      const T* sK = reinterpret_cast<const T*>(smem + st * Tr::STAGE_BYTES);
-      const T* sV = sK + TS * D;
+      uint8_t* pK = smem + st * Tr::STAGE_BYTES;
+      const uint32_t sK = smem_addr(pK);
       const int nv = info.n_tok - i * TS;
-      if (nv >= TS)
-        stage(sK, sV, TS, std::true_type{});
-      else
-        stage(sK, sV, nv, std::false_type{});
+      const bool v_ok = nv >= TS ? stage(sK, pK + Tr::TILE_BYTES, TS, std::true_type{})
+                                 : stage(sK, pK + Tr::TILE_BYTES, nv, std::false_type{});
+      if (!v_ok) {
+        if (lane == 0) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+        ok = false;
+        break;
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
+      if (lane == 0) mbar_arrive(&empty_v[st]);
       if (++st == STAGES) {
         st = 0;
         ph ^= 1;
       }
     }
 
-    // ---- merge the four warps of this item, HG heads per round
-#pragma unroll
-    for (int m = LPT; m < 32; m <<= 1) l_lane += __shfl_xor_sync(0xffffffffu, l_lane, m);
-    if (tg == 0 && p_writer) {
-      s_m[warp * G + my_h] = m_run;
-      s_l[warp * G + my_h] = l_lane;
+    // ---- combine the four warps: weight of warp w for head g is
+    // 2^(m_w - M) / L with M = max_w m_w and L = sum_w 2^(m_w - M) l_w.
+    l_lane += __shfl_xor_sync(0xffffffffu, l_lane, 1);
+    l_lane += __shfl_xor_sync(0xffffffffu, l_lane, 2);
+    if (qc == 0 && quad < G) {
+      s_m[warp * G + quad] = m_run;
+      s_l[warp * G + quad] = l_lane;
     }
     if (named_barrier_or(1, NW * 32, !ok)) break;  // a timed-out stage: stop, output invalid
 
     const int s = info.s;
     const bool single = info.n_parts == 1;
+    float f_own = 0.f;  // this warp's weight for head `quad`
+    if (quad < G) {
+      float M = -CUDART_INF_F;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * G + quad]);
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float mw = s_m[w * G + quad];
+        L += mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M) * s_l[w * G + quad];
+      }
+      if (L > 0.f && m_run != -CUDART_INF_F) f_own = fast_exp2(m_run - M) / L;
+      if (!single && warp == 0 && qc == 0) {
+        const int64_t cell =
+            (static_cast<int64_t>(s) * a.num_heads + h0 + quad) * a.max_parts + info.part;
+        a.tmp_m[cell] = M;
+        a.tmp_l[cell] = L;
+      }
+    }
+    const float f_lo = __shfl_sync(0xffffffffu, f_own, 8 * qc);
+    const float f_hi = __shfl_sync(0xffffffffu, f_own, 8 * qc + 4);
+    // Rounds of HG heads: each warp stores its weighted partial output into its
+    // own slot, then the slots are summed in warp order (the same order every
+    // run) and written out, four dims per thread.
     constexpr int HG = Tr::HG;
+    float* my_slot = s_acc + warp * HG * Tr::ACC_PITCH;
 #pragma unroll
     for (int r = 0; r < G / HG; ++r) {
-      if (r > 0) named_barrier_sync(1, NW * 32);  // previous round's reads are done
+      if (r > 0) named_barrier_sync(1, NW * 32);  // the previous round's slots are read
+      const int g_lo = 2 * qc - r * HG;          // this lane's heads, relative to the round
 #pragma unroll
-      for (int gg = 0; gg < HG; ++gg)
+      for (int j = 0; j < 2; ++j) {
+        const int gg = g_lo + j;
+        if (2 * qc + j < G && gg >= 0 && gg < HG) {
+          const float f = j ? f_hi : f_lo;
+          float* row = my_slot + gg * Tr::ACC_PITCH + quad;
 #pragma unroll
-        for (int kk = 0; kk < DPL / 2; ++kk)
-          *reinterpret_cast<float2*>(s_acc + (warp * HG + gg) * D + lane * DPL + 2 * kk) = acc[r * HG + gg][kk];
-      named_barrier_sync(1, NW * 32);
-      for (int idx = threadIdx.x; idx < HG * D; idx += NW * 32) {
-        const int gg = idx / D, d = idx % D;
-        const int g = r * HG + gg;
-        float M = -CUDART_INF_F;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w * G + g]);
-        float lsum = 0.f, o = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          const float mw = s_m[w * G + g];
-          const float f = mw == -CUDART_INF_F ? 0.f : fast_exp2(mw - M);
-          lsum += f * s_l[w * G + g];
-          o += f * s_acc[(w * HG + gg) * D + d];
-        }
-        if (single) {
-          static_cast<T*>(a.out)[(static_cast<int64_t>(s) * a.num_heads + h0 + g) * D + d] =
-              from_float<T>(lsum > 0.f ? o / lsum : 0.f);
-        } else {
-          const int64_t cell = (static_cast<int64_t>(s) * a.num_heads + h0 + g) * a.max_parts + info.part;
-          a.tmp_out[cell * D + d] = o / lsum;
-          if (d == 0) {
-            a.tmp_m[cell] = M;
-            a.tmp_l[cell] = lsum;
+          for (int mt = 0; mt < MT; ++mt) {
+            row[16 * mt] = acc[mt][j] * f;
+            row[16 * mt + 8] = acc[mt][2 + j] * f;
           }
         }
       }
+      named_barrier_sync(1, NW * 32);
+      for (int e = threadIdx.x; e < HG * D / 4; e += NW * 32) {
+        const int gg = e / (D / 4), d = (e % (D / 4)) * 4;
+        const int g = r * HG + gg;
+        float4 o = *reinterpret_cast<const float4*>(s_acc + gg * Tr::ACC_PITCH + d);
+#pragma unroll
+        for (int w = 1; w < NW; ++w) {
+          const float4 t = *reinterpret_cast<const float4*>(s_acc + (w * HG + gg) * Tr::ACC_PITCH + d);
+          o.x += t.x;
+          o.y += t.y;
+          o.z += t.z;
+          o.w += t.w;
+        }
+        if (single) {
+          const uint2 packed = make_uint2(pack2<T>(o.x, o.y), pack2<T>(o.z, o.w));
+          *reinterpret_cast<uint2*>(static_cast<T*>(a.out) +
+                                    (static_cast<int64_t>(s) * a.num_heads + h0 + g) * D + d) = packed;
+        } else {
+          const int64_t cell =
+              (static_cast<int64_t>(s) * a.num_heads + h0 + g) * a.max_parts + info.part;
+          *reinterpret_cast<float4*>(a.tmp_out + cell * D + d) = o;
+        }
+      }
     }
-    named_barrier_sync(1, NW * 32);  // s_acc, s_m, s_l are free again
+    // The slots and s_m / s_l are rewritten only after the next item's first
+    // barrier, which every thread reaches after its reads here.
   }
 }
 
@@ -816,7 +893,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
 
 // Host-side launcher, instantiated per (dtype, head_dim) in its own file.
 template <typename T, int D>
-cudaError_t launch_decode(const DecodeArgs& a, int group, int block_size, bool paged, int num_sms,
-                          cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, int group, int block_size,
+                          bool paged, int num_sms, cudaStream_t stream);
 
 }  // namespace pkv

@@ -2,5 +2,6 @@
 #include "decode_launch.cuh"
 
 namespace pkv {
-template cudaError_t launch_decode<__nv_bfloat16, 64>(const DecodeArgs&, int, int, bool, int, cudaStream_t);
+template cudaError_t launch_decode<__nv_bfloat16, 64>(const DecodeArgs&, const DecodeMaps&, int, int,
+                                           bool, int, cudaStream_t);
 }  // namespace pkv

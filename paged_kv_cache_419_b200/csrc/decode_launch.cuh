@@ -31,7 +31,8 @@ cudaError_t decode_grid(int num_sms, int* grid) {
 }
 
 template <typename T, int D, int G, int B, bool PAGED>
-cudaError_t launch_decode_one(const DecodeArgs& args, int num_sms, cudaStream_t stream) {
+cudaError_t launch_decode_one(const DecodeArgs& args, const DecodeMaps& maps, int num_sms,
+                              cudaStream_t stream) {
   using Tr = DecodeTraits<T, D, G, B, PAGED>;
   int grid = 0;
   cudaError_t e = decode_grid<T, D, G, B, PAGED>(num_sms, &grid);
@@ -56,7 +57,7 @@ cudaError_t launch_decode_one(const DecodeArgs& args, int num_sms, cudaStream_t 
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kDecodeThreads);
   cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<T, D, G, B, PAGED>, a);
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<T, D, G, B, PAGED>, a, maps);
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess || a.max_parts <= 1) return e;
@@ -73,24 +74,25 @@ cudaError_t launch_decode_one(const DecodeArgs& args, int num_sms, cudaStream_t 
 }
 
 template <typename T, int D, int B, bool PAGED>
-cudaError_t launch_decode_group(const DecodeArgs& a, int group, int num_sms, cudaStream_t stream) {
+cudaError_t launch_decode_group(const DecodeArgs& a, const DecodeMaps& m, int group, int num_sms,
+                               cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_decode_one<T, D, 1, B, PAGED>(a, num_sms, stream);
-    case 2: return launch_decode_one<T, D, 2, B, PAGED>(a, num_sms, stream);
-    case 4: return launch_decode_one<T, D, 4, B, PAGED>(a, num_sms, stream);
-    case 8: return launch_decode_one<T, D, 8, B, PAGED>(a, num_sms, stream);
+    case 1: return launch_decode_one<T, D, 1, B, PAGED>(a, m, num_sms, stream);
+    case 2: return launch_decode_one<T, D, 2, B, PAGED>(a, m, num_sms, stream);
+    case 4: return launch_decode_one<T, D, 4, B, PAGED>(a, m, num_sms, stream);
+    case 8: return launch_decode_one<T, D, 8, B, PAGED>(a, m, num_sms, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <typename T, int D>
-cudaError_t launch_decode(const DecodeArgs& a, int group, int block_size, bool paged, int num_sms,
-                          cudaStream_t stream) {
-  if (!paged) return launch_decode_group<T, D, 32, false>(a, group, num_sms, stream);
+cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, int group, int block_size,
+                          bool paged, int num_sms, cudaStream_t stream) {
+  if (!paged) return launch_decode_group<T, D, 32, false>(a, m, group, num_sms, stream);
   switch (block_size) {
-    case 8: return launch_decode_group<T, D, 8, true>(a, group, num_sms, stream);
-    case 16: return launch_decode_group<T, D, 16, true>(a, group, num_sms, stream);
-    case 32: return launch_decode_group<T, D, 32, true>(a, group, num_sms, stream);
+    case 8: return launch_decode_group<T, D, 8, true>(a, m, group, num_sms, stream);
+    case 16: return launch_decode_group<T, D, 16, true>(a, m, group, num_sms, stream);
+    case 32: return launch_decode_group<T, D, 32, true>(a, m, group, num_sms, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -1,12 +1,15 @@
-// Device helpers shared by the kernels: shared-memory barriers, 1-D bulk
-// copies global -> shared (the sm_90+/sm_100 bulk-copy engine, no tensor map),
-// bounded waits, packed fp32 math and fp16/bf16 unpacking.
+// Device helpers shared by the kernels: shared-memory barriers, 1-D bulk and
+// tiled tensor (TMA) copies global -> shared, bounded waits, warp-level
+// tensor-core tiles (ldmatrix + mma.sync), packed fp32 math and fp16/bf16
+// packing and unpacking.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "pkv.h"
 
@@ -173,6 +176,74 @@ __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) {
 template <>
 __device__ __forceinline__ __half from_float<__half>(float x) {
   return __float2half_rn(x);
+}
+
+// Tiled 3-D tensor copy global -> shared through a tensor map (TMA): the box at
+// element coordinates (x, y, z) lands at dst_smem in the map's swizzled layout;
+// completion is signalled as transaction bytes (the whole box, out-of-range
+// elements zero-filled) on `bar`.  x must be a multiple of 8 (16 bytes).
+__device__ __forceinline__ void tma_load_3d(void* dst_smem, const void* tmap, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst_smem)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensor_map(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+// Four 8x8 16-bit matrices from shared memory; lane l supplies the address of
+// row l % 8 of matrix l / 8 and receives, of matrix i, row l / 4, columns
+// 2 (l % 4) and 2 (l % 4) + 1 in r[i] (low half first).
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+// As ldmatrix_x4, transposed: lane l receives, of matrix i, rows 2 (l % 4) and
+// 2 (l % 4) + 1 of column l / 4.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
+// d += A (16x16, row) * B (16x8, col) with 16-bit inputs of type T and fp32
+// accumulation (warp-wide tensor-core instruction).
+template <typename T>
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+  if constexpr (std::is_same<T, __half>::value) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+        " {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7},"
+        " {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+// Two floats -> two packed 16-bit values of type T (lo in the low half), round to nearest.
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (std::is_same<T, __half>::value) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  } else {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
 }
 
 __device__ __forceinline__ void set_error(unsigned int* err, unsigned int bit) {
