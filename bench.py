@@ -49,6 +49,18 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
 
+def l2_flush(buf, mode: str):
+    """Evict the 126 MB L2 before a timed step by writing a 256 MiB buffer.
+
+    mode "clean" then reads the buffer back, so that the L2 holds clean lines
+    only and the timed step does not pay for writing the flush buffer's dirty
+    lines back to HBM; "dirty" leaves them (the write alone).
+    """
+    buf.zero_()
+    if mode == "clean":
+        buf.view(torch.int32).sum()
+
+
 # ------------------------------------------------------------------ helpers
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -57,6 +69,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="gqa8b", choices=["tiny", "mha13b", "gqa8b", "long"])
+    ap.add_argument("--l2-flush", choices=["clean", "dirty"], default="clean",
+                    help="L2 eviction before each timed step: 256 MiB write then read (clean) or write only")
     ap.add_argument("--block-size", type=int, default=0, help="override the workload's block size")
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--num-seqs", type=int, default=0,
@@ -314,7 +328,7 @@ def run_ours(args, world, rank, local):
         barrier()
         torch.cuda.synchronize()
         for k in range(K):
-            flush.zero_()
+            l2_flush(flush, args.l2_flush)
             evs[k][0].record()
             run_write()
             evs[k][1].record()
@@ -325,7 +339,7 @@ def run_ours(args, world, rank, local):
         return ([e[0].elapsed_time(e[2]) for e in evs], [e[1].elapsed_time(e[2]) for e in evs])
 
     for _ in range(max(args.warmup, 0)):
-        flush.zero_()
+        l2_flush(flush, args.l2_flush)
         write_step()
         decode_step()
     torch.cuda.synchronize()
@@ -346,7 +360,7 @@ def run_ours(args, world, rank, local):
             decode_step()
         torch.cuda.current_stream().wait_stream(side)
         for _ in range(2):
-            flush.zero_()
+            l2_flush(flush, args.l2_flush)
             g_write.replay()
             g_decode.replay()
         torch.cuda.synchronize()
@@ -380,7 +394,9 @@ def run_ours(args, world, rank, local):
             "num_seqs_per_gpu": w.num_seqs, "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "block_size": w.block_size, "num_blocks": w.num_blocks,
             "context_tokens_per_gpu": int(inp.context_lens.sum()), "partition_size": part,
-            "l2": "flushed before every timed step (256 MiB write); K/V read per step > L2",
+            "l2": ("flushed before every timed step (256 MiB write, read back so no dirty lines remain)"
+                   if args.l2_flush == "clean" else "flushed before every timed step (256 MiB write)")
+                  + "; K/V read per step > L2",
             "execution": mode,
             "parallelism": f"dp{world} (sequences sharded, no collective)",
         },
@@ -422,7 +438,7 @@ def contiguous_compare(args, inp, b, ws, flush, part, device):
 
     def time_it(fn):
         for _ in range(3):
-            flush.zero_()
+            l2_flush(flush, args.l2_flush)
             fn()
         torch.cuda.synchronize()
         if not args.eager:
@@ -433,11 +449,11 @@ def contiguous_compare(args, inp, b, ws, flush, part, device):
                 fn()
             torch.cuda.current_stream().wait_stream(side)
             fn = g.replay
-            flush.zero_()
+            l2_flush(flush, args.l2_flush)
             fn()
         evs = []
         for _ in range(K):
-            flush.zero_()
+            l2_flush(flush, args.l2_flush)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             fn()

@@ -74,6 +74,7 @@ pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t str
 /*
  * Bytes of workspace the decode calls need (always > 0 for valid arguments):
  * 256 bytes of work counters, 4 * num_seqs bytes of sequence list,
+ * 4 * num_seqs * num_heads bytes of per-(sequence, kv head) completion counters,
  * 32 * num_seqs * P bytes of work records (one per context partition), and, when
  * P > 1, the partition results num_seqs * num_heads * P * (head_dim + 2) * 4
  * bytes; each piece rounded up to 256 bytes, with
@@ -112,7 +113,11 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t h
  *
  * Launches, in this order on `stream`: a one-CTA planning kernel (work list),
  * the persistent decode kernel and, when a context can span more than one
- * partition, the partition merge kernel (both with programmatic dependent launch).
+ * partition, the partition merge kernel (both with programmatic dependent
+ * launch).  The merge kernel starts while the decode grid drains and merges
+ * each (sequence, kv head) as soon as the decode grid has published all of its
+ * partitions; it completes after the decode grid, so work that follows on the
+ * stream sees the whole of `out`.
  */
 pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
                                       const void* v_cache, const int32_t* block_tables,

@@ -66,9 +66,10 @@ bool valid_partition(int p) { return p >= kStageTokens && p <= kMaxPartTokens &&
 int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
 
 // Workspace layout: [work counters | list of multi-partition sequences (S) |
-// work records (S x P) | partition results (only when P > 1)].
+// published partitions per (sequence, kv head) (S x Hkv <= S x Hq) | work
+// records (S x P) | partition results (only when P > 1)].
 struct WorkspaceLayout {
-  int64_t counters, merge, records, tmp, total;
+  int64_t counters, merge, done, records, tmp, total;
 };
 
 WorkspaceLayout workspace_layout(int64_t S, int64_t Hq, int64_t D, int64_t max_ctx, int64_t part) {
@@ -77,7 +78,8 @@ WorkspaceLayout workspace_layout(int64_t S, int64_t Hq, int64_t D, int64_t max_c
   WorkspaceLayout w;
   w.counters = 0;
   w.merge = 256;
-  w.records = w.merge + round256(4 * S);
+  w.done = w.merge + round256(4 * S);
+  w.records = w.done + round256(4 * S * Hq);
   w.tmp = w.records + round256(S * P * kRecordBytes);
   w.total = w.tmp + (P > 1 ? round256(S * Hq * P * (D + 2) * 4) : 0);
   return w;
@@ -162,6 +164,7 @@ pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pk
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.work = reinterpret_cast<uint32_t*>(ws + lay.counters);
   a.merge_seqs = reinterpret_cast<int32_t*>(ws + lay.merge);
+  a.pair_done = reinterpret_cast<uint32_t*>(ws + lay.done);
   a.records = ws + lay.records;
   a.block_size = block_size;
   if (a.max_parts > 1) {

@@ -64,6 +64,7 @@ struct DecodeArgs {
   float scale_log2;       // scale * log2(e)
   int32_t grid_ctas;      // decode CTAs; item c (c < grid_ctas) is CTA c's first item
   uint32_t* work;         // [0] next item, [1] item count, [2] multi-partition sequences
+  uint32_t* pair_done;    // [S * Hkv] partitions published per (sequence, kv head)
   int32_t* merge_seqs;    // [S] sequences whose context spans more than one partition
   uint8_t* records;       // [S * max_parts] work records, largest partition first (32 B each)
   float* tmp_out;         // [S, Hq, max_parts, D]
@@ -79,6 +80,9 @@ constexpr int kPlanThreads = 1024;
 constexpr int kItemSlots = 2;
 constexpr int kRecSlots = 2;   // records of items k and k+1
 constexpr int kStageTokens = 64;
+// Multi-partition items a CTA finishes before it publishes them (one fence for
+// the lot) to the merge grid; a full list is published at the next item.
+constexpr int kPubSlots = 32;
 // Work record of one (sequence, partition): int32 s, part, n_parts, t_begin,
 // n_tok, L, 0, 0.
 constexpr int kRecordBytes = 32;
@@ -146,7 +150,8 @@ struct DecodeTraits {
   static constexpr int OFF_TAB = OFF_REC + kRecSlots * kRecordBytes;    // 2 table buffers
   static constexpr int OFF_STAT = OFF_TAB + 2 * MAX_TABLE * 4;          // m, l per warp and head
   static constexpr int OFF_ITEM = OFF_STAT + 2 * kConsumerWarps * G * 4 + 16;
-  static constexpr int OFF_BARS = OFF_ITEM + kItemSlots * 32;
+  static constexpr int OFF_PUB = OFF_ITEM + kItemSlots * 32;           // pairs awaiting publication
+  static constexpr int OFF_BARS = OFF_PUB + (kPubSlots + 2) * 4;
   static constexpr int SMEM_USED = OFF_BARS + (4 * STAGES + 2 * kItemSlots + kRecSlots + 2) * 8;
   static constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for aligning the base
 
@@ -208,7 +213,10 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
     partition_of(L, a.part_tokens, n, size);
     for (int p = 0; p < n; ++p) atomicAdd(&count[size_class(min(size, L - p * size))], 1u);
     atomicAdd(&total, static_cast<uint32_t>(n));
-    if (n > 1) a.merge_seqs[atomicAdd(&n_multi, 1u)] = s;
+    if (n > 1) {
+      a.merge_seqs[atomicAdd(&n_multi, 1u)] = s;
+      for (int h = 0; h < a.num_kv_heads; ++h) a.pair_done[s * a.num_kv_heads + h] = 0u;
+    }
   }
   __syncthreads();
   if (threadIdx.x < 32) {  // exclusive scan of the class counts, one warp
@@ -282,6 +290,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
   float* s_acc = reinterpret_cast<float*>(smem + Tr::OFF_ACC);
   float* s_m = reinterpret_cast<float*>(smem + Tr::OFF_STAT);
   float* s_l = s_m + NW * G;
+  uint32_t* s_pub = reinterpret_cast<uint32_t*>(smem + Tr::OFF_PUB);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -305,6 +314,9 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
   __syncthreads();
   // Everything below reads what the plan kernel wrote.
   grid_dependency_wait();
+  // The merge grid may launch now: it reads what the plan wrote and waits per
+  // (sequence, kv head) for the partitions this grid publishes.
+  allow_dependent_launch();
 
   // ================================================================ producer
   // Item k (the k-th item this CTA takes).  The CTA's first item is item
@@ -546,13 +558,29 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
   const uint32_t v_lane =
       static_cast<uint32_t>((w_tok0 + 8 * (mat >> 1) + mrow) * 128 + (((mat & 1) ^ mrow) << 4));
   uint32_t st = 0, ph = 0;  // ring slot and use parity of the next stage
+  // Publication (thread 0): partial results of multi-partition items are
+  // announced to the merge grid by one gpu-scope fence followed by one counter
+  // increment per item.  The fence is cumulative over the other consumer
+  // threads' writes, which a named barrier ordered before it; batching makes it
+  // one fence per kPubSlots items instead of one per item.
+  // s_pub[kPubSlots] holds the count (thread 0 alone touches the list).
+  if (threadIdx.x == 0) s_pub[kPubSlots] = 0u;
+  auto publish = [&]() {
+    const uint32_t n = s_pub[kPubSlots];
+    if (n == 0) return;
+    __threadfence();
+    for (uint32_t i = 0; i < n; ++i) atomicAdd(&a.pair_done[s_pub[i]], 1u);
+    s_pub[kPubSlots] = 0u;
+  };
 
   for (uint32_t k = 0;; ++k) {
     const int slot = k & (kItemSlots - 1);
     const bool arrived = mbar_wait_bounded(&item_full[slot], (k / kItemSlots) & 1);
     if (!arrived && lane == 0) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
     const ItemInfo info = items[slot];
+    // Every consumer thread has finished the previous item's write-out here.
     if (named_barrier_or(1, NW * 32, !arrived || info.s < 0)) break;
+    if (threadIdx.x == 0 && s_pub[kPubSlots] == kPubSlots) publish();
     const int h0 = info.kvh * G;
 
     // Q as the A operand: lane holds head `quad`, dims 16 ks + 2 qc (+1) and the
@@ -581,22 +609,20 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
     auto stage = [&](uint32_t sK, uint8_t* pV, int nv, auto full_tag) -> bool {
       constexpr bool FULL = decltype(full_tag)::value;
       const uint32_t sV = sK + Tr::TILE_BYTES;
-      // ---- scores; even and odd k-steps accumulate apart (shorter chains)
-      float sacc[2][2][4];
+      // ---- scores, one accumulation chain per 8-token n-tile
+      float sacc[2][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) sacc[nt][c][0] = sacc[nt][c][1] = sacc[nt][c][2] = sacc[nt][c][3] = 0.f;
+      for (int kp = 0; kp < KS / 2; ++kp) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-        for (int kp = 0; kp < KS / 2; ++kp) {
+        for (int nt = 0; nt < 2; ++nt) {
           uint32_t kb[4];
           ldmatrix_x4(kb, sK + (kp >> 1) * Tr::PANEL_BYTES + nt * 1024 + (k_lane ^ ((kp & 1) << 6)));
           const uint32_t a0[4] = {qa[2 * kp][0], 0u, qa[2 * kp][1], 0u};
           const uint32_t a1[4] = {qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u};
-          mma_16816<T>(sacc[nt][0], a0, kb[0], kb[1]);
-          mma_16816<T>(sacc[nt][1], a1, kb[2], kb[3]);
+          mma_16816<T>(sacc[nt], a0, kb[0], kb[1]);
+          mma_16816<T>(sacc[nt], a1, kb[2], kb[3]);
         }
       }
       // x[nt][e]: head quad, token w_tok0 + 8 nt + 2 qc + e, in base-2 units
@@ -605,7 +631,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          x[nt][e] = (sacc[nt][0][e] + sacc[nt][1][e]) * a.scale_log2;
+          x[nt][e] = sacc[nt][e] * a.scale_log2;
           if constexpr (!FULL) {
             if (w_tok0 + 8 * nt + 2 * qc + e >= nv) x[nt][e] = -CUDART_INF_F;
           }
@@ -711,6 +737,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
 
     const int s = info.s;
     const bool single = info.n_parts == 1;
+    if (threadIdx.x == 0 && !single)
+      s_pub[s_pub[kPubSlots]++] = static_cast<uint32_t>(s * a.num_kv_heads + info.kvh);
     float f_own = 0.f;  // this warp's weight for head `quad`
     if (quad < G) {
       float M = -CUDART_INF_F;
@@ -781,6 +809,9 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
     // The slots and s_m / s_l are rewritten only after the next item's first
     // barrier, which every thread reaches after its reads here.
   }
+  // Every loop exit follows a barrier that all consumer threads passed after
+  // their last write-out (or a stage timeout, whose item is not listed).
+  if (threadIdx.x == 0) publish();
 }
 
 // ---------------------------------------------------------------- merge
@@ -800,17 +831,29 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a) {
   __shared__ float s_m[G][kMergeStat], s_l[G][kMergeStat], s_w[G][kPre];
   __shared__ float s_M[G], s_L[G];
-  grid_dependency_wait();
+  __shared__ int s_ready;
   constexpr int kPer = (G * D + kMergeThreads - 1) / kMergeThreads;
   const uint32_t Hkv = static_cast<uint32_t>(a.num_kv_heads);
-  const uint32_t n_tasks = a.work[2] * Hkv;
+  // The plan finished before the decode grid let this grid launch.
+  const uint32_t n_tasks = __ldcg(a.work + 2) * Hkv;
   for (uint32_t t = blockIdx.x; t < n_tasks; t += gridDim.x) {
-    const int s = a.merge_seqs[t / Hkv];
-    const int h0 = static_cast<int>(t % Hkv) * G;
+    const int s = __ldcg(a.merge_seqs + t / Hkv);
+    const int kvh = static_cast<int>(t % Hkv);
+    const int h0 = kvh * G;
     int np, psize;
     partition_of(clamp_len(a.lens[s], a.max_ctx), a.part_tokens, np, psize);
     const int64_t base0 = (static_cast<int64_t>(s) * a.num_heads + h0) * a.max_parts;
     auto cell = [&](int g, int p) { return base0 + static_cast<int64_t>(g) * a.max_parts + p; };
+    // Wait (bounded) until the decode grid has published all np partitions of
+    // this pair; their results are then read from L2 (__ldcg), never from a
+    // possibly stale L1 line.
+    if (threadIdx.x == 0) {
+      s_ready = wait_counter_bounded(a.pair_done + static_cast<int64_t>(s) * Hkv + kvh,
+                                     static_cast<uint32_t>(np), a.err);
+      if (!s_ready) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+    }
+    __syncthreads();
+    if (!s_ready) continue;  // uniform: results of this pair stay unwritten
 
     float pre[kPre][kPer];  // outputs of partitions 0 .. kPre-1
 #pragma unroll
@@ -818,7 +861,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
         const int idx = threadIdx.x + k * kMergeThreads;
-        pre[p][k] = (p < np && idx < G * D) ? a.tmp_out[cell(idx / D, p) * D + idx % D] : 0.f;
+        pre[p][k] = (p < np && idx < G * D) ? __ldcg(a.tmp_out + cell(idx / D, p) * D + idx % D) : 0.f;
       }
 
     // M and the normaliser per head, online over rounds of kMergeStat partitions
@@ -830,8 +873,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
       const int cn = min(kMergeStat, np - c0);
       for (int i = threadIdx.x; i < G * cn; i += kMergeThreads) {
         const int g = i / cn, p = i % cn;
-        s_m[g][p] = a.tmp_m[cell(g, c0 + p)];
-        s_l[g][p] = a.tmp_l[cell(g, c0 + p)];
+        s_m[g][p] = __ldcg(a.tmp_m + cell(g, c0 + p));
+        s_l[g][p] = __ldcg(a.tmp_l + cell(g, c0 + p));
       }
       __syncthreads();
       if (threadIdx.x < G) {
@@ -853,7 +896,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
       const int pc = min(kPre, np - p0);
       if (threadIdx.x < G * pc) {
         const int g = threadIdx.x / pc, p = threadIdx.x % pc;
-        s_w[g][p] = a.tmp_l[cell(g, p0 + p)] * fast_exp2(a.tmp_m[cell(g, p0 + p)] - s_M[g]) / s_L[g];
+        s_w[g][p] = __ldcg(a.tmp_l + cell(g, p0 + p)) * fast_exp2(__ldcg(a.tmp_m + cell(g, p0 + p)) - s_M[g]) / s_L[g];
       }
       if (p0 > 0) {
 #pragma unroll
@@ -861,7 +904,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
 #pragma unroll
           for (int k = 0; k < kPer; ++k) {
             const int idx = threadIdx.x + k * kMergeThreads;
-            pre[p][k] = (p < pc && idx < G * D) ? a.tmp_out[cell(idx / D, p0 + p) * D + idx % D] : 0.f;
+            pre[p][k] = (p < pc && idx < G * D) ? __ldcg(a.tmp_out + cell(idx / D, p0 + p) * D + idx % D) : 0.f;
           }
       }
       __syncthreads();
@@ -889,6 +932,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
       }
     }
   }
+  // Complete only after the decode grid: work behind this grid on the stream
+  // then sees every output row, including the single-partition ones.
+  grid_dependency_wait();
 }
 
 // Host-side launcher, instantiated per (dtype, head_dim) in its own file.

@@ -88,6 +88,29 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return true;
 }
 
+// Load with gpu-scope acquire semantics.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until *counter >= target (each read a gpu-scope acquire).  False after
+// kWaitLimitNs, or at once when another wait has already timed out
+// (PKV_DEVERR_WAIT_TIMEOUT set in *err): the work it was waiting for will not come.
+__device__ __forceinline__ bool wait_counter_bounded(const uint32_t* counter, uint32_t target,
+                                                     const unsigned int* err) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (;;) {
+    __nanosleep(200);
+    if (ld_acquire_gpu(counter) >= target) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (err && (*reinterpret_cast<const volatile unsigned int*>(err) & PKV_DEVERR_WAIT_TIMEOUT))
+      return false;
+  }
+}
+
 // Order this thread's earlier generic-proxy accesses to shared memory before
 // its later async-proxy (bulk copy) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -38,7 +38,7 @@ def _layout_bytes(S, Hq, D, ctx, part=512):
     r = lambda x: (x + 255) // 256 * 256
     P = max(1, -(-ctx // part))
     rec = 32
-    return 256 + r(4 * S) + r(S * P * rec) + (r(S * Hq * P * (D + 2) * 4) if P > 1 else 0)
+    return 256 + r(4 * S) + r(4 * S * Hq) + r(S * P * rec) + (r(S * Hq * P * (D + 2) * 4) if P > 1 else 0)
 
 
 def test_workspace_bytes_formula():
