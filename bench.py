@@ -72,7 +72,7 @@ def parse_args(argv=None):
     ap.add_argument("--l2-flush", choices=["clean", "dirty"], default="clean",
                     help="L2 eviction before each timed step: 256 MiB write then read (clean) or write only")
     ap.add_argument("--block-size", type=int, default=0, help="override the workload's block size")
-    ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--partition", type=int, default=1024)
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="smaller batch of the same length law, pool sized to fit (profiling)")
     ap.add_argument("--no-contiguous", action="store_true")
@@ -346,31 +346,53 @@ def run_ours(args, world, rank, local):
     if pkv.device_error():
         raise RuntimeError("device error flags set during warm-up")
 
+    def timed_graph(g, evs, K):
+        # One replay per step; the events are nodes of the graph, so they are
+        # read after each replay (the host waits between steps, the GPU clock
+        # only runs inside the replay).
+        step, dec = [], []
+        barrier()
+        torch.cuda.synchronize()
+        for _ in range(K):
+            l2_flush(flush, args.l2_flush)
+            g.replay()
+            torch.cuda.synchronize()
+            step.append(evs[0].elapsed_time(evs[2]))
+            dec.append(evs[1].elapsed_time(evs[2]))
+        barrier()
+        return step, dec
+
     eager_step_ms, _ = timed_steps(write_step, decode_step, min(args.steps, 5))
+    K = args.steps
     if args.eager:
-        run_write, run_decode, mode = write_step, decode_step, "eager launches"
+        mode = "eager launches"
+        run = lambda: timed_steps(write_step, decode_step, K)
     else:
-        # A serving engine replays the decode step as a CUDA graph; so does the bench.
+        # A serving engine replays its whole decode step as one CUDA graph; so
+        # does the bench: cache write then decode, with timing events recorded
+        # as nodes of the graph (before the write, between, after the decode).
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
-        g_write, g_decode = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_write, stream=side):
+        g_step = torch.cuda.CUDAGraph()
+        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+        with torch.cuda.graph(g_step, stream=side):
+            gev[0].record()
             write_step()
-        with torch.cuda.graph(g_decode, stream=side):
+            gev[1].record()
             decode_step()
+            gev[2].record()
         torch.cuda.current_stream().wait_stream(side)
         for _ in range(2):
             l2_flush(flush, args.l2_flush)
-            g_write.replay()
-            g_decode.replay()
+            g_step.replay()
         torch.cuda.synchronize()
-        run_write, run_decode, mode = g_write.replay, g_decode.replay, "CUDA graph replay"
+        mode = "CUDA graph replay (cache write + decode in one graph, events as graph nodes)"
+        run = lambda: timed_graph(g_step, gev, K)
 
-    K = args.steps
     sampler = ClockSampler(local) if rank == 0 else None
     if sampler:
         sampler.start()
-    step_ms, decode_ms = timed_steps(run_write, run_decode, K)
+    step_ms, decode_ms = run()
     clocks = sampler.stop() if sampler else None
     if pkv.device_error():
         raise RuntimeError("device error flags set during the timed steps")

@@ -78,7 +78,7 @@ pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t str
  * 32 * num_seqs * P bytes of work records (one per context partition), and, when
  * P > 1, the partition results num_seqs * num_heads * P * (head_dim + 2) * 4
  * bytes; each piece rounded up to 256 bytes, with
- * P = ceil(max_context_len / partition_size).  partition_size 0 = default (512).
+ * P = ceil(max_context_len / partition_size).  partition_size 0 = default (1024).
  * Returns 0 for invalid arguments; the decode call then rejects them.
  */
 size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
@@ -102,7 +102,7 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t h
  *   block_tables device int32 [num_seqs, max_blocks_per_seq]; only the first
  *                ceil(context_lens[s] / block_size) entries of row s are read
  *   context_lens device int32 [num_seqs], 0 <= context_lens[s] <= max_blocks_per_seq * block_size
- *   partition_size maximum tokens per context partition (0 = 512); a multiple of 64
+ *   partition_size maximum tokens per context partition (0 = 1024); a multiple of 64
  *                in [64, 2048].  A context of L tokens is split into ceil(L / partition_size)
  *                near-equal partitions (multiples of 64 tokens) that run on different
  *                CTAs and are merged with a log-sum-exp in the same launch sequence.

@@ -17,7 +17,7 @@ static __device__ unsigned int g_device_error;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kDefaultPartition = 512;
+constexpr int kDefaultPartition = 1024;
 
 struct DeviceInfo {
   bool ready = false;

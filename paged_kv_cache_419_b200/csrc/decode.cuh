@@ -101,6 +101,15 @@ __device__ __forceinline__ void partition_of(int L, int part_tokens, int& n, int
   n = (L + size - 1) / size;
 }
 
+// Sequences whose partition 0 runs as a static first item: decode CTA c
+// (c < this * Hkv) starts with partition 0 of sequence c / Hkv, kv head c % Hkv,
+// computed from the inputs alone, so it does not wait for the plan; the plan
+// lists every other (sequence, partition).
+__device__ __forceinline__ int static_first_seqs(const int num_seqs, const int grid_ctas, const int Hkv) {
+  const int n = grid_ctas / Hkv;
+  return n < num_seqs ? n : num_seqs;
+}
+
 __device__ __forceinline__ int clamp_len(int L, int max_ctx) {
   return L < 0 ? 0 : (L > max_ctx ? max_ctx : L);
 }
@@ -186,22 +195,25 @@ __device__ __forceinline__ void allow_dependent_launch() {
 // all threads at once (one round trip); the lengths are kept in shared memory
 // for the second pass.
 constexpr int kPlanSmemSeqs = 8192;
+constexpr int kPlanDirect = 8;   // partitions a thread writes itself
+constexpr int kPlanWide = 512;   // sequences listed for warp-wide record writing
 
 static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeArgs a) {
-  // The decode grid may start its set-up now; it waits for this grid to finish
-  // before it reads anything written here.  This grid itself starts behind its
-  // predecessor on the stream and waits for it before reading any input.
+  // This grid is launched in plain stream order, so its predecessor has
+  // completed.  The decode grid may start now: its static first items read only
+  // inputs, and it waits for this grid before it touches anything written here.
   allow_dependent_launch();
-  grid_dependency_wait();
+  const int n_static = static_first_seqs(a.num_seqs, a.grid_ctas, a.num_kv_heads);
   constexpr int kMaxClasses = kMaxPartTokens / 32 + 2;
   __shared__ uint32_t count[kMaxClasses];
   __shared__ uint32_t cursor[kMaxClasses];
-  __shared__ uint32_t total, n_multi;
+  __shared__ uint32_t total, n_multi, n_wide;
+  __shared__ int4 s_wide[kPlanWide];  // (sequence, first full-size slot, last slot, first listed partition)
   __shared__ int s_len[kPlanSmemSeqs];
   const int classes = a.part_tokens / 32 + 2;  // class c: size in (part - 32(c+1), part - 32c]; last: empty
   const bool cached = a.num_seqs <= kPlanSmemSeqs;
   for (int c = threadIdx.x; c < classes; c += blockDim.x) count[c] = 0;
-  if (threadIdx.x == 0) total = n_multi = 0;
+  if (threadIdx.x == 0) total = n_multi = n_wide = 0;
   __syncthreads();
   auto size_class = [&](int sz) { return sz == 0 ? classes - 1 : (a.part_tokens - sz) / 32; };
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
@@ -211,8 +223,13 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
     if (cached) s_len[s] = L;
     int n, size;
     partition_of(L, a.part_tokens, n, size);
-    for (int p = 0; p < n; ++p) atomicAdd(&count[size_class(min(size, L - p * size))], 1u);
-    atomicAdd(&total, static_cast<uint32_t>(n));
+    // listed partitions: skip .. n-1 (partition 0 of a static sequence is not
+    // listed); partitions below n-1 have `size` tokens, the last one the rest
+    const int skip = s < n_static ? 1 : 0;
+    const int n_full = n - 1 - skip;
+    if (n_full > 0) atomicAdd(&count[size_class(size)], static_cast<uint32_t>(n_full));
+    if (n - 1 >= skip) atomicAdd(&count[size_class(L - (n - 1) * size)], 1u);
+    atomicAdd(&total, static_cast<uint32_t>(n - skip));
     if (n > 1) {
       a.merge_seqs[atomicAdd(&n_multi, 1u)] = s;
       for (int h = 0; h < a.num_kv_heads; ++h) a.pair_done[s * a.num_kv_heads + h] = 0u;
@@ -244,21 +261,64 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
     }
   }
   __syncthreads();
+  // Records: one reservation per size class and sequence (its full-size
+  // partitions take consecutive slots).  A sequence with more than
+  // kPlanDirect partitions has its records written by a whole warp afterwards
+  // (one lane per partition) instead of by one thread in a loop.  The first
+  // records of the list (about one item per decode CTA: record r holds items
+  // r * Hkv .. r * Hkv + Hkv - 1) are taken within microseconds of the start,
+  // so their block-table entries are prefetched into L2 here.
+  const uint32_t first_wave_records =
+      (static_cast<uint32_t>(a.grid_ctas) + a.num_kv_heads - 1) / a.num_kv_heads;
+  auto write_record = [&](int s, int p, int n, int size, int L, uint32_t pos) {
+    const int t_begin = p * size;
+    const int n_tok = min(size, L - t_begin);
+    int4* rec = reinterpret_cast<int4*>(a.records + static_cast<int64_t>(pos) * kRecordBytes);
+    rec[0] = make_int4(s, p, n, t_begin);
+    rec[1] = make_int4(n_tok, L, 0, 0);
+    if (a.tables != nullptr && pos < first_wave_records && n_tok > 0) {
+      const int32_t* row = a.tables + static_cast<int64_t>(s) * a.max_blocks + t_begin / a.block_size;
+      const int nb = (n_tok + a.block_size - 1) / a.block_size;
+      for (int e = 0; e < nb; e += 32) prefetch_l2(row + e);  // one per 128-byte line
+      prefetch_l2(row + nb - 1);                                // the line of the last entry
+    }
+  };
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int L = cached ? s_len[s] : clamp_len(a.lens[s], a.max_ctx);
     int n, size;
     partition_of(L, a.part_tokens, n, size);
-    for (int p = 0; p < n; ++p) {
-      const int t_begin = p * size;
-      const int n_tok = min(size, L - t_begin);
-      const uint32_t pos = atomicAdd(&cursor[size_class(n_tok)], 1u);
-      int4* rec = reinterpret_cast<int4*>(a.records + static_cast<int64_t>(pos) * kRecordBytes);
-      rec[0] = make_int4(s, p, n, t_begin);
-      rec[1] = make_int4(n_tok, L, 0, 0);
+    const int last = L - (n - 1) * size;
+    const int skip = s < n_static ? 1 : 0;
+    const int n_full = n - 1 - skip;
+    const uint32_t base = n_full > 0 ? atomicAdd(&cursor[size_class(size)], static_cast<uint32_t>(n_full)) : 0u;
+    const uint32_t last_pos = n - 1 >= skip ? atomicAdd(&cursor[size_class(last)], 1u) : 0u;
+    if (n > kPlanDirect) {
+      const uint32_t i = atomicAdd(&n_wide, 1u);
+      if (i < kPlanWide) {
+        s_wide[i] = make_int4(s, static_cast<int>(base), static_cast<int>(last_pos), skip);
+        continue;
+      }
+    }
+    for (int p = skip; p < n; ++p)
+      write_record(s, p, n, size, L, p < n - 1 ? base + static_cast<uint32_t>(p - skip) : last_pos);
+  }
+  __syncthreads();
+  {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_w = min(static_cast<int>(n_wide), kPlanWide);
+    for (int i = warp; i < n_w; i += kPlanThreads / 32) {
+      const int4 e = s_wide[i];
+      const int s = e.x;
+      const int L = cached ? s_len[s] : clamp_len(a.lens[s], a.max_ctx);
+      int n, size;
+      partition_of(L, a.part_tokens, n, size);
+      for (int p = e.w + lane; p < n; p += 32)
+        write_record(s, p, n, size, L,
+                     p < n - 1 ? static_cast<uint32_t>(e.y + p - e.w) : static_cast<uint32_t>(e.z));
     }
   }
   if (threadIdx.x == 0) {
-    a.work[0] = static_cast<uint32_t>(a.grid_ctas);  // item c is CTA c's first
+    a.work[0] = 0u;  // next list item
     a.work[1] = total * static_cast<uint32_t>(a.num_kv_heads);
     a.work[2] = n_multi;
   }
@@ -312,15 +372,15 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
     fence_barrier_init();
   }
   __syncthreads();
-  // Everything below reads what the plan kernel wrote.
-  grid_dependency_wait();
-  // The merge grid may launch now: it reads what the plan wrote and waits per
-  // (sequence, kv head) for the partitions this grid publishes.
-  allow_dependent_launch();
+  // The plan grid was launched in plain stream order and let this grid start,
+  // so every input is ready here; what the plan writes (work list, counters) is
+  // read only after grid_dependency_wait (plan_wait below).
 
   // ================================================================ producer
-  // Item k (the k-th item this CTA takes).  The CTA's first item is item
-  // blockIdx.x of the largest-first list; each later one comes from the work
+  // Item k (the k-th item this CTA takes).  CTAs below static_first_seqs * Hkv
+  // start with partition 0 of sequence blockIdx.x / Hkv (kv head blockIdx.x %
+  // Hkv), described from the inputs alone, while the plan is still running.
+  // Every other item comes from the largest-first list through the work
   // counter, taken while the previous item streams: right after that item's
   // first stage is issued (a stage is in flight while the atomic returns), its
   // 32-byte record is bulk-copied; after the second stage (or at the end of a
@@ -329,8 +389,19 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
   // the list stays dynamic.
   if (warp == NW) {
     if (lane < 4) prefetch_tensor_map(&maps.k + lane);
-    const uint32_t n_items = *reinterpret_cast<volatile uint32_t*>(a.work + 1);
     const uint32_t Hkv = static_cast<uint32_t>(a.num_kv_heads);
+    uint32_t n_items = 0;
+    bool plan_done = false;
+    // Wait for the plan grid (its list and counters), then let the merge grid
+    // launch: it also reads what the plan wrote.
+    auto plan_wait = [&]() {
+      if (!plan_done) {
+        grid_dependency_wait();
+        allow_dependent_launch();
+        n_items = *reinterpret_cast<volatile uint32_t*>(a.work + 1);
+        plan_done = true;
+      }
+    };
     int32_t* s_tab = reinterpret_cast<int32_t*>(smem + Tr::OFF_TAB);
     auto rec_slot = [&](uint32_t j) {
       return reinterpret_cast<const int32_t*>(smem + Tr::OFF_REC + (j & 1) * kRecordBytes);
@@ -381,11 +452,37 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
     };
 
     bool ok = true;
-    uint32_t cur = blockIdx.x;  // this CTA's first item
-    if (cur < n_items) {
-      if (lane == 0) copy_record(0, cur);
-      ok = wait_record(0);
-      if (ok) fetch_table(0);
+    const bool static_first =
+        blockIdx.x < static_cast<uint32_t>(static_first_seqs(a.num_seqs, a.grid_ctas, a.num_kv_heads)) * Hkv;
+    uint32_t cur = 0;  // list index of the current item (items after a static first one)
+    if (static_first) {
+      if (lane == 0) {  // record of partition 0 of sequence blockIdx.x / Hkv, in slot 0
+        int32_t* r = reinterpret_cast<int32_t*>(smem + Tr::OFF_REC);
+        const int s = static_cast<int>(blockIdx.x / Hkv);
+        const int L = clamp_len(a.lens[s], a.max_ctx);
+        int n, size;
+        partition_of(L, a.part_tokens, n, size);
+        r[0] = s;
+        r[1] = 0;
+        r[2] = n;
+        r[3] = 0;
+        r[4] = min(size, L);
+        r[5] = L;
+        // Complete phase 0 of the slot's barrier as a copy would have: slot 0
+        // is next used by item 2, which waits for phase 1.
+        mbar_arrive(&rec_bar[0]);
+      }
+      __syncwarp();
+      fetch_table(0);
+    } else {
+      plan_wait();
+      if (lane == 0) cur = atomicAdd(a.work, 1u);
+      cur = __shfl_sync(0xffffffffu, cur, 0);
+      if (cur < n_items) {
+        if (lane == 0) copy_record(0, cur);
+        ok = wait_record(0);
+        if (ok) fetch_table(0);
+      }
     }
     uint32_t issued = 0, st = 0, ph = 0;  // stages issued; ring slot and use parity of the next
     for (uint32_t k = 0; ok; ++k) {
@@ -397,7 +494,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      if (cur >= n_items) {
+      const bool is_static = k == 0 && static_first;
+      if (!is_static && cur >= n_items) {
         if (lane == 0) {
           items[slot].s = -1;  // no more work
           mbar_arrive(&item_full[slot]);
@@ -407,7 +505,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
       if (!wait_table(k)) break;  // fetched while the previous item streamed
       const int32_t* rec = rec_slot(k);
       const int s = rec[0], part = rec[1], n_parts = rec[2], t_begin = rec[3], n_tok = rec[4];
-      const int kvh = static_cast<int>(cur % Hkv);
+      const int kvh = static_cast<int>((is_static ? blockIdx.x : cur) % Hkv);
       if (lane == 0) {
         ItemInfo& info = items[slot];
         info.s = s;
@@ -427,6 +525,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
       bool next_ready = false;    // its record waited for and its table requested
       auto prepare_next = [&](int step) {
         if (step == 0) {
+          plan_wait();
           if (lane == 0) {
             nxt = atomicAdd(a.work, 1u);
             if (nxt < n_items) copy_record(k + 1, nxt);
@@ -812,27 +911,39 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
   // Every loop exit follows a barrier that all consumer threads passed after
   // their last write-out (or a stage timeout, whose item is not listed).
   if (threadIdx.x == 0) publish();
+  // The merge grid may launch once every thread of every CTA has passed the
+  // plan (the producer did so before its first list access).
+  grid_dependency_wait();
+  allow_dependent_launch();
 }
 
 // ---------------------------------------------------------------- merge
 // Contexts that span several partitions: out = sum_p w_p o_p with
-// w_p = l_p 2^(m_p - M) / sum_q l_q 2^(m_q - M), M = max_p m_p, summed in
-// partition order.  One CTA of 128 threads per (sequence, kv head) pair listed
-// by the plan kernel (grid-stride when there are more pairs than CTAs).  The
-// outputs of the first kPre partitions are loaded into registers up front, so
-// with up to kPre partitions a pair costs about one memory round trip.
-// Launched behind the decode grid (programmatic dependent launch): it waits for
-// the whole decode grid before reading its results.
-constexpr int kMergeThreads = 128;
-constexpr int kMergeStat = 64;  // partitions per statistics round
-constexpr int kPre = 8;         // partitions per output round
+// w_p = l_p 2^(m_p - M) / sum_q l_q 2^(m_q - M), M = max_p m_p.  One CTA of
+// kMergeThreads threads per (sequence, kv head) pair listed by the plan kernel
+// (grid-stride when there are more pairs than CTAs).  Thread t owns float4 group
+// t % NV of the pair's G x D output and the partitions p with p % SLICES ==
+// t / NV, so a pair's partial outputs are all requested at once; the slices are
+// summed in shared memory (fixed order) at the end.  Statistics are read in
+// chunks of kMergeChunk partitions (one chunk for up to 64).
+// The grid launches while the decode grid still runs: each pair waits for the
+// decode grid's per-pair count, and its partials are read from L2.
+constexpr int kMergeThreads = 256;
+constexpr int kMergeChunk = 64;
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a) {
-  __shared__ float s_m[G][kMergeStat], s_l[G][kMergeStat], s_w[G][kPre];
+  constexpr int NV = G * D / 4;  // float4 groups of one pair's output
+  static_assert(NV <= kMergeThreads && kMergeThreads % NV == 0, "whole slices");
+  constexpr int SLICES = kMergeThreads / NV;
+  constexpr int NWARP = kMergeThreads / 32;
+  __shared__ float s_m[G][kMergeChunk], s_w[G][kMergeChunk];
   __shared__ float s_M[G], s_L[G];
+  __shared__ float4 s_part[SLICES > 1 ? SLICES - 1 : 1][NV];
   __shared__ int s_ready;
-  constexpr int kPer = (G * D + kMergeThreads - 1) / kMergeThreads;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int v = tid % NV, slice = tid / NV;
+  const int vg = v / (D / 4), vd = (v % (D / 4)) * 4;  // head and first dim of this thread's group
   const uint32_t Hkv = static_cast<uint32_t>(a.num_kv_heads);
   // The plan finished before the decode grid let this grid launch.
   const uint32_t n_tasks = __ldcg(a.work + 2) * Hkv;
@@ -847,7 +958,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
     // Wait (bounded) until the decode grid has published all np partitions of
     // this pair; their results are then read from L2 (__ldcg), never from a
     // possibly stale L1 line.
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
       s_ready = wait_counter_bounded(a.pair_done + static_cast<int64_t>(s) * Hkv + kvh,
                                      static_cast<uint32_t>(np), a.err);
       if (!s_ready) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
@@ -855,82 +966,89 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
     __syncthreads();
     if (!s_ready) continue;  // uniform: results of this pair stay unwritten
 
-    float pre[kPre][kPer];  // outputs of partitions 0 .. kPre-1
-#pragma unroll
-    for (int p = 0; p < kPre; ++p)
-#pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int idx = threadIdx.x + k * kMergeThreads;
-        pre[p][k] = (p < np && idx < G * D) ? __ldcg(a.tmp_out + cell(idx / D, p) * D + idx % D) : 0.f;
-      }
-
-    // M and the normaliser per head, online over rounds of kMergeStat partitions
-    if (threadIdx.x < G) {
-      s_M[threadIdx.x] = -CUDART_INF_F;
-      s_L[threadIdx.x] = 0.f;
-    }
-    for (int c0 = 0; c0 < np; c0 += kMergeStat) {
-      const int cn = min(kMergeStat, np - c0);
-      for (int i = threadIdx.x; i < G * cn; i += kMergeThreads) {
+    // ---- M and L per head (warp g reduces head g; online across chunks)
+    float M = -CUDART_INF_F, L = 0.f;  // valid in warp g < G
+    for (int c0 = 0; c0 < np; c0 += kMergeChunk) {
+      const int cn = min(kMergeChunk, np - c0);
+      if (c0 > 0) __syncthreads();  // the previous chunk's s_m / s_w are no longer read
+      for (int i = tid; i < G * cn; i += kMergeThreads) {
         const int g = i / cn, p = i % cn;
         s_m[g][p] = __ldcg(a.tmp_m + cell(g, c0 + p));
-        s_l[g][p] = __ldcg(a.tmp_l + cell(g, c0 + p));
+        s_w[g][p] = __ldcg(a.tmp_l + cell(g, c0 + p));  // l for now
       }
       __syncthreads();
-      if (threadIdx.x < G) {
-        const int g = threadIdx.x;
-        float M = s_M[g];
-        for (int p = 0; p < cn; ++p) M = fmaxf(M, s_m[g][p]);
-        float L = s_L[g] * fast_exp2(s_M[g] - M);  // 0 on the first round
-        for (int p = 0; p < cn; ++p) L += s_l[g][p] * fast_exp2(s_m[g][p] - M);
-        s_M[g] = M;
-        s_L[g] = L;
+      for (int g = warp; g < G; g += NWARP) {
+        float mc = -CUDART_INF_F;
+        for (int p = lane; p < cn; p += 32) mc = fmaxf(mc, s_m[g][p]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+        const float Mn = fmaxf(M, mc);
+        float lc = 0.f;
+        for (int p = lane; p < cn; p += 32) lc += s_w[g][p] * fast_exp2(s_m[g][p] - Mn);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lc += __shfl_xor_sync(0xffffffffu, lc, o);
+        L = L * fast_exp2(M - Mn) + lc;  // M = -inf on the first chunk: the old sum is 0
+        M = Mn;
       }
-      __syncthreads();
     }
+    if (warp < G && lane == 0) {
+      s_M[warp] = M;
+      s_L[warp] = L;
+    }
+    __syncthreads();
 
-    float o_reg[kPer];
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) o_reg[k] = 0.f;
-    for (int p0 = 0; p0 < np; p0 += kPre) {
-      const int pc = min(kPre, np - p0);
-      if (threadIdx.x < G * pc) {
-        const int g = threadIdx.x / pc, p = threadIdx.x % pc;
-        s_w[g][p] = __ldcg(a.tmp_l + cell(g, p0 + p)) * fast_exp2(__ldcg(a.tmp_m + cell(g, p0 + p)) - s_M[g]) / s_L[g];
+    // ---- weighted sum of the partial outputs
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < np; c0 += kMergeChunk) {
+      const int cn = min(kMergeChunk, np - c0);
+      if (c0 > 0) {
+        __syncthreads();  // the previous chunk's weights are no longer read
+        for (int i = tid; i < G * cn; i += kMergeThreads) {
+          const int g = i / cn, p = i % cn;
+          s_m[g][p] = __ldcg(a.tmp_m + cell(g, c0 + p));
+          s_w[g][p] = __ldcg(a.tmp_l + cell(g, c0 + p));
+        }
+        __syncthreads();
       }
-      if (p0 > 0) {
-#pragma unroll
-        for (int p = 0; p < kPre; ++p)
-#pragma unroll
-          for (int k = 0; k < kPer; ++k) {
-            const int idx = threadIdx.x + k * kMergeThreads;
-            pre[p][k] = (p < pc && idx < G * D) ? __ldcg(a.tmp_out + cell(idx / D, p0 + p) * D + idx % D) : 0.f;
-          }
+      // weights, in place of l: l_p 2^(m_p - M) / L
+      for (int i = tid; i < G * cn; i += kMergeThreads) {
+        const int g = i / cn, p = i % cn;
+        s_w[g][p] = s_w[g][p] * fast_exp2(s_m[g][p] - s_M[g]) / s_L[g];
       }
       __syncthreads();
+      const float* wrow = s_w[vg];
+      const float* src = a.tmp_out + cell(vg, c0) * D + vd;
+#pragma unroll 8
+      for (int p = slice; p < cn; p += SLICES) {
+        const float4 o = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(p) * D));
+        const float wp = wrow[p];
+        acc.x += wp * o.x;
+        acc.y += wp * o.y;
+        acc.z += wp * o.z;
+        acc.w += wp * o.w;
+      }
+    }
+    // ---- slices 1.. hand their sums to slice 0, which adds them in order
+    if (SLICES > 1) {
+      if (slice > 0) s_part[slice - 1][v] = acc;
+      __syncthreads();
+      if (slice == 0) {
 #pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int idx = threadIdx.x + k * kMergeThreads;
-        if (idx < G * D) {
-          const int g = idx / D;
-          float o = o_reg[k];
-#pragma unroll
-          for (int p = 0; p < kPre; ++p)
-            if (p < pc) o += s_w[g][p] * pre[p][k];
-          o_reg[k] = o;
+        for (int j = 0; j < SLICES - 1; ++j) {
+          const float4 o = s_part[j][v];
+          acc.x += o.x;
+          acc.y += o.y;
+          acc.z += o.z;
+          acc.w += o.w;
         }
       }
-      __syncthreads();
     }
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int idx = threadIdx.x + k * kMergeThreads;
-      if (idx < G * D) {
-        const int g = idx / D, d = idx % D;
-        static_cast<T*>(a.out)[(static_cast<int64_t>(s) * a.num_heads + h0 + g) * D + d] =
-            from_float<T>(o_reg[k]);
-      }
+    if (slice == 0) {
+      const uint2 packed = make_uint2(pack2<T>(acc.x, acc.y), pack2<T>(acc.z, acc.w));
+      *reinterpret_cast<uint2*>(static_cast<T*>(a.out) +
+                                (static_cast<int64_t>(s) * a.num_heads + h0 + vg) * D + vd) = packed;
     }
+    __syncthreads();  // shared state is reused by the next pair
   }
   // Complete only after the decode grid: work behind this grid on the stream
   // then sees every output row, including the single-partition ones.

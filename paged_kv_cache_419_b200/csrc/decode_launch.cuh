@@ -39,21 +39,24 @@ cudaError_t launch_decode_one(const DecodeArgs& args, const DecodeMaps& maps, in
   if (e != cudaSuccess) return e;
   DecodeArgs a = args;
   a.grid_ctas = grid;
-  // Programmatic dependent launch for all three kernels: each may start (and
-  // set up) while its predecessor finishes, and waits for it in-kernel before
-  // touching anything the predecessor writes.
+  // The plan grid is launched in plain stream order: it starts once everything
+  // before it on the stream has completed, so the kernels behind it may read
+  // their inputs as soon as they start.  Decode and merge use programmatic
+  // dependent launch: each may start while its predecessor runs and waits for
+  // it in-kernel before touching anything the predecessor writes.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 0;
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(kPlanThreads);
   cfg.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&cfg, plan_kernel, a);
   if (e != cudaSuccess) return e;
+  cfg.numAttrs = 1;
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kDecodeThreads);
   cfg.dynamicSmemBytes = Tr::SMEM_BYTES;
@@ -61,10 +64,12 @@ cudaError_t launch_decode_one(const DecodeArgs& args, const DecodeMaps& maps, in
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess || a.max_parts <= 1) return e;
-  // Partition merge, also behind its predecessor: its CTAs start as decode CTAs
-  // retire and wait in-kernel for the whole decode grid.
+  // Partition merge, also behind its predecessor: its CTAs become resident as
+  // decode CTAs retire and merge each pair once the decode grid has published
+  // it.  At most one wave (8 CTAs of 256 threads per SM), so that no merge CTA
+  // waits for a slot behind one that is parked at its final grid wait.
   const int64_t pairs = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
-  const int64_t want = static_cast<int64_t>(num_sms) * 16;  // one wave of 128-thread CTAs
+  const int64_t want = static_cast<int64_t>(num_sms) * (2048 / kMergeThreads);
   cfg.gridDim = dim3(static_cast<unsigned>(pairs < want ? pairs : want));
   cfg.blockDim = dim3(kMergeThreads);
   cfg.dynamicSmemBytes = 0;

@@ -81,14 +81,15 @@ def test_mha13b_contiguous_matches_oracle_and_paged():
     assert torch.equal(out, out_paged)
 
 
-def test_gqa8b_full_size_sampled_sequences():
-    """The benchmark's batch and launch configuration (partition 512), all 256
-    sequences run on the GPU; the oracle checks 40 of them spread over the batch,
-    including the shortest and the longest."""
+@pytest.mark.parametrize("part", [512, 1024])
+def test_gqa8b_full_size_sampled_sequences(part):
+    """The benchmark's batch and launch configuration (partition 1024, the
+    default; and 512), all 256 sequences run on the GPU; the oracle checks 40 of
+    them spread over the batch, including the shortest and the longest."""
     inp = wl.make_decode_inputs("gqa8b")
     B = _bin()
     b = gpu_step_inputs(inp)
-    out = gpu_decode_step(inp, b, 512)
+    out = gpu_decode_step(inp, b, part)
     torch.cuda.synchronize()
     assert B.device_error() == 0
     ob = oracle_step_inputs(inp)
