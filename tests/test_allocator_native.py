@@ -144,3 +144,42 @@ def test_decode_workload_tables_follow_the_frame_order():
     used = np.concatenate([table[s][table[s] >= 0] for s in range(16)])
     assert used.tolist() == inp.frame_order[: used.size].tolist()
     assert lens.tolist() == inp.context_lens.tolist()
+
+
+def test_kv_memory_report_matches_the_model():
+    """The bench's KV memory report (native allocator) against the Python model
+    on the same batches: useful-KV share of the gqa8b batch (the pages report
+    96.3 % useful KV memory, dataarena note section 2) and the frames saved by
+    sharing prompts among 4 samples with copy-on-write (slides 13-14)."""
+    import bench
+
+    w = wl.WORKLOADS["gqa8b"]
+    lens = wl.make_decode_inputs(w).context_lens
+    rep = bench.kv_memory_report(w, lens)
+    m = AllocatorModel(w.num_blocks, w.block_size)
+    for s, L in enumerate(lens):
+        m.add_seq(s, int(L))
+    st = m.stats()
+    assert rep["frames"] == st["used_blocks"] == int(sum(-(-int(L) // w.block_size) for L in lens))
+    assert rep["tokens"] == int(lens.sum())
+    assert rep["useful_kv_pct"] == round(100.0 * lens.sum() / (st["used_blocks"] * w.block_size), 2)
+    assert rep["useful_kv_pct"] > 96.3  # only each sequence's last block is partial
+
+    sh = wl.make_shared_inputs()
+    ws = sh.w
+    m = AllocatorModel(ws.num_blocks, ws.block_size, sh.frame_order)
+    n = ws.samples_per_prompt
+    for p in range(ws.num_prompts):
+        m.add_seq(p * n, sh.prompt_len)
+        for c in range(1, n):
+            m.fork(p * n, p * n + c)
+    copies = 0
+    for step in range(int(sh.gen_lens.max())):
+        for s in range(ws.num_seqs):
+            if sh.gen_lens[s] > step:
+                _, src, _ = m.append(s)
+                copies += src >= 0
+    ms = m.stats()
+    assert rep["sharing_frames"] == ms["used_blocks"]
+    assert rep["sharing_unshared_frames"] == ms["logical_blocks"]
+    assert rep["sharing_cow_copies"] == copies
