@@ -571,6 +571,9 @@ def kv_memory_report(w: wl.Workload, lens: np.ndarray) -> dict:
     sharing_saving_pct: 1 - frames held / frames the same tables would need
     unshared, for 16 prompts of 1000 tokens x 4 samples that each decode 0-200
     tokens with copy-on-write (slides 13-14 report 6-66 % savings).
+    beam_saving_pct: the same for 4 beams over a block tree (slide 14), 200 steps
+    from one 1000-token prompt (kashii section 3: beam search memory cut by up to
+    55 %).
     """
     from paged_kv_cache_419_b200 import binding as pkv
 
@@ -596,6 +599,16 @@ def kv_memory_report(w: wl.Workload, lens: np.ndarray) -> dict:
         copies += len(pairs)
     ss = a.stats()
     a.close()
+    bm = wl.make_beam_inputs()
+    wb = bm.w
+    a = pkv.BlockAllocator(wb.num_blocks, wb.block_size, bm.frame_order)
+    a.add_seq(0, bm.prompt_len)
+    beams, nid, beam_copies = np.zeros(1, np.int32), 1, 0
+    for step in range(bm.steps):
+        beams, _, pairs, nid = a.beam_step(beams, bm.parents[step], nid)
+        beam_copies += len(pairs)
+    bs = a.stats()
+    a.close()
     return {
         "useful_kv_pct": round(100.0 * st["tokens"] / capacity, 2),
         "frames": int(st["used_blocks"]), "tokens": int(st["tokens"]), "block_size": w.block_size,
@@ -603,6 +616,9 @@ def kv_memory_report(w: wl.Workload, lens: np.ndarray) -> dict:
         "sharing_saving_pct": round(100.0 * (1 - ss["used_blocks"] / ss["logical_blocks"]), 2),
         "sharing_frames": int(ss["used_blocks"]), "sharing_unshared_frames": int(ss["logical_blocks"]),
         "sharing_cow_copies": int(copies),
+        "beam_saving_pct": round(100.0 * (1 - bs["used_blocks"] / bs["logical_blocks"]), 2),
+        "beam_frames": int(bs["used_blocks"]), "beam_unshared_frames": int(bs["logical_blocks"]),
+        "beam_cow_copies": int(beam_copies),
     }
 
 

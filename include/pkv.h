@@ -266,6 +266,29 @@ pkv_status pkv_alloc_append(pkv_allocator* alloc, int32_t seq_id, int64_t* slot_
 pkv_status pkv_alloc_append_batch(pkv_allocator* alloc, const int32_t* seq_ids, int32_t n,
                                   int64_t* slots_out, int64_t* pairs_out, int32_t* num_pairs_out);
 pkv_status pkv_alloc_free_seq(pkv_allocator* alloc, int32_t seq_id);
+/*
+ * One beam-search step over a block tree (slides 13-14 "Beam search: a block
+ * tree, not copies": candidates share their prefix like forked processes;
+ * kashii section 3: copy on write when their tokens diverge).
+ *   beams[0..k-1]       the live beams' sequence ids (distinct)
+ *   parents[0..k_new-1] new beam j continues beam parents[j] (index into beams)
+ *   *next_id            first id for extra continuations; advanced past the ids used
+ *   new_ids_out[k_new]  sequence id of each new beam: a parent's first continuation
+ *                       keeps the parent's id, every further one is a fork with a
+ *                       fresh id (all of the parent's frames shared, counts + 1)
+ *   slots_out[k_new]    slot of the token appended to each new beam
+ *   pairs_out[k_new, 2] copy pairs (shared frame, private frame), *num_pairs_out
+ * Order: the forks (in new-beam order), then the frees of the beams without a
+ * continuation (in beam order; their frames go to the tail of the free queue),
+ * then one append per new beam in order, with the copy-on-write rule of
+ * pkv_alloc_append.  All-or-nothing: PKV_ENOMEM (nothing changed) when the step
+ * needs more frames than are free after the frees; PKV_EINVAL for unknown or
+ * repeated beams, a parent index outside [0, k), or a fresh id already in use.
+ */
+pkv_status pkv_alloc_beam_step(pkv_allocator* alloc, const int32_t* beams, int32_t k,
+                               const int32_t* parents, int32_t k_new, int32_t* next_id,
+                               int32_t* new_ids_out, int64_t* slots_out, int64_t* pairs_out,
+                               int32_t* num_pairs_out);
 /* Block tables of seq_ids as host int32 [n, max_blocks] padded with -1, and
  * their lengths (lens_out may be NULL).  PKV_ERANGE if a table is longer than
  * max_blocks. */

@@ -127,6 +127,50 @@ class AllocatorModel:
         self.lens[seq] = t + 1
         return self.slot(seq, t), src, dst
 
+    def beam_step(self, beams, parents, next_id: int):
+        """One beam-search step over the block tree (slide 14: candidates share
+        their prefix like forked processes; kashii section 3: copy on write when
+        tokens diverge).  New beam j continues beams[parents[j]]: the first
+        continuation of a beam keeps its id, each further one is a fork with the
+        next fresh id; beams with no continuation are freed; then every new beam
+        appends one token.  Order: forks, frees, appends.  All-or-nothing:
+        ENOMEM restores the state.  Returns (new_ids, slots, pairs, next_id)."""
+        beams = [int(b) for b in beams]
+        parents = [int(p) for p in parents]
+        if len(set(beams)) != len(beams) or any(b not in self.tables for b in beams):
+            raise AllocatorError("EINVAL")
+        if any(p < 0 or p >= len(beams) for p in parents):
+            raise AllocatorError("EINVAL")
+        ids, first = [], set()
+        for p in parents:
+            if p not in first:
+                first.add(p)
+                ids.append(beams[p])
+            else:
+                if next_id in self.tables:
+                    raise AllocatorError("EINVAL")
+                ids.append(next_id)
+                next_id += 1
+        saved = ({k: list(v) for k, v in self.tables.items()}, dict(self.lens), list(self.ref),
+                 deque(self.free))
+        try:
+            for j, p in enumerate(parents):
+                if ids[j] != beams[p]:
+                    self.fork(beams[p], ids[j])
+            for i, b in enumerate(beams):
+                if i not in first:
+                    self.free_seq(b)
+            slots, pairs = [], []
+            for j in range(len(parents)):
+                slot, src, dst = self.append(ids[j])
+                slots.append(slot)
+                if src >= 0:
+                    pairs.append([src, dst])
+        except AllocatorError:
+            self.tables, self.lens, self.ref, self.free = saved
+            raise
+        return ids, slots, pairs, next_id
+
     def free_seq(self, seq: int):
         if seq not in self.tables:
             raise AllocatorError("EINVAL")

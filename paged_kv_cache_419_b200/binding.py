@@ -28,7 +28,7 @@ EXPORTS = (
     "pkv_contiguous_attention_decode", "pkv_reshape_and_cache",
     "pkv_copy_blocks", "pkv_alloc_create", "pkv_alloc_destroy", "pkv_alloc_add_seq",
     "pkv_alloc_fork", "pkv_alloc_append", "pkv_alloc_append_batch", "pkv_alloc_free_seq",
-    "pkv_alloc_block_table", "pkv_alloc_refcount", "pkv_alloc_stats",
+    "pkv_alloc_beam_step", "pkv_alloc_block_table", "pkv_alloc_refcount", "pkv_alloc_stats",
 )
 
 
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "pkv_alloc_append": ([P, i32, P, P, P], ctypes.c_int),
             "pkv_alloc_append_batch": ([P, P, i32, P, P, P], ctypes.c_int),
             "pkv_alloc_free_seq": ([P, i32], ctypes.c_int),
+            "pkv_alloc_beam_step": ([P, P, i32, P, i32, P, P, P, P, P], ctypes.c_int),
             "pkv_alloc_block_table": ([P, P, i32, i32, P, P], ctypes.c_int),
             "pkv_alloc_refcount": ([P, i32, P], ctypes.c_int),
             "pkv_alloc_stats": ([P, ctypes.POINTER(AllocStats)], ctypes.c_int),
@@ -280,6 +281,25 @@ class BlockAllocator:
 
     def free_seq(self, seq_id: int):
         _check(lib().pkv_alloc_free_seq(self._h, seq_id), "pkv_alloc_free_seq")
+
+    def beam_step(self, beams, parents, next_id: int):
+        """One beam-search step (pkv_alloc_beam_step): returns (new_ids, slots,
+        copy pairs, next_id)."""
+        np = self._np
+        b = np.ascontiguousarray(beams, dtype=np.int32)
+        p = np.ascontiguousarray(parents, dtype=np.int32)
+        k, kn = b.shape[0], p.shape[0]
+        ids = np.empty(max(kn, 1), dtype=np.int32)
+        slots = np.empty(max(kn, 1), dtype=np.int64)
+        pairs = np.empty((max(kn, 1), 2), dtype=np.int64)
+        nid, npairs = ctypes.c_int32(next_id), ctypes.c_int32()
+        _check(lib().pkv_alloc_beam_step(self._h, b.ctypes.data_as(ctypes.c_void_p), k,
+                                         p.ctypes.data_as(ctypes.c_void_p), kn, ctypes.byref(nid),
+                                         ids.ctypes.data_as(ctypes.c_void_p),
+                                         slots.ctypes.data_as(ctypes.c_void_p),
+                                         pairs.ctypes.data_as(ctypes.c_void_p), ctypes.byref(npairs)),
+               "pkv_alloc_beam_step")
+        return ids[:kn], slots[:kn], pairs[: npairs.value], nid.value
 
     def block_table(self, seq_ids, max_blocks: int):
         np = self._np

@@ -173,6 +173,98 @@ pkv_status pkv_alloc_append_batch(pkv_allocator* a, const int32_t* seq_ids, int3
   return PKV_OK;
 }
 
+pkv_status pkv_alloc_beam_step(pkv_allocator* a, const int32_t* beams, int32_t k,
+                               const int32_t* parents, int32_t k_new, int32_t* next_id,
+                               int32_t* new_ids_out, int64_t* slots_out, int64_t* pairs_out,
+                               int32_t* num_pairs_out) {
+  if (!a || k < 0 || k_new < 0 || !next_id || !num_pairs_out ||
+      (k > 0 && !beams) || (k_new > 0 && (!parents || !new_ids_out || !slots_out || !pairs_out)))
+    return PKV_EINVAL;
+  // Check everything and count the frames the step needs before changing anything.
+  std::vector<pkv_allocator::Seq*> old(k);
+  std::unordered_set<int32_t> seen;
+  for (int32_t i = 0; i < k; ++i) {
+    auto it = a->seqs.find(beams[i]);
+    if (it == a->seqs.end() || !seen.insert(beams[i]).second) return PKV_EINVAL;
+    old[i] = &it->second;
+  }
+  std::vector<int32_t> children(k, 0);
+  for (int32_t j = 0; j < k_new; ++j) {
+    if (parents[j] < 0 || parents[j] >= k) return PKV_EINVAL;
+    children[parents[j]] += 1;
+  }
+  // ids of the new beams: a parent's first continuation keeps its id, the others
+  // take fresh ids counting up from *next_id
+  std::vector<int32_t> ids(k_new);
+  std::vector<char> taken(k, 0);
+  int32_t fresh = *next_id;
+  for (int32_t j = 0; j < k_new; ++j) {
+    const int32_t i = parents[j];
+    if (!taken[i]) {
+      taken[i] = 1;
+      ids[j] = beams[i];
+    } else {
+      if (a->seqs.count(fresh)) return PKV_EINVAL;
+      ids[j] = fresh++;
+    }
+  }
+  // reference counts after the forks and frees, then the appends' needs
+  std::unordered_map<int32_t, int32_t> counts;
+  auto count_of = [&](int32_t f) {
+    auto it = counts.find(f);
+    return it == counts.end() ? a->ref[f] : it->second;
+  };
+  for (int32_t i = 0; i < k; ++i) {
+    const int32_t delta = children[i] == 0 ? -1 : children[i] - 1;  // forks add, a free drops
+    if (delta != 0)
+      for (int32_t f : old[i]->frames) counts[f] = count_of(f) + delta;
+  }
+  int64_t freed = 0;
+  for (const auto& kv : counts) freed += kv.second == 0 && a->ref[kv.first] > 0;
+  int64_t need = 0;
+  for (int32_t j = 0; j < k_new; ++j) {
+    const pkv_allocator::Seq& sq = *old[parents[j]];
+    if (sq.len % a->block_size == 0) {
+      need += 1;
+    } else {
+      const int32_t last = sq.frames.back();
+      const int32_t c = count_of(last);
+      if (c > 1) {
+        counts[last] = c - 1;
+        need += 1;
+      }
+    }
+  }
+  if (need > static_cast<int64_t>(a->free_frames.size()) + freed) return PKV_ENOMEM;
+  // forks, in new-beam order
+  for (int32_t j = 0; j < k_new; ++j) {
+    const int32_t i = parents[j];
+    if (ids[j] != beams[i]) {
+      pkv_allocator::Seq c = *old[i];
+      for (int32_t f : c.frames) a->ref[f] += 1;
+      a->seqs.emplace(ids[j], std::move(c));
+    }
+  }
+  // beams without a continuation, in beam order
+  for (int32_t i = 0; i < k; ++i)
+    if (children[i] == 0) pkv_alloc_free_seq(a, beams[i]);
+  // one token per new beam, in order
+  int32_t np = 0;
+  for (int32_t j = 0; j < k_new; ++j) {
+    int32_t src, dst;
+    slots_out[j] = a->append(a->seqs.at(ids[j]), &src, &dst);
+    new_ids_out[j] = ids[j];
+    if (src >= 0) {
+      pairs_out[2 * np] = src;
+      pairs_out[2 * np + 1] = dst;
+      ++np;
+    }
+  }
+  *num_pairs_out = np;
+  *next_id = fresh;
+  return PKV_OK;
+}
+
 pkv_status pkv_alloc_free_seq(pkv_allocator* a, int32_t seq_id) {
   if (!a) return PKV_EINVAL;
   auto it = a->seqs.find(seq_id);

@@ -130,3 +130,73 @@ def test_shared_workload_memory_saving():
     # per prompt: one copy per writer while the partial prompt block is shared
     writers = (inp.gen_lens.reshape(w.num_prompts, n) > 0).sum(axis=1)
     assert pairs == int(np.minimum(writers, n - 1).sum())
+
+
+# ------------------------------------------------------------ beam search (slide 14)
+def test_beam_step_candidates_share_the_prefix_like_forked_processes():
+    """Slide 14: beam candidates share their prefix like forked processes.  Four
+    candidates that all continue one beam hold every full block of it once (count
+    4); the partial last block is copied once per writer while it is shared
+    (slide 13's rule), so 3 copies, and the last writer appends in place."""
+    a = AllocatorModel(64, 4)
+    a.add_seq(0, 10)  # blocks 0, 1 full, block 2 holds 2 tokens
+    ids, slots, pairs, nxt = a.beam_step([0], [0, 0, 0, 0], next_id=100)
+    assert ids == [0, 100, 101, 102] and nxt == 103
+    full = a.tables[0][:2]
+    for s in ids:
+        assert a.tables[s][:2] == full and a.lens[s] == 11
+    assert all(a.ref[b] == 4 for b in full)
+    assert len(pairs) == 3 and all(src == 2 for src, _ in pairs)
+    # each pair's destination became that beam's private last block; the last writer kept the shared one
+    assert [a.tables[s][2] for s in ids[:3]] == [dst for _, dst in pairs]
+    assert a.tables[102][2] == 2 and a.ref[2] == 1
+    # the appended token goes at offset 2 of each beam's last block
+    assert slots == [a.tables[s][2] * 4 + 2 for s in ids]
+
+
+def test_beam_step_frees_dropped_beams_and_copies_only_on_divergence():
+    """Beams with no continuation release their frames (dataarena note section 4
+    step 2); a beam that continues alone writes in place once its last block is
+    private, so copies happen only where a shared partial block diverges."""
+    a = AllocatorModel(64, 4)
+    a.add_seq(0, 8)  # two full blocks
+    ids, _, pairs, nxt = a.beam_step([0], [0, 0], next_id=10)
+    assert ids == [0, 10] and pairs == []  # block boundary: new frames, nothing to copy
+    ids, _, pairs, nxt = a.beam_step([0, 10], [1, 1], next_id=nxt)  # beam 0 dropped, 10 forks
+    assert ids == [10, 11] and pairs and 0 not in a.tables
+    ids, _, pairs, nxt = a.beam_step([10, 11], [0, 1], next_id=nxt)  # each continues itself
+    assert pairs == []  # both last blocks are private now
+    st = a.stats()
+    assert st["used_blocks"] == 2 + 2 and st["logical_blocks"] == 2 * 3
+
+
+def test_beam_tree_frames_closed_form():
+    """k beams forked from a P-token prompt (P a multiple of B), each continuing
+    itself for T steps, hold P/B + k * ceil(T/B) frames against k * (P/B +
+    ceil(T/B)) unshared: the saving the pages quote 'up to 55 %' for beam search."""
+    B, P, k, T = 16, 1024, 4, 100
+    a = AllocatorModel(4096, B)
+    a.add_seq(0, P)
+    beams, nxt = [0], 1
+    beams, _, _, nxt = a.beam_step(beams, [0] * k, nxt)
+    for _ in range(T - 1):
+        beams, _, pairs, nxt = a.beam_step(beams, list(range(k)), nxt)
+        assert pairs == []
+    st = a.stats()
+    tb = -(-T // B)
+    assert st["used_blocks"] == P // B + k * tb
+    assert st["logical_blocks"] == k * (P // B + tb)
+
+
+def test_beam_step_enomem_changes_nothing():
+    a = AllocatorModel(4, 4)
+    a.add_seq(0, 6)  # 2 frames, the second holding 2 tokens
+    snap = lambda: ({k: list(v) for k, v in a.tables.items()}, dict(a.lens), list(a.ref), list(a.free))
+    before = snap()
+    with pytest.raises(AllocatorError):
+        a.beam_step([0], [0, 0, 0, 0], next_id=5)  # 3 copies need 3 frames, 2 are free
+    assert snap() == before
+    with pytest.raises(AllocatorError):
+        a.beam_step([0], [1], next_id=5)  # parent index out of range
+    with pytest.raises(AllocatorError):
+        a.beam_step([0, 0], [0], next_id=5)  # repeated beam

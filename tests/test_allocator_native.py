@@ -134,6 +134,59 @@ def test_random_scripts_match_the_model(seed):
     same_state(n, m, live, 64)
 
 
+@pytest.mark.parametrize("seed", range(6))
+def test_beam_search_scripts_match_the_model(seed):
+    """Beam-search steps (slide 14's block tree) on the native allocator and the
+    model: same ids, slots, copy pairs, tables, counts and free queue, including
+    width changes, dropped beams and pool exhaustion (all-or-nothing)."""
+    rng = np.random.default_rng(300 + seed)
+    N, Bsz = int(rng.integers(12, 64)), int(rng.choice([8, 16, 32]))
+    order = rng.permutation(N).astype(np.int32)
+    n, m = BlockAllocator(N, Bsz, order), AllocatorModel(N, Bsz, order)
+    P = int(rng.integers(1, 4 * Bsz))
+    assert n.add_seq(0, P).tolist() == m.add_seq(0, P)
+    beams, nid_n, nid_m, failures = [0], 1, 1, 0
+    for step in range(120):
+        k = len(beams)
+        # mostly narrow steps; now and then a wide one that can exhaust the pool
+        k_new = int(rng.integers(8, 33)) if rng.random() < 0.1 else int(rng.integers(1, 6))
+        # skewed parents: most candidates continue the first (best) beams
+        parents = [int(min(k - 1, rng.geometric(0.5) - 1)) for _ in range(k_new)]
+        try:
+            ids, slots, pairs, nid_m = m.beam_step(beams, parents, nid_m)
+        except AllocatorError:
+            failures += 1
+            with pytest.raises(PkvError) as e:
+                n.beam_step(beams, parents, nid_n)
+            assert e.value.status == PKV_ENOMEM
+            # free a beam to make room, as a scheduler would
+            if len(beams) > 1:
+                victim = beams.pop()
+                m.free_seq(victim)
+                n.free_seq(victim)
+            continue
+        ids_n, slots_n, pairs_n, nid_n = n.beam_step(beams, parents, nid_n)
+        assert ids_n.tolist() == ids and slots_n.tolist() == slots
+        assert pairs_n.tolist() == pairs and nid_n == nid_m
+        beams = ids
+        if step % 10 == 0:
+            same_state(n, m, beams, 4 * N)
+    same_state(n, m, beams, 4 * N)
+    assert n.stats() == m.stats()
+    assert failures > 0 or seed in (2, 4)  # the pool runs out in most scripts
+
+
+def test_beam_step_rejects_bad_arguments():
+    n = BlockAllocator(16, 4)
+    n.add_seq(0, 5)
+    n.add_seq(1, 5)
+    for beams, parents, nid in (([0, 0], [0], 5), ([0, 7], [0], 5), ([0, 1], [2], 5), ([0, 1], [0, 0], 1)):
+        with pytest.raises(PkvError) as e:
+            n.beam_step(beams, parents, nid)
+        assert e.value.status == PKV_EINVAL
+    assert n.stats()["logical_blocks"] == 4  # nothing changed
+
+
 def test_decode_workload_tables_follow_the_frame_order():
     w = wl.WORKLOADS["gqa8b"]
     inp = wl.make_decode_inputs(w, num_seqs=16)
@@ -183,3 +236,15 @@ def test_kv_memory_report_matches_the_model():
     assert rep["sharing_frames"] == ms["used_blocks"]
     assert rep["sharing_unshared_frames"] == ms["logical_blocks"]
     assert rep["sharing_cow_copies"] == copies
+
+    bm = wl.make_beam_inputs()
+    m = AllocatorModel(bm.w.num_blocks, bm.w.block_size, bm.frame_order)
+    m.add_seq(0, bm.prompt_len)
+    beams, nid, copies = [0], 1, 0
+    for step in range(bm.steps):
+        beams, _, pairs, nid = m.beam_step(beams, bm.parents[step], nid)
+        copies += len(pairs)
+    ms = m.stats()
+    assert rep["beam_frames"] == ms["used_blocks"] and rep["beam_unshared_frames"] == ms["logical_blocks"]
+    assert rep["beam_cow_copies"] == copies
+    assert rep["beam_saving_pct"] == round(100.0 * (1 - ms["used_blocks"] / ms["logical_blocks"]), 2)

@@ -280,6 +280,60 @@ def test_shared_prefix_parallel_sampling_with_copy_on_write():
     assert max_abs_err(out, ref) <= TOL[w.dtype]
 
 
+def test_beam_search_block_tree_decode():
+    """Beam search over a block tree (slide 14): 4 beams from one 1000-token
+    prompt, 200 steps.  Each step goes allocator beam_step (forks, frees,
+    appends) -> copy_blocks (CoW pairs) -> cache write of the new tokens; the
+    native allocator and the model must agree on every step.  Then decode the
+    final beams with the same kernel against the oracle's replay, and check that
+    the tree holds far fewer frames than unshared beams would."""
+    Bn = _bin()
+    inp = wl.make_beam_inputs()
+    w = inp.w
+    shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+    td = torch_dtype(w.dtype)
+    gk = torch.full(shape, POISON[w.dtype], dtype=torch.int16, device="cuda").view(td)
+    gv = torch.full(shape, POISON[w.dtype], dtype=torch.int16, device="cuda").view(td)
+    ok = np.full(shape, POISON[w.dtype], np.uint16)
+    ov = np.full(shape, POISON[w.dtype], np.uint16)
+    na = Bn.BlockAllocator(w.num_blocks, w.block_size, inp.frame_order)
+    ma = AllocatorModel(w.num_blocks, w.block_size, inp.frame_order)
+    slots = na.add_seq(0, inp.prompt_len)
+    assert slots.tolist() == ma.add_seq(0, inp.prompt_len)
+    Bn.reshape_and_cache(to_dev(inp.prompt_k, w.dtype), to_dev(inp.prompt_v, w.dtype), gk, gv,
+                         torch.from_numpy(slots).cuda())
+    oracle.reshape_and_cache(ok, ov, inp.prompt_k, inp.prompt_v, slots, w.block_size)
+    beams, nid_n, nid_m = np.zeros(1, np.int32), 1, 1
+    for step in range(inp.steps):
+        ids, slots, pairs, nid_n = na.beam_step(beams, inp.parents[step], nid_n)
+        e_ids, e_slots, e_pairs, nid_m = ma.beam_step(beams.tolist(), inp.parents[step], nid_m)
+        assert ids.tolist() == e_ids and slots.tolist() == e_slots and pairs.tolist() == e_pairs
+        if len(pairs):
+            Bn.copy_blocks(gk, gv, torch.from_numpy(pairs).cuda())
+            oracle.copy_blocks(ok, ov, pairs)
+        Bn.reshape_and_cache(to_dev(inp.step_k[step], w.dtype), to_dev(inp.step_v[step], w.dtype), gk, gv,
+                             torch.from_numpy(slots).cuda())
+        oracle.reshape_and_cache(ok, ov, inp.step_k[step], inp.step_v[step], slots, w.block_size)
+        beams = ids
+    table, lens = na.block_table(beams, w.max_blocks_per_seq)
+    mt, ml = ma.block_table(beams.tolist(), w.max_blocks_per_seq)
+    assert table.tolist() == mt and lens.tolist() == ml
+    assert (lens == inp.prompt_len + inp.steps).all()
+    st = na.stats()
+    assert st["used_blocks"] < 0.5 * st["logical_blocks"]  # the tree, not copies
+    q = to_dev(inp.q, w.dtype)
+    out = torch.empty_like(q)
+    Bn.paged_attention_decode(out, q, gk, gv, torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda(),
+                              w.scale, partition_size=512)
+    torch.cuda.synchronize()
+    assert Bn.device_error() == 0
+    used = np.unique(table[table >= 0])
+    assert np.array_equal(from_dev(gk)[used], ok[used]) and np.array_equal(from_dev(gv)[used], ov[used])
+    ref = oracle.paged_decode(inp.q, ok, ov, np.array(mt, np.int32), np.array(ml, np.int32), w.scale,
+                              w.num_kv_heads, w.block_size, w.dtype)
+    assert max_abs_err(out, ref) <= TOL[w.dtype]
+
+
 # ------------------------------------------------------------ bad device data
 def test_bad_indices_set_device_flags_without_faulting():
     B = _bin()

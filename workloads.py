@@ -53,6 +53,7 @@ class Workload:
     scale: float
     k_scale: float = 1.0
     # length law: ("uniform", lo, hi) | ("lognormal", median, sigma, lo, hi) | ("shared", prompt, gmax)
+    # | ("beam", prompt, steps)
     lengths: tuple = ()
     # shared-prefix workloads only
     num_prompts: int = 0
@@ -90,6 +91,9 @@ WORKLOADS = {
                        lengths=("shared", 1000, 200), num_prompts=16, samples_per_prompt=4),
     "long": Workload("long", 4, 4, 32, 8, 128, 32, 8192, BF16, 1024, 1.0 / math.sqrt(128),
                      lengths=("uniform", 16384, 32768)),
+    # beam search over a block tree: one 1000-token prompt, 4 beams, 200 steps
+    "beam": Workload("beam", 5, 4, 32, 8, 128, 16, 4096, BF16, 76, 1.0 / math.sqrt(128),
+                     lengths=("beam", 1000, 200)),
 }
 
 
@@ -155,7 +159,7 @@ class DecodeInputs:
 
 def make_decode_inputs(name_or_w, seed: int | None = None, num_seqs: int | None = None,
                        lengths: np.ndarray | None = None) -> DecodeInputs:
-    """Seeded decode batch for one of the workloads (not ``shared``).
+    """Seeded decode batch for one of the workloads (not ``shared`` or ``beam``).
 
     ``num_seqs`` truncates the batch (the first sequences of the same draw of
     lengths are kept, so a truncated batch is a prefix of the full one only in
@@ -164,6 +168,8 @@ def make_decode_inputs(name_or_w, seed: int | None = None, num_seqs: int | None 
     w = WORKLOADS[name_or_w] if isinstance(name_or_w, str) else name_or_w
     if w.lengths and w.lengths[0] == "shared":
         raise ValueError("use make_shared_inputs for the shared-prefix workload")
+    if w.lengths and w.lengths[0] == "beam":
+        raise ValueError("use make_beam_inputs for the beam-search workload")
     rng = np.random.default_rng(w.seed if seed is None else seed)
     lens = draw_lengths(w, rng)
     if lengths is not None:
@@ -221,6 +227,47 @@ def make_shared_inputs(seed: int | None = None, num_prompts: int | None = None) 
     offs = np.zeros(w.num_seqs + 1, dtype=np.int64)
     np.cumsum(gen, out=offs[1:])
     return SharedInputs(w, prompt_len, gen, frame_order, q, pk, pv, gk, gv, offs)
+
+
+@dataclasses.dataclass
+class BeamInputs:
+    """Beam-search script over a block tree (slide 14).
+
+    One prompt of ``prompt_len`` tokens; at each of ``steps`` steps the ``k``
+    beams are replaced by ``k`` candidates, candidate j continuing beam
+    ``parents[step, j]`` with one token whose K/V rows are ``step_k[step, j]``
+    (step 0 starts from the prompt alone, so ``parents[0]`` is all 0).
+    Parents are drawn skewed towards the first beams (geometric, p = 1/2), the
+    way the best-scoring beams collect most continuations; the scores themselves
+    are not modelled.  ``q`` holds the final beams' queries.
+    """
+    w: Workload
+    prompt_len: int
+    k: int
+    steps: int
+    parents: np.ndarray       # int32 [steps, k]
+    frame_order: np.ndarray   # int32 [N]
+    q: np.ndarray             # uint16 [k, Hq, D]
+    prompt_k: np.ndarray      # uint16 [prompt_len, Hkv, D]
+    prompt_v: np.ndarray
+    step_k: np.ndarray        # uint16 [steps, k, Hkv, D]
+    step_v: np.ndarray
+
+
+def make_beam_inputs(seed: int | None = None, steps: int | None = None) -> BeamInputs:
+    w = WORKLOADS["beam"]
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    prompt_len, nsteps = w.lengths[1], w.lengths[2] if steps is None else steps
+    k = w.num_seqs
+    parents = np.minimum(rng.geometric(0.5, size=(nsteps, k)) - 1, k - 1).astype(np.int32)
+    parents[0] = 0  # the first step continues the single prompt beam k times
+    frame_order = rng.permutation(w.num_blocks).astype(np.int32)
+    q = _normal_bits(rng, (k, w.num_heads, w.head_dim), w.dtype)
+    pk = _normal_bits(rng, (prompt_len, w.num_kv_heads, w.head_dim), w.dtype)
+    pv = _normal_bits(rng, (prompt_len, w.num_kv_heads, w.head_dim), w.dtype)
+    sk = _normal_bits(rng, (nsteps, k, w.num_kv_heads, w.head_dim), w.dtype)
+    sv = _normal_bits(rng, (nsteps, k, w.num_kv_heads, w.head_dim), w.dtype)
+    return BeamInputs(w, prompt_len, k, nsteps, parents, frame_order, q, pk, pv, sk, sv)
 
 
 def make_token_rows(rng_seed: int, num_tokens: int, num_kv_heads: int, head_dim: int,
