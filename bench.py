@@ -574,6 +574,10 @@ def kv_memory_report(w: wl.Workload, lens: np.ndarray) -> dict:
     beam_saving_pct: the same for 4 beams over a block tree (slide 14), 200 steps
     from one 1000-token prompt (kashii section 3: beam search memory cut by up to
     55 %).
+    prefix_cache_*: 64 requests on 4 shared 1024-token system prompts through
+    the prefix cache (dataarena note section 3.1): prompt tokens whose KV is
+    reused instead of written, and frames held against the frames the same
+    prompts take without the cache.
     """
     from paged_kv_cache_419_b200 import binding as pkv
 
@@ -609,6 +613,13 @@ def kv_memory_report(w: wl.Workload, lens: np.ndarray) -> dict:
         beam_copies += len(pairs)
     bs = a.stats()
     a.close()
+    px = wl.make_prefix_inputs()
+    wp = px.w
+    a = pkv.BlockAllocator(wp.num_blocks, wp.block_size, px.frame_order)
+    cached = sum(a.add_seq_cached(i, px.token_ids[i])[1] for i in range(wp.num_seqs))
+    ps = a.stats()
+    a.close()
+    prompt_tokens = int(sum(len(t) for t in px.token_ids))
     return {
         "useful_kv_pct": round(100.0 * st["tokens"] / capacity, 2),
         "frames": int(st["used_blocks"]), "tokens": int(st["tokens"]), "block_size": w.block_size,
@@ -619,6 +630,8 @@ def kv_memory_report(w: wl.Workload, lens: np.ndarray) -> dict:
         "beam_saving_pct": round(100.0 * (1 - bs["used_blocks"] / bs["logical_blocks"]), 2),
         "beam_frames": int(bs["used_blocks"]), "beam_unshared_frames": int(bs["logical_blocks"]),
         "beam_cow_copies": int(beam_copies),
+        "prefix_cache_reused_tokens_pct": round(100.0 * cached / prompt_tokens, 2),
+        "prefix_cache_frames": int(ps["used_blocks"]), "prefix_cache_uncached_frames": int(ps["logical_blocks"]),
     }
 
 

@@ -245,6 +245,7 @@ typedef struct {
   int64_t tokens;         /* sum of the live sequences' lengths */
   int64_t shared_blocks;  /* frames with count > 1 */
   int64_t logical_blocks; /* sum of the live sequences' table lengths */
+  int64_t cached_blocks;  /* frames holding a prefix-cache key (in use or free) */
 } pkv_alloc_stats_t;
 
 pkv_status pkv_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* frame_order,
@@ -254,6 +255,27 @@ void pkv_alloc_destroy(pkv_allocator* alloc);
  * NULL) receives the slot of every prompt token. */
 pkv_status pkv_alloc_add_seq(pkv_allocator* alloc, int32_t seq_id, int32_t prompt_len,
                              int64_t* slots_out);
+/*
+ * Automatic prefix caching (dataarena note section 3.1: a hash of each prompt
+ * block; a request whose block hash already has a frame maps its logical block
+ * to that frame and increments its reference count: no KV is recomputed).
+ * Like pkv_alloc_add_seq for a prompt of token_ids[0..prompt_len-1], except that
+ * each full block j gets the key pkv_block_hash(key of block j-1, or NULL for
+ * j = 0, its B token ids).  The leading blocks whose keys are cached reuse their
+ * frames (count + 1; a cached frame that was free leaves the free queue); the
+ * rest take fresh frames from the free queue, and their full blocks enter the
+ * cache.  *cached_tokens_out = B x the reused blocks: the caller writes K/V only
+ * for tokens from there on.  A cached frame keeps its key while it sits free
+ * and loses it when taken for other content.  All-or-nothing on PKV_ENOMEM.
+ */
+pkv_status pkv_alloc_add_seq_cached(pkv_allocator* alloc, int32_t seq_id, const int32_t* token_ids,
+                                    int32_t prompt_len, int64_t* slots_out,
+                                    int32_t* cached_tokens_out);
+/* The prefix-cache key of a block: SHA-256 (FIPS 180-4) of the 32-byte parent
+ * key (32 zero bytes when parent_key is NULL) followed by token_ids[0..n-1] as
+ * little-endian int32; 32 bytes into key_out. */
+pkv_status pkv_block_hash(const uint8_t* parent_key, const int32_t* token_ids, int32_t n,
+                          uint8_t* key_out);
 /* child shares all of parent's frames (parallel sampling, beam search). */
 pkv_status pkv_alloc_fork(pkv_allocator* alloc, int32_t parent, int32_t child);
 /* Reserve the slot of the next token of seq_id; *cow_src/*cow_dst = -1 unless a

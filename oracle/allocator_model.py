@@ -30,9 +30,21 @@ Readings where the pages are silent:
   and the shared frame's count drops by one.  A full last block is never copied:
   the writer simply starts a new frame.
 * slot = frame * B + offset (offset = token index mod B).
+
+Automatic prefix caching (dataarena note, section 3.1: a cryptographic hash of
+each prompt block; a request whose block hash already has a frame maps its
+logical block to it and increments the count, so no KV is recomputed).  Readings:
+
+* Only full prompt blocks are keyed; the key of block j is SHA-256 of the key of
+  block j-1 (32 zero bytes for j = 0) and block j's token ids as little-endian
+  int32, so equal keys mean equal prefixes and hits are always a leading run.
+* A cached frame whose count falls to 0 returns to the free queue with its key;
+  a later hit takes it back out of the queue, and taking it for other content
+  drops the key.
 """
 from __future__ import annotations
 
+import hashlib
 from collections import deque
 
 ENOMEM = "ENOMEM"
@@ -55,6 +67,8 @@ class AllocatorModel:
         self.ref = [0] * num_blocks
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
+        self.cache: dict[bytes, int] = {}      # prefix-cache key -> frame
+        self.frame_key: dict[int, bytes] = {}  # frame -> its key
 
     # -- queries -----------------------------------------------------------
     def slot(self, seq: int, t: int) -> int:
@@ -76,13 +90,62 @@ class AllocatorModel:
         tokens = sum(self.lens.values())
         logical = sum(len(t) for t in self.tables.values())
         return {"used_blocks": used, "free_blocks": len(self.free), "tokens": tokens,
-                "shared_blocks": shared, "logical_blocks": logical}
+                "shared_blocks": shared, "logical_blocks": logical, "cached_blocks": len(self.cache)}
 
     # -- operations --------------------------------------------------------
     def _take(self) -> int:
         b = self.free.popleft()
         self.ref[b] = 1
+        key = self.frame_key.pop(b, None)  # new content: the frame leaves the prefix cache
+        if key is not None:
+            del self.cache[key]
         return b
+
+    @staticmethod
+    def block_key(parent, tokens) -> bytes:
+        """Prefix-cache key of a full block (dataarena note section 3.1: a
+        cryptographic hash of each prompt block): SHA-256 of the previous block's
+        key (32 zero bytes for the first block) and the block's token ids as
+        little-endian int32, so that equal keys mean equal prefixes."""
+        data = (parent if parent is not None else bytes(32)) + b"".join(
+            int(t).to_bytes(4, "little", signed=True) for t in tokens)
+        return hashlib.sha256(data).digest()
+
+    def add_seq_cached(self, seq: int, token_ids):
+        """Like add_seq for a prompt given by its token ids, through the prefix
+        cache: leading full blocks whose keys are cached map to those frames
+        (count + 1; a free cached frame leaves the free queue), the rest take
+        fresh frames and their full blocks enter the cache.  Returns (slots,
+        cached_tokens)."""
+        toks = [int(t) for t in token_ids]
+        L = len(toks)
+        if seq in self.tables:
+            raise AllocatorError("EINVAL")
+        nb, full = -(-L // self.B), L // self.B
+        keys, hit, parent = [], [], None
+        for j in range(full):
+            parent = self.block_key(parent, toks[j * self.B:(j + 1) * self.B])
+            keys.append(parent)
+            if len(hit) == j and parent in self.cache:
+                hit.append(self.cache[parent])
+        revived = sum(1 for f in hit if self.ref[f] == 0)
+        if nb - len(hit) > len(self.free) - revived:
+            raise AllocatorError(ENOMEM)
+        tab = []
+        for f in hit:
+            if self.ref[f] == 0:
+                self.free.remove(f)
+            self.ref[f] += 1
+            tab.append(f)
+        for j in range(len(hit), nb):
+            f = self._take()
+            tab.append(f)
+            if j < full:
+                self.cache[keys[j]] = f
+                self.frame_key[f] = keys[j]
+        self.tables[seq] = tab
+        self.lens[seq] = L
+        return [self.slot(seq, t) for t in range(L)], len(hit) * self.B
 
     def add_seq(self, seq: int, prompt_len: int):
         """Allocate frames for a prompt of ``prompt_len`` tokens; returns its slots."""
@@ -152,7 +215,7 @@ class AllocatorModel:
                 ids.append(next_id)
                 next_id += 1
         saved = ({k: list(v) for k, v in self.tables.items()}, dict(self.lens), list(self.ref),
-                 deque(self.free))
+                 deque(self.free), dict(self.cache), dict(self.frame_key))
         try:
             for j, p in enumerate(parents):
                 if ids[j] != beams[p]:
@@ -167,7 +230,7 @@ class AllocatorModel:
                 if src >= 0:
                     pairs.append([src, dst])
         except AllocatorError:
-            self.tables, self.lens, self.ref, self.free = saved
+            self.tables, self.lens, self.ref, self.free, self.cache, self.frame_key = saved
             raise
         return ids, slots, pairs, next_id
 

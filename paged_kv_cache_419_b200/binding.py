@@ -29,6 +29,7 @@ EXPORTS = (
     "pkv_copy_blocks", "pkv_alloc_create", "pkv_alloc_destroy", "pkv_alloc_add_seq",
     "pkv_alloc_fork", "pkv_alloc_append", "pkv_alloc_append_batch", "pkv_alloc_free_seq",
     "pkv_alloc_beam_step", "pkv_alloc_block_table", "pkv_alloc_refcount", "pkv_alloc_stats",
+    "pkv_alloc_add_seq_cached", "pkv_block_hash",
 )
 
 
@@ -41,7 +42,20 @@ class PkvError(RuntimeError):
 class AllocStats(ctypes.Structure):
     _fields_ = [("used_blocks", ctypes.c_int64), ("free_blocks", ctypes.c_int64),
                 ("tokens", ctypes.c_int64), ("shared_blocks", ctypes.c_int64),
-                ("logical_blocks", ctypes.c_int64)]
+                ("logical_blocks", ctypes.c_int64), ("cached_blocks", ctypes.c_int64)]
+
+
+def block_hash(parent_key, token_ids) -> bytes:
+    """Prefix-cache key of one block (pkv_block_hash): SHA-256 of the parent key
+    (32 zero bytes when None) and the token ids as little-endian int32."""
+    import numpy as np
+
+    toks = np.ascontiguousarray(token_ids, dtype=np.int32)
+    out = (ctypes.c_uint8 * 32)()
+    par = None if parent_key is None else (ctypes.c_uint8 * 32).from_buffer_copy(bytes(parent_key))
+    _check(lib().pkv_block_hash(par, toks.ctypes.data_as(ctypes.c_void_p), toks.shape[0], out),
+           "pkv_block_hash")
+    return bytes(out)
 
 
 _lib = None
@@ -82,6 +96,8 @@ def lib() -> ctypes.CDLL:
             "pkv_alloc_append_batch": ([P, P, i32, P, P, P], ctypes.c_int),
             "pkv_alloc_free_seq": ([P, i32], ctypes.c_int),
             "pkv_alloc_beam_step": ([P, P, i32, P, i32, P, P, P, P, P], ctypes.c_int),
+            "pkv_alloc_add_seq_cached": ([P, i32, P, i32, P, P], ctypes.c_int),
+            "pkv_block_hash": ([P, P, i32, P], ctypes.c_int),
             "pkv_alloc_block_table": ([P, P, i32, i32, P, P], ctypes.c_int),
             "pkv_alloc_refcount": ([P, i32, P], ctypes.c_int),
             "pkv_alloc_stats": ([P, ctypes.POINTER(AllocStats)], ctypes.c_int),
@@ -256,6 +272,18 @@ class BlockAllocator:
         _check(lib().pkv_alloc_add_seq(self._h, seq_id, prompt_len,
                                        slots.ctypes.data_as(ctypes.c_void_p)), "pkv_alloc_add_seq")
         return slots[:prompt_len]
+
+    def add_seq_cached(self, seq_id: int, token_ids):
+        """New sequence through the prefix cache: returns (slots, cached_tokens)."""
+        np = self._np
+        toks = np.ascontiguousarray(token_ids, dtype=np.int32)
+        n = toks.shape[0]
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        cached = ctypes.c_int32()
+        _check(lib().pkv_alloc_add_seq_cached(self._h, seq_id, toks.ctypes.data_as(ctypes.c_void_p), n,
+                                              slots.ctypes.data_as(ctypes.c_void_p), ctypes.byref(cached)),
+               "pkv_alloc_add_seq_cached")
+        return slots[:n], cached.value
 
     def fork(self, parent: int, child: int):
         _check(lib().pkv_alloc_fork(self._h, parent, child), "pkv_alloc_fork")

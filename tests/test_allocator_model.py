@@ -200,3 +200,76 @@ def test_beam_step_enomem_changes_nothing():
         a.beam_step([0], [1], next_id=5)  # parent index out of range
     with pytest.raises(AllocatorError):
         a.beam_step([0, 0], [0], next_id=5)  # repeated beam
+
+
+# ------------------------------------------------------------ prefix caching (dataarena note 3.1)
+def _prompt(rng, n):
+    return [int(x) for x in rng.integers(0, 32000, size=n)]
+
+
+def test_prefix_cache_second_request_maps_to_the_same_frames():
+    """A second request with the same system prompt maps its logical blocks to
+    the frames of the first (count 2) and needs no KV written for them; only the
+    full blocks are cached, so a private suffix and the partial last block get
+    their own frames."""
+    rng = np.random.default_rng(1)
+    B = 16
+    system = _prompt(rng, 5 * B)  # five full blocks
+    a = AllocatorModel(64, B)
+    s1, c1 = a.add_seq_cached(0, system + _prompt(rng, 20))
+    assert c1 == 0 and len(a.cache) == 6  # 5 system blocks + 1 full user block
+    s2, c2 = a.add_seq_cached(1, system + _prompt(rng, 7))
+    assert c2 == 5 * B
+    assert a.tables[1][:5] == a.tables[0][:5] and a.tables[1][5] != a.tables[0][5]
+    assert all(a.ref[f] == 2 for f in a.tables[0][:5])
+    assert s2[:5 * B] == s1[:5 * B]  # the cached tokens' slots are the first request's
+    st = a.stats()
+    assert st["used_blocks"] == 6 + 1 + 1 and st["logical_blocks"] == 7 + 6
+
+
+def test_prefix_cache_keys_chain_the_whole_prefix():
+    """A block's key covers every earlier token: a request that differs only in
+    its first block reuses nothing, even where later blocks hold equal tokens."""
+    rng = np.random.default_rng(2)
+    B = 8
+    blocks = [_prompt(rng, B) for _ in range(4)]
+    a = AllocatorModel(64, B)
+    a.add_seq_cached(0, sum(blocks, []))
+    other = _prompt(rng, B)
+    _, c = a.add_seq_cached(1, other + sum(blocks[1:], []))
+    assert c == 0 and not set(a.tables[1]) & set(a.tables[0])
+    k0 = AllocatorModel.block_key(None, blocks[0])
+    assert a.cache[AllocatorModel.block_key(k0, blocks[1])] == a.tables[0][1]
+
+
+def test_prefix_cache_survives_free_and_is_evicted_only_by_reuse():
+    """Frames of a finished request stay cached while free (a later request
+    revives them out of the free queue); once the pool hands them out for other
+    content their keys are gone."""
+    rng = np.random.default_rng(3)
+    B = 4
+    system = _prompt(rng, 3 * B)
+    a = AllocatorModel(6, B)
+    a.add_seq_cached(0, system)
+    frames = list(a.tables[0])
+    a.free_seq(0)
+    assert a.stats()["cached_blocks"] == 3 and len(a.free) == 6
+    _, c = a.add_seq_cached(1, system)
+    assert c == 3 * B and a.tables[1] == frames and len(a.free) == 3
+    a.free_seq(1)
+    # the free queue now ends with the three cached frames; a 6-block request takes all of them
+    a.add_seq(2, 6 * B)
+    assert a.stats()["cached_blocks"] == 0
+    a.free_seq(2)
+    _, c = a.add_seq_cached(3, system)
+    assert c == 0
+
+
+def test_prefix_cache_enomem_changes_nothing():
+    rng = np.random.default_rng(4)
+    a = AllocatorModel(4, 4)
+    a.add_seq_cached(0, _prompt(rng, 12))
+    snap = ({k: list(v) for k, v in a.tables.items()}, list(a.ref), list(a.free), dict(a.cache))
+    with pytest.raises(AllocatorError):
+        a.add_seq_cached(1, _prompt(rng, 8))  # needs 2 frames, 1 is free
+    assert ({k: list(v) for k, v in a.tables.items()}, list(a.ref), list(a.free), dict(a.cache)) == snap

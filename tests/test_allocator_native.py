@@ -248,3 +248,84 @@ def test_kv_memory_report_matches_the_model():
     assert rep["beam_frames"] == ms["used_blocks"] and rep["beam_unshared_frames"] == ms["logical_blocks"]
     assert rep["beam_cow_copies"] == copies
     assert rep["beam_saving_pct"] == round(100.0 * (1 - ms["used_blocks"] / ms["logical_blocks"]), 2)
+
+    px = wl.make_prefix_inputs()
+    m = AllocatorModel(px.w.num_blocks, px.w.block_size, px.frame_order)
+    cached = sum(m.add_seq_cached(i, px.token_ids[i])[1] for i in range(px.w.num_seqs))
+    ms = m.stats()
+    total = sum(len(t) for t in px.token_ids)
+    assert rep["prefix_cache_frames"] == ms["used_blocks"]
+    assert rep["prefix_cache_uncached_frames"] == ms["logical_blocks"]
+    assert rep["prefix_cache_reused_tokens_pct"] == round(100.0 * cached / total, 2)
+    # every request after the first on a system prompt reuses that prompt's 64 full blocks
+    firsts = len(set(px.system.tolist()))
+    assert cached == (px.w.num_seqs - firsts) * px.prompt_len
+
+
+def test_block_hash_is_sha256():
+    """pkv_block_hash is SHA-256 (FIPS 180-4) of the parent key and the token ids
+    as little-endian int32, checked against hashlib on messages of 0 to 300
+    tokens (1 to 20 SHA-256 blocks) with and without a parent key."""
+    import hashlib
+    from paged_kv_cache_419_b200.binding import block_hash
+
+    rng = np.random.default_rng(11)
+    for n in (0, 1, 7, 8, 15, 16, 31, 32, 100, 300):
+        toks = rng.integers(-2**31, 2**31, size=n, dtype=np.int64).astype(np.int32)
+        for parent in (None, bytes(rng.integers(0, 256, size=32, dtype=np.uint8))):
+            msg = (parent if parent is not None else bytes(32)) + toks.astype("<i4").tobytes()
+            assert block_hash(parent, toks) == hashlib.sha256(msg).digest()
+    assert AllocatorModel.block_key(None, [1, 2, 3]) == block_hash(None, [1, 2, 3])
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_prefix_cache_scripts_match_the_model(seed):
+    """Requests built from a few shared system prompts plus private suffixes,
+    mixed with frees, appends and forks: the native allocator and the model agree
+    on slots, cached-token counts, tables, counts and the cache size."""
+    rng = np.random.default_rng(500 + seed)
+    N, Bsz = int(rng.integers(24, 120)), int(rng.choice([4, 8, 16]))
+    order = rng.permutation(N).astype(np.int32)
+    n, m = BlockAllocator(N, Bsz, order), AllocatorModel(N, Bsz, order)
+    systems = [[int(x) for x in rng.integers(0, 1000, size=int(rng.integers(0, 5 * Bsz)))] for _ in range(3)]
+    live, next_id, hits = [], 0, 0
+    for step in range(300):
+        op = rng.choice(["req", "free", "append", "fork"], p=[0.4, 0.3, 0.2, 0.1])
+        if op == "req" or not live:
+            toks = systems[int(rng.integers(0, 3))] + [int(x) for x in rng.integers(0, 1000, size=int(rng.integers(0, 2 * Bsz)))]
+            try:
+                exp_slots, exp_cached = m.add_seq_cached(next_id, toks)
+            except AllocatorError:
+                with pytest.raises(PkvError) as e:
+                    n.add_seq_cached(next_id, toks)
+                assert e.value.status == PKV_ENOMEM
+            else:
+                slots, cached = n.add_seq_cached(next_id, toks)
+                assert slots.tolist() == exp_slots and cached == exp_cached
+                hits += cached > 0
+                live.append(next_id)
+            next_id += 1
+        elif op == "free":
+            s = int(rng.choice(live))
+            live.remove(s)
+            m.free_seq(s)
+            n.free_seq(s)
+        elif op == "append":
+            s = int(rng.choice(live))
+            try:
+                exp = m.append(s)
+            except AllocatorError:
+                with pytest.raises(PkvError):
+                    n.append(s)
+            else:
+                assert n.append(s) == exp
+        else:
+            p = int(rng.choice(live))
+            m.fork(p, next_id)
+            n.fork(p, next_id)
+            live.append(next_id)
+            next_id += 1
+        if step % 20 == 0:
+            same_state(n, m, live, 4 * N)
+    same_state(n, m, live, 4 * N)
+    assert hits > 0

@@ -334,6 +334,58 @@ def test_beam_search_block_tree_decode():
     assert max_abs_err(out, ref) <= TOL[w.dtype]
 
 
+def test_prefix_cache_reuses_frames_and_writes_no_kv():
+    """Automatic prefix caching (dataarena note section 3.1): 16 requests on 4
+    shared 1024-token system prompts.  Each request goes through the cached
+    add_seq of the native allocator (checked against the model) and writes K/V
+    only for its tokens past the cached ones, so a system prompt is written once.
+    Decoding every request over the shared frames matches the oracle, and the
+    cached frames' contents equal the oracle's."""
+    Bn = _bin()
+    inp = wl.make_prefix_inputs(num_seqs=16)
+    w = inp.w
+    S = w.num_seqs
+    shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+    td = torch_dtype(w.dtype)
+    gk = torch.full(shape, POISON[w.dtype], dtype=torch.int16, device="cuda").view(td)
+    gv = torch.full(shape, POISON[w.dtype], dtype=torch.int16, device="cuda").view(td)
+    ok = np.full(shape, POISON[w.dtype], np.uint16)
+    ov = np.full(shape, POISON[w.dtype], np.uint16)
+    na = Bn.BlockAllocator(w.num_blocks, w.block_size, inp.frame_order)
+    ma = AllocatorModel(w.num_blocks, w.block_size, inp.frame_order)
+    written = 0
+    for i in range(S):
+        slots, cached = na.add_seq_cached(i, inp.token_ids[i])
+        e_slots, e_cached = ma.add_seq_cached(i, inp.token_ids[i])
+        assert slots.tolist() == e_slots and cached == e_cached
+        rows_k = np.concatenate([inp.system_k[inp.system[i]], inp.own_k[inp.own_offsets[i]:inp.own_offsets[i + 1]]])
+        rows_v = np.concatenate([inp.system_v[inp.system[i]], inp.own_v[inp.own_offsets[i]:inp.own_offsets[i + 1]]])
+        new = slice(cached, len(slots))  # only the tokens past the cached prefix
+        Bn.reshape_and_cache(to_dev(rows_k[new], w.dtype), to_dev(rows_v[new], w.dtype), gk, gv,
+                             torch.from_numpy(slots[new].copy()).cuda())
+        oracle.reshape_and_cache(ok, ov, rows_k[new], rows_v[new], slots[new], w.block_size)
+        written += len(slots) - cached
+    total = sum(len(t) for t in inp.token_ids)
+    firsts = len(set(inp.system.tolist()))
+    # each system prompt's full blocks are written once
+    full = (inp.prompt_len // w.block_size) * w.block_size
+    assert written == total - (S - firsts) * full
+    table, lens = na.block_table(np.arange(S, dtype=np.int32), w.max_blocks_per_seq)
+    mt, ml = ma.block_table(range(S), w.max_blocks_per_seq)
+    assert table.tolist() == mt and lens.tolist() == ml
+    q = to_dev(inp.q, w.dtype)
+    out = torch.empty_like(q)
+    Bn.paged_attention_decode(out, q, gk, gv, torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda(),
+                              w.scale)
+    torch.cuda.synchronize()
+    assert Bn.device_error() == 0
+    used = np.unique(table[table >= 0])
+    assert np.array_equal(from_dev(gk)[used], ok[used]) and np.array_equal(from_dev(gv)[used], ov[used])
+    ref = oracle.paged_decode(inp.q, ok, ov, np.array(mt, np.int32), np.array(ml, np.int32), w.scale,
+                              w.num_kv_heads, w.block_size, w.dtype)
+    assert max_abs_err(out, ref) <= TOL[w.dtype]
+
+
 # ------------------------------------------------------------ bad device data
 def test_bad_indices_set_device_flags_without_faulting():
     B = _bin()

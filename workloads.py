@@ -53,7 +53,7 @@ class Workload:
     scale: float
     k_scale: float = 1.0
     # length law: ("uniform", lo, hi) | ("lognormal", median, sigma, lo, hi) | ("shared", prompt, gmax)
-    # | ("beam", prompt, steps)
+    # | ("beam", prompt, steps) | ("prefix", system prompt, max own tokens)
     lengths: tuple = ()
     # shared-prefix workloads only
     num_prompts: int = 0
@@ -91,6 +91,9 @@ WORKLOADS = {
                        lengths=("shared", 1000, 200), num_prompts=16, samples_per_prompt=4),
     "long": Workload("long", 4, 4, 32, 8, 128, 32, 8192, BF16, 1024, 1.0 / math.sqrt(128),
                      lengths=("uniform", 16384, 32768)),
+    # prefix caching: 64 requests on 4 shared 1024-token system prompts + 16-256 own tokens
+    "prefix": Workload("prefix", 6, 64, 32, 8, 128, 16, 8192, BF16, 81, 1.0 / math.sqrt(128),
+                       lengths=("prefix", 1024, 256), num_prompts=4),
     # beam search over a block tree: one 1000-token prompt, 4 beams, 200 steps
     "beam": Workload("beam", 5, 4, 32, 8, 128, 16, 4096, BF16, 76, 1.0 / math.sqrt(128),
                      lengths=("beam", 1000, 200)),
@@ -168,8 +171,8 @@ def make_decode_inputs(name_or_w, seed: int | None = None, num_seqs: int | None 
     w = WORKLOADS[name_or_w] if isinstance(name_or_w, str) else name_or_w
     if w.lengths and w.lengths[0] == "shared":
         raise ValueError("use make_shared_inputs for the shared-prefix workload")
-    if w.lengths and w.lengths[0] == "beam":
-        raise ValueError("use make_beam_inputs for the beam-search workload")
+    if w.lengths and w.lengths[0] in ("beam", "prefix"):
+        raise ValueError("use make_beam_inputs / make_prefix_inputs for these workloads")
     rng = np.random.default_rng(w.seed if seed is None else seed)
     lens = draw_lengths(w, rng)
     if lengths is not None:
@@ -252,6 +255,53 @@ class BeamInputs:
     prompt_v: np.ndarray
     step_k: np.ndarray        # uint16 [steps, k, Hkv, D]
     step_v: np.ndarray
+
+
+@dataclasses.dataclass
+class PrefixInputs:
+    """Requests that share system prompts (automatic prefix caching).
+
+    Request i is system prompt ``system[i]`` (``prompt_len`` tokens) followed by
+    ``own_lens[i]`` tokens of its own; ``token_ids[i]`` holds its whole prompt.
+    K/V rows depend on the token's prefix: system prompt p's rows are
+    ``system_k[p]`` (equal in every request that uses p), request i's own rows
+    are ``own_k[own_offsets[i]:own_offsets[i+1]]``.
+    """
+    w: Workload
+    prompt_len: int
+    system: np.ndarray        # int32 [S]
+    own_lens: np.ndarray      # int32 [S]
+    token_ids: list           # S int32 arrays
+    frame_order: np.ndarray   # int32 [N]
+    q: np.ndarray             # uint16 [S, Hq, D]
+    system_k: np.ndarray      # uint16 [P, prompt_len, Hkv, D]
+    system_v: np.ndarray
+    own_k: np.ndarray         # uint16 [sum own, Hkv, D]
+    own_v: np.ndarray
+    own_offsets: np.ndarray   # int64 [S + 1]
+
+
+def make_prefix_inputs(seed: int | None = None, num_seqs: int | None = None) -> PrefixInputs:
+    w = WORKLOADS["prefix"]
+    if num_seqs is not None:
+        w = dataclasses.replace(w, num_seqs=num_seqs)
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    plen, omax = w.lengths[1], w.lengths[2]
+    system = rng.integers(0, w.num_prompts, size=w.num_seqs).astype(np.int32)
+    own = rng.integers(16, omax, size=w.num_seqs, endpoint=True).astype(np.int32)
+    sys_tokens = rng.integers(0, 128000, size=(w.num_prompts, plen)).astype(np.int32)
+    token_ids = [np.concatenate([sys_tokens[system[i]], rng.integers(0, 128000, size=own[i]).astype(np.int32)])
+                 for i in range(w.num_seqs)]
+    frame_order = rng.permutation(w.num_blocks).astype(np.int32)
+    q = _normal_bits(rng, (w.num_seqs, w.num_heads, w.head_dim), w.dtype)
+    sk = _normal_bits(rng, (w.num_prompts, plen, w.num_kv_heads, w.head_dim), w.dtype)
+    sv = _normal_bits(rng, (w.num_prompts, plen, w.num_kv_heads, w.head_dim), w.dtype)
+    total = int(own.astype(np.int64).sum())
+    ok = _normal_bits(rng, (total, w.num_kv_heads, w.head_dim), w.dtype)
+    ov = _normal_bits(rng, (total, w.num_kv_heads, w.head_dim), w.dtype)
+    offs = np.zeros(w.num_seqs + 1, dtype=np.int64)
+    np.cumsum(own, out=offs[1:])
+    return PrefixInputs(w, plen, system, own, token_ids, frame_order, q, sk, sv, ok, ov, offs)
 
 
 def make_beam_inputs(seed: int | None = None, steps: int | None = None) -> BeamInputs:
