@@ -508,52 +508,92 @@ def contiguous_compare(args, inp, b, ws, flush, part, device):
 def e2e_run(args, inp, b, ws, part, nbytes, device):
     """The same step through the public API from pinned host buffers: host->device
     copies of the step's inputs (q, the new token's K/V, its slots, the block tables
-    and context lengths) and the device->host read of the output are timed."""
+    and context lengths), the cache write and decode, and the device->host read of
+    the step's output, every step.
+
+    Steps are pipelined the way a serving loop overlaps its transfers: inputs and
+    outputs are double-buffered, the copies in run on one stream, the kernels on
+    another and the copies out on a third, so step k+1's inputs and step k-1's
+    output cross the host link while step k computes.  Each stage of each buffer
+    is a CUDA graph of the public calls (eager calls with --eager); the stages are
+    ordered by events.  The time is the device time from the first step's input
+    copy to the last step's output copy, divided by the steps."""
     from paged_kv_cache_419_b200 import binding as pkv
 
     w = inp.w
-    host = {name: b[name].cpu().pin_memory() for name in ("q", "new_k", "new_v", "slots", "tables", "lens")}
-    out_h = torch.empty(b["out"].shape, dtype=b["out"].dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * out_h.element_size()
-    dev = {name: torch.empty_like(b[name]) for name in host}
+    names = ("q", "new_k", "new_v", "slots", "tables", "lens")
+    host = [{n: b[n].cpu().pin_memory() for n in names} for _ in range(2)]
+    out_h = [torch.empty(b["out"].shape, dtype=b["out"].dtype).pin_memory() for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host[0].values())
+    d2h = out_h[0].numel() * out_h[0].element_size()
+    dev = [{n: torch.empty_like(b[n]) for n in names} for _ in range(2)]
+    out_d = [torch.empty_like(b["out"]) for _ in range(2)]
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-    def step():
-        for name, t in host.items():
-            dev[name].copy_(t, non_blocking=True)
-        pkv.reshape_and_cache(dev["new_k"], dev["new_v"], b["k_cache"], b["v_cache"], dev["slots"])
-        pkv.paged_attention_decode(b["out"], dev["q"], b["k_cache"], b["v_cache"], dev["tables"],
-                                   dev["lens"], w.scale, partition_size=part, workspace=ws)
-        out_h.copy_(b["out"], non_blocking=True)
+    def copy_in(i):
+        for n in names:
+            dev[i][n].copy_(host[i][n], non_blocking=True)
 
-    for _ in range(3):
-        step()
+    def compute(i):
+        d = dev[i]
+        pkv.reshape_and_cache(d["new_k"], d["new_v"], b["k_cache"], b["v_cache"], d["slots"])
+        pkv.paged_attention_decode(out_d[i], d["q"], b["k_cache"], b["v_cache"], d["tables"], d["lens"],
+                                   w.scale, partition_size=part, workspace=ws)
+
+    def copy_out(i):
+        out_h[i].copy_(out_d[i], non_blocking=True)
+
+    stages = {"in": copy_in, "comp": compute, "out": copy_out}
+    streams = {"in": s_in, "comp": s_comp, "out": s_out}
+    run = {(k, i): (lambda f=f, i=i: f(i)) for k, f in stages.items() for i in range(2)}
+    for _ in range(2):  # warm-up (and first-call set-up) in stream order
+        for i in range(2):
+            for k in ("in", "comp", "out"):
+                run[(k, i)]()
     torch.cuda.synchronize()
-    run, mode = step, "eager public-API calls"
+    mode = "eager public-API calls, pipelined over 3 streams"
     if not args.eager:
-        # The same calls captured once as a CUDA graph (as a serving engine runs
-        # its step): the pinned host->device copies, the cache write, the decode
-        # and the device->host read are nodes of the graph, replayed every step.
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=side):
-            step()
-        torch.cuda.current_stream().wait_stream(side)
-        for _ in range(2):
-            g.replay()
+        graphs = {}
+        for key in run:
+            st = streams[key[0]]
+            st.wait_stream(torch.cuda.current_stream())
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st):
+                run[key]()
+            graphs[key] = g
         torch.cuda.synchronize()
-        run, mode = g.replay, "CUDA graph of the public-API step (copies included)"
-    K = args.steps
-    evs = []
-    for _ in range(K):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        run()
-        e1.record()
-        evs.append((e0, e1))
+        run = {key: g.replay for key, g in graphs.items()}
+        mode = "CUDA graphs of the public-API calls, pipelined over 3 streams (copies in, kernels, copy out)"
+
+    K = max(args.steps, 4)
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    ms = statistics.mean(a.elapsed_time(c) for a, c in evs)
+    for k in range(K):
+        i = k % 2
+        with torch.cuda.stream(s_in):
+            if k == 0:
+                t0.record()
+            if k >= 2:
+                s_in.wait_event(comp_done[i])   # step k-2 no longer reads these inputs
+            run[("in", i)]()
+            in_done[i].record()
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(in_done[i])
+            if k >= 2:
+                s_comp.wait_event(out_done[i])  # step k-2's output has been read out
+            run[("comp", i)]()
+            comp_done[i].record()
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[i])
+            run[("out", i)]()
+            out_done[i].record()
+            if k == K - 1:
+                t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / K
     ms_max, _, _ = aggregate(ms, 0.0, 0.0, device)
     return {"value": round(nbytes["step"] / (ms_max * 1e-3) / 1e9, 1), "unit": "GB/s",
             "ms_per_step": round(ms_max, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
