@@ -72,6 +72,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--op", choices=["decode", "cache-ops"], default="decode",
+                    help="cache-ops: time reshape_and_cache and copy_blocks alone at HBM-bound sizes")
     ap.add_argument("--workload", default="gqa8b", choices=["tiny", "mha13b", "gqa8b", "long"])
     ap.add_argument("--l2-flush", choices=["clean", "dirty"], default="clean",
                     help="L2 eviction before each timed step: 256 MiB write then read (clean) or write only")
@@ -600,6 +602,62 @@ def e2e_run(args, inp, b, ws, part, nbytes, device):
             "execution": mode}
 
 
+# ------------------------------------------------------------------ cache ops alone
+def run_cache_ops(args, local):
+    """reshape_and_cache and copy_blocks on their own at sizes where HBM bounds
+    them (the decode step's own cache write moves only 1 MB and is launch-bound):
+    a gqa8b-shaped pool of 16,384 frames (8 kv heads x 16 x 128 bf16, 1.07 GB for
+    K and V), 32,768 new tokens written at distinct random slots, and 2,048 copy
+    pairs between distinct random frames.  L2 flushed before every launch; CUDA
+    events on the launching stream.  Algorithmic bytes: the cache write reads key
+    and value and writes both (plus the int64 slots); the block copy reads and
+    writes both frames of every pair.  One JSON line per kernel."""
+    from paged_kv_cache_419_b200 import binding as pkv
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    N, Hkv, B, D, T, P = 16384, 8, 16, 128, 32768, 2048
+    rng = np.random.default_rng(21)
+    kc = torch.zeros((N, Hkv, B, D), dtype=torch.bfloat16, device=device)
+    vc = torch.zeros_like(kc)
+    key = torch.randn((T, Hkv, D), dtype=torch.bfloat16, device=device)
+    val = torch.randn_like(key)
+    slots = torch.from_numpy(rng.choice(N * B, size=T, replace=False).astype(np.int64)).to(device)
+    frames = rng.permutation(N)[: 2 * P].astype(np.int64)
+    pairs = torch.from_numpy(np.stack([frames[:P], frames[P:]], axis=1).copy()).to(device)
+    flush = torch.zeros(2 * L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    frame_bytes = Hkv * B * D * 2
+    ops = {
+        "reshape_and_cache": (lambda: pkv.reshape_and_cache(key, val, kc, vc, slots),
+                              4 * T * Hkv * D * 2 + T * 8, f"{T} tokens, 8 kv heads x 128 bf16"),
+        "copy_blocks": (lambda: pkv.copy_blocks(kc, vc, pairs),
+                        2 * 2 * P * frame_bytes, f"{P} pairs of 32 KB frames, K and V"),
+    }
+    peak, peak_kind = measured_hbm_peak()
+    for name, (fn, nbytes, what) in ops.items():
+        for _ in range(max(args.warmup, 3)):
+            l2_flush(flush, args.l2_flush)
+            fn()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(args.steps):
+            l2_flush(flush, args.l2_flush)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        if pkv.device_error():
+            raise RuntimeError(f"device error flags set by {name}")
+        ms = statistics.mean(times)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({"op": name, "metric": f"{name} HBM GB/s", "value": round(gbs, 1), "unit": "GB/s",
+                          "ms": round(ms, 5), "bytes": int(nbytes), "workload": what, "steps": args.steps,
+                          "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                                       "peak_kind": peak_kind, "frac": round(gbs / peak, 4)}}), flush=True)
+
+
 # ------------------------------------------------------------------ KV memory
 def kv_memory_report(w: wl.Workload, lens: np.ndarray) -> dict:
     """KV-cache memory use of this batch and of the parallel-sampling batch, from
@@ -761,6 +819,9 @@ def main(argv=None):
     world, rank, local = dist_env()
     if args.impl == "reference":
         run_reference(args, world, rank, local)
+    elif args.op == "cache-ops":
+        if rank == 0:
+            run_cache_ops(args, local)
     else:
         run_ours(args, world, rank, local)
 

@@ -194,7 +194,8 @@ pkv_status pkv_contiguous_attention_decode(void* out, const void* q, const void*
  *   slot_mapping device int64 [num_tokens]; slots must be distinct (two tokens
  *                writing one slot race).  A slot >= num_blocks * block_size is
  *                not written and sets PKV_DEVERR_SLOT.
- *   head_dim * element size must be a multiple of 16 bytes.
+ *   head_dim * element size must be 16 bytes times a power of two (head_dim 8,
+ *   16, 32, 64, 128, 256 for 16-bit types); other head_dim: PKV_EUNSUPPORTED.
  */
 pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
                                  const int64_t* slot_mapping, int32_t num_tokens,

@@ -352,7 +352,8 @@ pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cac
     return PKV_EINVAL;
   if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EUNSUPPORTED;
   const int32_t row_bytes = head_dim * 2;
-  if (row_bytes % 16 != 0) return PKV_EUNSUPPORTED;
+  // rows move as 16-byte vectors, a power of two of them per row
+  if (row_bytes % 16 != 0 || ((row_bytes / 16) & (row_bytes / 16 - 1)) != 0) return PKV_EUNSUPPORTED;
   if (num_tokens == 0) return PKV_OK;
   if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PKV_EINVAL;
   if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
@@ -387,7 +388,7 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_
   pkv_status st = device_info(&dev);
   if (st != PKV_OK) return st;
   return from_cuda(launch_copy_blocks(k_cache, v_cache, src_dst_pairs, num_pairs, block_bytes,
-                                      num_blocks, dev->err, stream));
+                                      num_blocks, dev->num_sms, dev->err, stream));
 }
 
 }  // extern "C"

@@ -14,6 +14,6 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* k
 
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs,
                                int32_t num_pairs, int64_t block_bytes, int32_t num_blocks,
-                               unsigned int* err, cudaStream_t stream);
+                               int num_sms, unsigned int* err, cudaStream_t stream);
 
 }  // namespace pkv

@@ -103,6 +103,8 @@ def test_cache_ops_reject_bad_arguments_before_launch():
     L = B.lib()
     # head_dim 4 (8 bytes per row) cannot be moved in 16-byte vectors
     assert L.pkv_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 4, 16, 8, 0, None) == B.PKV_EUNSUPPORTED
+    # head_dim 96: 12 vectors per row, not a power of two
+    assert L.pkv_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 96, 16, 8, 0, None) == B.PKV_EUNSUPPORTED
     assert L.pkv_reshape_and_cache(None, FAKE, FAKE, FAKE, FAKE, 4, 2, 64, 16, 8, 0, None) == B.PKV_EINVAL
     assert L.pkv_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 64, 16, 8, 0, None) == B.PKV_EINVAL
     assert L.pkv_reshape_and_cache(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 64, 16, 8, 0, None) == B.PKV_OK
