@@ -5,35 +5,42 @@
 // tokens at arbitrary frames of a pool, found through the sequence's block table.
 // Attention is softmax(scale q K^T) V, accumulated in fp32.
 //
-// Kernel design (B200).  Single-token decode is a bandwidth-bound GEMV, so the
-// kernels are built to keep HBM busy, not to feed tensor cores.
+// Kernel design (B200).  The kernels are built to keep HBM busy; the
+// contractions of the G query heads that share a kv head run as small
+// tensor-core tiles only so that issuing them never holds the loads back.
 //
 //  * Work item = (sequence, kv head, context partition).  A context of L tokens
 //    is cut into n = ceil(L / part_tokens) near-equal partitions whose sizes are
-//    multiples of 32 tokens.  All G = Hq/Hkv query heads of the kv head share one
+//    multiples of 64 tokens.  All G = Hq/Hkv query heads of the kv head share one
 //    K/V fetch.
-//  * plan_kernel (one CTA) lists the items, largest first, lists the contexts
-//    that span several partitions, and resets the work counter.
-//  * decode_kernel is persistent: (SM count x occupancy) CTAs, launched with
-//    programmatic dependent launch so that their set-up overlaps the plan.  Each
+//  * plan_kernel (one CTA, plain stream order) lists the items, largest first,
+//    lists the contexts that span several partitions and zeroes their
+//    completion counters.  Partition 0 of the first grid/Hkv sequences is not
+//    listed: decode CTA c starts with it (sequence c / Hkv, kv head c % Hkv),
+//    described from the context length alone, while the plan still runs.
+//  * decode_kernel is persistent: (SM count x occupancy) CTAs, launched behind
+//    the plan with programmatic dependent launch.  After its first item each
 //    CTA takes items from the list with an atomic counter until it runs dry.
 //  * Inside a CTA, warp 4 is the producer: it takes the next item, copies its q
 //    rows into an item slot and streams the item's K and V through a ring of
-//    STAGES shared-memory stages with 1-D bulk copies (one copy per block of K
-//    and of V: a (frame, kv head) tile is contiguous in [N, Hkv, B, D]).  It runs
-//    ahead across items, so the next item's data arrives while the consumers
-//    finish the current one.  mbarriers hand stages and item slots over.
-//  * Stage = 32 logical tokens; consumer warp w owns tokens 8w..8w+7 of each
-//    stage with its own online-softmax state.  Scores: LPT lanes share a token
-//    (16-byte shared loads, packed fp32 FMA), then a reduce-scatter across the
-//    LPT lanes leaves every lane holding the finished score of one head.  PV:
-//    each lane owns D/32 output dims of all G heads.
-//  * Epilogue per item: the four warps merge in shared memory.  A one-partition
-//    context writes `out`; otherwise the partition's normalised output, max and
-//    sum go to the workspace, and merge_kernel (launched behind the decode grid)
-//    merges the partitions of each such context (log-sum-exp) into `out`.
-//  * Scores are kept in base-2 units (q is pre-scaled by scale * log2 e), so the
-//    exponentials are single ex2 instructions.
+//    two 64-token stages with TMA tensor copies (one 128-byte panel of a block
+//    per box, 128-byte swizzle; the ragged end of a context in 8-row boxes).
+//    It runs ahead across items, so the next item's data arrives while the
+//    consumers finish the current one.  mbarriers hand stages (K and V halves
+//    separately) and item slots over.
+//  * Consumer warp w owns tokens 16w..16w+15 of each stage with its own
+//    online-softmax state.  Scores: S^T = Q K^T as mma.sync m16n8k16 tiles (fp32
+//    accumulation), K fragments read with ldmatrix from the swizzled stage.  PV:
+//    O^T += V^T P^T, P^T taken from the score accumulators as they lie (rounded
+//    to the input type), V^T read with transposing ldmatrix.
+//  * Epilogue per item: the four warps merge through shared memory in a fixed
+//    order (bit-reproducible).  A one-partition context writes `out`; otherwise
+//    the partition's normalised output, max and sum go to the workspace.  Each
+//    CTA publishes its multi-partition items to per-(sequence, kv head)
+//    counters, and merge_kernel, which runs in the decode grid's tail, merges
+//    each such context (log-sum-exp) into `out` as soon as its count is complete.
+//  * Scores are kept in base-2 units (scale * log2 e folded into one multiply),
+//    so the exponentials are single ex2 instructions.
 #pragma once
 
 #include <cuda.h>
@@ -59,7 +66,7 @@ struct DecodeArgs {
   int32_t num_heads;
   int32_t num_kv_heads;
   int32_t max_ctx;        // capacity in tokens: MB * B (paged) or the contiguous stride
-  int32_t part_tokens;    // maximum tokens per partition (multiple of 32)
+  int32_t part_tokens;    // maximum tokens per partition (multiple of 64)
   int32_t max_parts;      // ceil(max_ctx / part_tokens): upper bound of partitions per context
   float scale_log2;       // scale * log2(e)
   int32_t grid_ctas;      // decode CTAs; item c (c < grid_ctas) is CTA c's first item
