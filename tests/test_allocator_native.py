@@ -329,3 +329,108 @@ def test_prefix_cache_scripts_match_the_model(seed):
             same_state(n, m, live, 4 * N)
     same_state(n, m, live, 4 * N)
     assert hits > 0
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_mixed_scripts_match_the_model(seed):
+    """Everything at once: cached and plain prompts, forks, appends and batches,
+    beam steps over a live group of sequences, and frees (which also release
+    cached frames for revival or eviction).  Native allocator and model agree on
+    every result and on the whole state."""
+    rng = np.random.default_rng(900 + seed)
+    N, Bsz = int(rng.integers(20, 96)), int(rng.choice([4, 8, 16]))
+    order = rng.permutation(N).astype(np.int32)
+    n, m = BlockAllocator(N, Bsz, order), AllocatorModel(N, Bsz, order)
+    systems = [[int(x) for x in rng.integers(0, 50, size=int(rng.integers(Bsz, 4 * Bsz)))] for _ in range(2)]
+    live, next_id = [], 0
+    for step in range(400):
+        op = rng.choice(["cached", "plain", "fork", "append", "batch", "beam", "free"],
+                        p=[0.2, 0.1, 0.1, 0.15, 0.1, 0.15, 0.2])
+        if op in ("cached", "plain") or not live:
+            toks = systems[int(rng.integers(0, 2))] + [int(x) for x in rng.integers(0, 50, size=int(rng.integers(0, Bsz)))]
+            try:
+                exp = m.add_seq_cached(next_id, toks) if op == "cached" else (m.add_seq(next_id, len(toks)), 0)
+            except AllocatorError:
+                with pytest.raises(PkvError):
+                    n.add_seq_cached(next_id, toks) if op == "cached" else n.add_seq(next_id, len(toks))
+            else:
+                got = n.add_seq_cached(next_id, toks) if op == "cached" else (n.add_seq(next_id, len(toks)), 0)
+                assert got[0].tolist() == exp[0] and got[1] == exp[1]
+                live.append(next_id)
+            next_id += 1
+        elif op == "fork":
+            p = int(rng.choice(live))
+            m.fork(p, next_id)
+            n.fork(p, next_id)
+            live.append(next_id)
+            next_id += 1
+        elif op == "append":
+            s = int(rng.choice(live))
+            try:
+                exp = m.append(s)
+            except AllocatorError:
+                with pytest.raises(PkvError):
+                    n.append(s)
+            else:
+                assert n.append(s) == exp
+        elif op == "batch":
+            ids = [int(x) for x in rng.choice(live, size=int(rng.integers(1, len(live) + 1)), replace=False)]
+            snap = (type(m.free)(m.free), list(m.ref), {k: list(v) for k, v in m.tables.items()}, dict(m.lens),
+                    dict(m.cache), dict(m.frame_key))
+            try:
+                exp = [m.append(s) for s in ids]
+            except AllocatorError:
+                m.free, m.ref, m.tables, m.lens, m.cache, m.frame_key = snap
+                with pytest.raises(PkvError):
+                    n.append_batch(ids)
+            else:
+                slots, pairs = n.append_batch(ids)
+                assert slots.tolist() == [e[0] for e in exp]
+                assert pairs.tolist() == [[e[1], e[2]] for e in exp if e[1] >= 0]
+        elif op == "beam":
+            k = int(rng.integers(1, len(live) + 1))
+            beams = [int(x) for x in rng.choice(live, size=k, replace=False)]
+            parents = [int(rng.integers(0, k)) for _ in range(int(rng.integers(0, k + 3)))]
+            try:
+                ids, slots, pairs, nid = m.beam_step(beams, parents, next_id)
+            except AllocatorError:
+                with pytest.raises(PkvError):
+                    n.beam_step(beams, parents, next_id)
+            else:
+                ids_n, slots_n, pairs_n, nid_n = n.beam_step(beams, parents, next_id)
+                assert ids_n.tolist() == ids and slots_n.tolist() == slots and pairs_n.tolist() == pairs
+                assert nid_n == nid
+                live = [s for s in live if s not in beams] + ids
+                next_id = nid
+        else:
+            s = int(rng.choice(live))
+            live.remove(s)
+            m.free_seq(s)
+            n.free_seq(s)
+        if step % 25 == 0:
+            same_state(n, m, live, 8 * N)
+    same_state(n, m, live, 8 * N)
+
+
+def test_prefix_cache_and_beam_edge_cases():
+    n, m = BlockAllocator(8, 4), AllocatorModel(8, 4)
+    # an empty prompt and a prompt shorter than a block: nothing is cached
+    for obj in (n, m):
+        assert obj.add_seq_cached(0, [])[1] == 0
+        assert obj.add_seq_cached(1, [7, 8, 9])[1] == 0
+    assert n.stats()["cached_blocks"] == m.stats()["cached_blocks"] == 0
+    # exactly one full block is cached and reused, the partial one is not
+    for obj in (n, m):
+        obj.add_seq_cached(2, [1, 2, 3, 4, 5])
+        assert obj.add_seq_cached(3, [1, 2, 3, 4, 6])[1] == 4
+    assert n.stats() == m.stats() and n.stats()["cached_blocks"] == 1
+    # a beam step with no candidates frees every beam
+    ids, slots, pairs, nid = n.beam_step([2, 3], [], 50)
+    e_ids, e_slots, e_pairs, e_nid = m.beam_step([2, 3], [], 50)
+    assert ids.tolist() == e_ids == [] and nid == e_nid == 50
+    assert n.stats() == m.stats()
+    # a fresh id that is already live is refused, nothing changes
+    before = n.stats()
+    with pytest.raises(PkvError) as e:
+        n.beam_step([0], [0, 0], 1)
+    assert e.value.status == PKV_EINVAL and n.stats() == before
