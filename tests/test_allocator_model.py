@@ -273,3 +273,19 @@ def test_prefix_cache_enomem_changes_nothing():
     with pytest.raises(AllocatorError):
         a.add_seq_cached(1, _prompt(rng, 8))  # needs 2 frames, 1 is free
     assert ({k: list(v) for k, v in a.tables.items()}, list(a.ref), list(a.free), dict(a.cache)) == snap
+
+
+def test_prefix_cache_block_after_a_different_prefix_is_not_reused():
+    """A block's KV depends on every earlier token (dataarena note section 3.1
+    hashes prompt blocks; the reading chains each key to its prefix).  With
+    A = [X, Y] and C = [Z, W] cached, B = [X, W] reuses X's frame but not W's:
+    W was cached after Z, not after X."""
+    rng = np.random.default_rng(5)
+    B = 4
+    X, Y, Z, W = (_prompt(rng, B) for _ in range(4))
+    a = AllocatorModel(32, B)
+    a.add_seq_cached(0, X + Y)
+    a.add_seq_cached(1, Z + W)
+    _, c = a.add_seq_cached(2, X + W)
+    assert c == B
+    assert a.tables[2][0] == a.tables[0][0] and a.tables[2][1] not in (a.tables[0][1], a.tables[1][1])
