@@ -7,7 +7,7 @@ importing the package does not load the library until a call needs it.
 
 _EXPORTS = (
     "paged_attention_decode", "contiguous_attention_decode", "reshape_and_cache", "copy_blocks",
-    "decode_workspace_bytes", "device_error", "BlockAllocator", "PkvError",
+    "decode_workspace_bytes", "device_error", "BlockAllocator", "PkvError", "block_hash",
 )
 
 __all__ = list(_EXPORTS)
