@@ -55,8 +55,10 @@ def lib():
         L.oracle_dense_decode.argtypes = [P, P, P, P, P, i32, i32, i32, dbl, i32, i32, i32, i32]
         L.oracle_reshape_and_cache.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32]
         L.oracle_copy_blocks.argtypes = [P, P, P, i32, i64, i32]
+        L.oracle_paged_prefill.argtypes = [P, P, P, P, P, i32, i32, i32, dbl, i32, i32, i32, i32, i32,
+                                           i32]
         for f in ("oracle_paged_decode", "oracle_attention_weights", "oracle_dense_decode",
-                  "oracle_reshape_and_cache", "oracle_copy_blocks"):
+                  "oracle_reshape_and_cache", "oracle_copy_blocks", "oracle_paged_prefill"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -102,6 +104,23 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_
                                    num_kv_heads, D, block_size, N, dtype)
     if rc != OR_OK:
         raise OracleError(rc, "paged_decode")
+    return out
+
+
+def paged_prefill(q, k_cache, v_cache, table_row, p0, scale, num_kv_heads, block_size, dtype) -> np.ndarray:
+    """Causal attention of T new tokens of one sequence at positions p0 .. p0 + T - 1
+    (their K/V already in the cache): query i sees positions 0 .. p0 + i through the
+    block-table row.  q: uint16 [T, Hq, D]; returns float64 [T, Hq, D]."""
+    q = _c(q, np.uint16)
+    kc, vc = _c(k_cache, np.uint16), _c(v_cache, np.uint16)
+    row = _c(table_row, np.int32)
+    T, Hq, D = q.shape
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    rc = lib().oracle_paged_prefill(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(row), row.shape[0],
+                                    int(p0), T, float(scale), Hq, num_kv_heads, D, block_size,
+                                    kc.shape[0], dtype)
+    if rc != OR_OK:
+        raise OracleError(rc, "paged_prefill")
     return out
 
 

@@ -1,6 +1,7 @@
 /*
  * Plain CPU oracle for paged decode attention, the paged cache write and the
- * copy-on-write block copy.
+ * copy-on-write block copy, and for paged prefill attention (the definition a
+ * prefill kernel would be checked against).
  *
  * TEST INFRASTRUCTURE.  Only the tests, the package smoke check and the CPU
  * baseline leg of the benchmark may load this library.  The CUDA library never
@@ -164,6 +165,49 @@ int oracle_paged_decode(double* out, const uint16_t* q, const uint16_t* k_cache,
  * Softmax weights w_t / Z of one (sequence, query head) over its context, in
  * logical token order (length context_lens[s]).
  */
+/*
+ * Paged prefill of one sequence: the prefill phase of the vLLM and
+ * PagedAttention slides (slide 3: the prompt is processed in parallel before
+ * decoding) over the paged cache of slides 9-10.  T new tokens sit at positions
+ * p0 .. p0 + T - 1 and their keys and values are already in the cache; query
+ * token i attends causally over positions 0 .. p0 + i (itself and everything
+ * before it), softmax(scale q K^T) V per query head as in the decode.
+ *   q          [T, Hq, D] fp16/bf16 bits     out [T, Hq, D] double
+ *   table_row  [max_blocks] int32, the sequence's block table row
+ * Returns OR_ERANGE if a table entry that the context p0 + T needs is outside
+ * [0, N), or if that context needs more than max_blocks entries.
+ */
+int oracle_paged_prefill(double* out, const uint16_t* q, const uint16_t* k_cache,
+                         const uint16_t* v_cache, const int32_t* table_row, int32_t max_blocks,
+                         int32_t p0, int32_t T, double scale, int32_t Hq, int32_t Hkv, int32_t D,
+                         int32_t B, int32_t N, int32_t dtype) {
+  if (check_heads(Hq, Hkv, D) || B <= 0 || max_blocks < 0 || p0 < 0 || T < 0) return OR_EINVAL;
+  const int64_t n = (int64_t)p0 + T;
+  if ((n + B - 1) / B > max_blocks) return OR_ERANGE;
+  if (T == 0) return OR_OK;
+  const int G = Hq / Hkv;
+  double* K = malloc((size_t)n * D * sizeof(double));
+  double* V = malloc((size_t)n * D * sizeof(double));
+  double* x = malloc((size_t)n * sizeof(double));
+  double* qd = malloc((size_t)D * sizeof(double));
+  int rc = (!K || !V || !x || !qd) ? OR_ENOMEM : OR_OK;
+  for (int g = 0; g < Hkv && rc == OR_OK; ++g) {
+    rc = gather_paged(K, V, k_cache, v_cache, table_row, n, g, Hkv, D, B, N, dtype);
+    for (int32_t i = 0; i < T && rc == OR_OK; ++i) {
+      for (int h = g * G; h < (g + 1) * G; ++h) {
+        const uint16_t* qrow = q + ((int64_t)i * Hq + h) * D;
+        for (int d = 0; d < D; ++d) qd[d] = to_double(qrow[d], dtype);
+        attend(out + ((int64_t)i * Hq + h) * D, NULL, x, qd, K, V, (int64_t)p0 + i + 1, D, scale);
+      }
+    }
+  }
+  free(K);
+  free(V);
+  free(x);
+  free(qd);
+  return rc;
+}
+
 int oracle_attention_weights(double* weights, const uint16_t* q, const uint16_t* k_cache,
                              const uint16_t* v_cache, const int32_t* tables, int32_t max_blocks,
                              const int32_t* context_lens, int32_t s, int32_t h, double scale,

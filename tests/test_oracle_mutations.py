@@ -1,4 +1,4 @@
-"""The oracle's pins catch plausible mistakes.
+"""The oracle's pins (decode and prefill) catch plausible mistakes.
 
 Each case plants one mistake in a copy of oracle.c (a dropped term, a wrong
 sign, a wrong index, a transposed operand ...), builds it into a temporary
@@ -28,6 +28,12 @@ MUTATIONS = {
                           "v = ldexp((double)(f | 0x400), e - 24);"),
     "scatter_offset": ("int64_t frame = slot / B, off = slot % B;",
                        "int64_t frame = slot / B, off = (B - 1) - slot % B;"),
+    "prefill_not_causal": ("attend(out + ((int64_t)i * Hq + h) * D, NULL, x, qd, K, V, (int64_t)p0 + i + 1, D, scale);",
+                           "attend(out + ((int64_t)i * Hq + h) * D, NULL, x, qd, K, V, n, D, scale);"),
+    "prefill_excludes_self": ("attend(out + ((int64_t)i * Hq + h) * D, NULL, x, qd, K, V, (int64_t)p0 + i + 1, D, scale);",
+                              "attend(out + ((int64_t)i * Hq + h) * D, NULL, x, qd, K, V, (int64_t)p0 + i, D, scale);"),
+    "prefill_head_group_interleaved": ("for (int32_t i = 0; i < T && rc == OR_OK; ++i) {\n      for (int h = g * G; h < (g + 1) * G; ++h) {",
+                                       "for (int32_t i = 0; i < T && rc == OR_OK; ++i) {\n      for (int h = g; h < Hq; h += Hkv) {"),
 }
 
 
@@ -43,7 +49,8 @@ def test_pins_fail_on_planted_mistake(name, tmp_path):
                            str(mutated), "-lm"])
     env = dict(os.environ, PKV_ORACLE_LIB=str(so))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_prefill.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch mutation {name}:\n{r.stdout[-2000:]}"
     assert "failed" in r.stdout or "error" in r.stdout.lower()
