@@ -24,10 +24,18 @@
  *    {8, 16, 32}, num_heads / num_kv_heads in {1, 2, 4, 8}.  Anything else
  *    returns PKV_EUNSUPPORTED.
  *
- * Environment: PKV_VALIDATE=1 makes the decode and cache-write calls copy the
- * block tables / context lengths / slots back to the host, check every index
- * the kernels would use, and return PKV_ERANGE instead of launching when one is
- * out of range (this synchronises the stream).
+ * Environment: PKV_VALIDATE=1 makes the decode, cache-write and block-copy calls
+ * copy the block tables / context lengths / slots / copy pairs back to the host,
+ * check every index the kernels would use, and return PKV_ERANGE (PKV_EINVAL
+ * for a copy list whose pairs depend on their order) instead of launching
+ * (this synchronises the stream).
+ *
+ * CUDA graphs: the first call on a device sets up per-device state (the device
+ * address of the error flags, the SM count) and the first decode call of each
+ * kernel variant (dtype, head_dim, query heads per kv head, block size) on a
+ * device sets that kernel's shared-memory limit and queries its occupancy.
+ * Make one warm-up call per device and variant before capturing calls into a
+ * CUDA graph; captured calls then run no set-up.
  */
 #ifndef PKV_H_
 #define PKV_H_
@@ -57,7 +65,9 @@ typedef enum { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
 #define PKV_DEVERR_CONTEXT_LEN 2u  /* a context length < 0 or above the table's capacity: clamped */
 #define PKV_DEVERR_SLOT 4u         /* a slot >= num_blocks * block_size: row not written */
 #define PKV_DEVERR_COPY_PAIR 8u    /* a copy pair naming a frame outside [0, num_blocks): skipped */
-#define PKV_DEVERR_WAIT_TIMEOUT 16u /* a bounded shared-memory barrier wait expired: output invalid */
+#define PKV_DEVERR_WAIT_TIMEOUT 16u /* a bounded wait (a shared-memory barrier, or the partition
+                                        merge waiting for a context's partitions) expired:
+                                        output invalid */
 
 /* Human-readable name of a status code (static storage). */
 const char* pkv_status_string(pkv_status status);
@@ -66,6 +76,20 @@ const char* pkv_status_string(pkv_status status);
  * work queued on `stream` has finished (synchronises `stream`); clears them
  * when `clear` != 0. */
 pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t stream);
+
+/*
+ * Test hook for the bounded waits (no counterpart on the pages).  Kernels never
+ * spin forever: a wait that gives up sets PKV_DEVERR_WAIT_TIMEOUT and the
+ * kernel returns.  This call lets a test make the one wait that has no copies
+ * in flight run out on purpose: the partition merge's wait for the decode grid
+ * to publish a (sequence, kv head) pair.  Every later decode call in the
+ * process makes that wait expect `extra` more publications than the decode grid
+ * makes and give up after `limit_ns` nanoseconds (0 = the normal 1 s bound).
+ * The pairs that time out keep whatever their output rows held.  Call
+ * pkv_test_set_merge_wait(0, 0) to restore normal operation.  Not for
+ * production use; not synchronised with calls in flight on other threads.
+ */
+pkv_status pkv_test_set_merge_wait(uint64_t limit_ns, uint32_t extra);
 
 /* ------------------------------------------------------------------------ */
 /* Decode attention                                                         */
@@ -104,7 +128,9 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t h
  *   k_cache      device [num_blocks, num_kv_heads, block_size, head_dim] dtype
  *   v_cache      device, same shape as k_cache
  *   block_tables device int32 [num_seqs, max_blocks_per_seq]; only the first
- *                ceil(context_lens[s] / block_size) entries of row s are read
+ *                ceil(context_lens[s] / block_size) entries of row s are used (the
+ *                kernel may read further entries of the row, up to one partition's
+ *                worth, without using them, so the whole row must be readable)
  *   context_lens device int32 [num_seqs], 0 <= context_lens[s] <= max_blocks_per_seq * block_size
  *   partition_size maximum tokens per context partition (0 = 1024); a multiple of 64
  *                in [64, 2048].  A context of L tokens is split into ceil(L / partition_size)
@@ -117,11 +143,13 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t h
  *
  * Launches, in this order on `stream`: a one-CTA planning kernel (work list),
  * the persistent decode kernel and, when a context can span more than one
- * partition, the partition merge kernel (both with programmatic dependent
- * launch).  The merge kernel starts while the decode grid drains and merges
- * each (sequence, kv head) as soon as the decode grid has published all of its
- * partitions; it completes after the decode grid, so work that follows on the
- * stream sees the whole of `out`.
+ * partition, the partition merge kernel, all with programmatic dependent
+ * launch.  The planning kernel may become resident while the work queued before
+ * it finishes (when that work lets dependents launch early) and waits for it to
+ * complete before anything else runs.  The merge kernel starts while the decode
+ * grid drains and merges each (sequence, kv head) as soon as the decode grid
+ * has published all of its partitions; it completes after the decode grid, so
+ * work that follows on the stream sees the whole of `out`.
  */
 pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
                                       const void* v_cache, const int32_t* block_tables,
@@ -200,6 +228,10 @@ pkv_status pkv_contiguous_attention_decode(void* out, const void* q, const void*
  *                not written and sets PKV_DEVERR_SLOT.
  *   head_dim * element size must be 16 bytes times a power of two (head_dim 8,
  *   16, 32, 64, 128, 256 for 16-bit types); other head_dim: PKV_EUNSUPPORTED.
+ * The kernel lets a kernel queued behind it with programmatic dependent launch
+ * become resident at once; such a kernel must wait for this grid in-kernel
+ * before it reads the caches (the decode call's planning kernel does).  The
+ * block copy below does the same.
  */
 pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
                                  const int64_t* slot_mapping, int32_t num_tokens,
@@ -214,7 +246,9 @@ pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cac
  *   src_dst_pairs device int64 [num_pairs, 2] = (src, dst) frame indices.  All
  *                pairs run concurrently: destinations must be distinct and no
  *                destination may be the source of another pair (the allocator's
- *                copy lists satisfy this).  src == dst is a no-op.  A frame index
+ *                copy lists satisfy this); otherwise the result depends on the
+ *                order the pairs happen to run in (PKV_VALIDATE=1 rejects such a
+ *                list with PKV_EINVAL).  src == dst is a no-op.  A frame index
  *                outside [0, num_blocks) skips the pair and sets PKV_DEVERR_COPY_PAIR.
  *   block_bytes  bytes of one frame of one cache = num_kv_heads * block_size *
  *                head_dim * element size; a multiple of 16.

@@ -48,6 +48,12 @@ def lib():
         L.oracle_f16_to_double.restype = dbl
         L.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
         L.oracle_bf16_to_double.restype = dbl
+        L.oracle_double_to_f16.argtypes = [dbl]
+        L.oracle_double_to_f16.restype = ctypes.c_uint16
+        L.oracle_double_to_bf16.argtypes = [dbl]
+        L.oracle_double_to_bf16.restype = ctypes.c_uint16
+        L.oracle_round_array.argtypes = [P, P, i64, i32]
+        L.oracle_round_array.restype = ctypes.c_int
         L.oracle_paged_decode.argtypes = [P, P, P, P, P, i32, P, i32, i32, dbl, i32, i32, i32, i32,
                                           i32, i32]
         L.oracle_attention_weights.argtypes = [P, P, P, P, P, i32, P, i32, i32, dbl, i32, i32, i32,
@@ -83,6 +89,17 @@ def to_double(bits: np.ndarray, dtype: int) -> np.ndarray:
     f = lib().oracle_f16_to_double if dtype == 0 else lib().oracle_bf16_to_double
     flat = np.asarray(bits, dtype=np.uint16).ravel()
     return np.array([f(int(b)) for b in flat], dtype=np.float64).reshape(np.shape(bits))
+
+
+def round_to_dtype(x, dtype: int) -> np.ndarray:
+    """float64 values -> fp16 (dtype 0) / bf16 (dtype 1) bit patterns, each rounded
+    to nearest with ties to even, straight from fp64 (one rounding)."""
+    src = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(src.shape, dtype=np.uint16)
+    rc = lib().oracle_round_array(_ptr(out), _ptr(src), src.size, int(dtype))
+    if rc != OR_OK:
+        raise OracleError(rc, "round_to_dtype")
+    return out
 
 
 def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, num_kv_heads, block_size,

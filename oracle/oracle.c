@@ -70,6 +70,71 @@ static double to_double(uint16_t bits, int dtype) {
 }
 
 /*
+ * Round a double to the nearest value of a binary format with `sig` significand
+ * bits (implicit bit included), exponent bias `bias` and all-ones exponent field
+ * `emax_field` (infinity / NaN), ties to the value whose last significand bit is
+ * 0 (IEEE 754 roundTiesToEven), and return its bit pattern.  This is the
+ * rounding the outputs are stored with ("RNE to the output dtype").
+ *   x = f * 2^(e - sig + 1) with f an integer in [2^(sig-1), 2^sig) when normal;
+ *   below the smallest normal exponent 1 - bias the quantum is fixed at
+ *   2^(1 - bias - sig + 1) (subnormals).  Scaling by a power of two is exact in
+ *   fp64 here, so the only rounding is the explicit integer rounding.
+ */
+static uint16_t round_to_format(double v, int sig, int bias, int emax_field) {
+  const int frac_bits = sig - 1;
+  const uint16_t sign = signbit(v) ? 0x8000u : 0u; /* bit 15 in both 16-bit formats */
+  const uint16_t inf_bits = (uint16_t)(emax_field << frac_bits);
+  if (isnan(v)) return (uint16_t)(inf_bits | (1u << (frac_bits - 1))); /* quiet NaN */
+  double x = fabs(v);
+  if (isinf(x)) return sign | inf_bits;
+  if (x == 0.0) return sign;
+  int E;
+  frexp(x, &E);              /* x = m 2^E, m in [0.5, 1): leading bit at 2^(E-1) */
+  int e = E - 1;             /* unbiased exponent of the leading bit */
+  const int emin = 1 - bias; /* smallest normal exponent */
+  const int qexp = (e >= emin ? e : emin) - frac_bits;  /* exponent of one quantum */
+  const double q = ldexp(x, -qexp);                     /* exact */
+  double f = floor(q);
+  const double r = q - f;                               /* exact: q < 2^sig */
+  if (r > 0.5 || (r == 0.5 && fmod(f, 2.0) != 0.0)) f += 1.0;
+  /* re-normalise: f may have reached 2^sig (carry into the exponent) */
+  int field;
+  long mant;
+  if (e < emin) {            /* subnormal range: field 0, f counts quanta (f = 2^frac_bits: smallest normal) */
+    if (f >= ldexp(1.0, frac_bits)) {
+      field = 1;
+      mant = (long)(f - ldexp(1.0, frac_bits));
+    } else {
+      field = 0;
+      mant = (long)f;
+    }
+  } else {
+    if (f >= ldexp(1.0, sig)) {
+      f = ldexp(1.0, frac_bits);
+      e += 1;
+    }
+    field = e + bias;
+    mant = (long)(f - ldexp(1.0, frac_bits));
+  }
+  if (field >= emax_field) return sign | inf_bits;  /* overflow rounds to infinity */
+  return sign | (uint16_t)((field << frac_bits) | mant);
+}
+
+/* IEEE binary16: 11 significand bits, bias 15. */
+uint16_t oracle_double_to_f16(double v) { return round_to_format(v, 11, 15, 31); }
+
+/* bfloat16: 8 significand bits, bias 127 (the upper half of a binary32). */
+uint16_t oracle_double_to_bf16(double v) { return round_to_format(v, 8, 127, 255); }
+
+/* Element-wise rounding of n doubles to fp16 (dtype 0) or bf16 (dtype 1) bits. */
+int oracle_round_array(uint16_t* out, const double* in, int64_t n, int32_t dtype) {
+  if (n < 0 || (dtype != OR_F16 && dtype != OR_BF16)) return OR_EINVAL;
+  for (int64_t i = 0; i < n; ++i)
+    out[i] = dtype == OR_F16 ? oracle_double_to_f16(in[i]) : oracle_double_to_bf16(in[i]);
+  return OR_OK;
+}
+
+/*
  * softmax(scale * K q) V over n rows given in logical order.
  *   x_t = scale * sum_d q_d K_{t,d}          (summed in order of d)
  *   m   = max_t x_t,  w_t = exp(x_t - m),  Z = sum_t w_t

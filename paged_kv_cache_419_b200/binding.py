@@ -29,7 +29,7 @@ EXPORTS = (
     "pkv_copy_blocks", "pkv_alloc_create", "pkv_alloc_destroy", "pkv_alloc_add_seq",
     "pkv_alloc_fork", "pkv_alloc_append", "pkv_alloc_append_batch", "pkv_alloc_free_seq",
     "pkv_alloc_beam_step", "pkv_alloc_block_table", "pkv_alloc_refcount", "pkv_alloc_stats",
-    "pkv_alloc_add_seq_cached", "pkv_block_hash",
+    "pkv_alloc_add_seq_cached", "pkv_block_hash", "pkv_test_set_merge_wait",
 )
 
 
@@ -101,6 +101,7 @@ def lib() -> ctypes.CDLL:
             "pkv_alloc_block_table": ([P, P, i32, i32, P, P], ctypes.c_int),
             "pkv_alloc_refcount": ([P, i32, P], ctypes.c_int),
             "pkv_alloc_stats": ([P, ctypes.POINTER(AllocStats)], ctypes.c_int),
+            "pkv_test_set_merge_wait": ([ctypes.c_uint64, ctypes.c_uint32], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -233,6 +234,13 @@ def device_error(clear: bool = True, stream=None) -> int:
     _check(lib().pkv_device_error(ctypes.byref(flags), int(clear), _stream(stream)),
            "pkv_device_error")
     return flags.value
+
+
+def set_merge_wait_hook(limit_ns: int = 0, extra: int = 0):
+    """Bounded-wait test hook (pkv_test_set_merge_wait): later decode calls make
+    the partition merge wait for ``extra`` more publications than the decode grid
+    makes and give up after ``limit_ns`` (0, 0 restores normal operation)."""
+    _check(lib().pkv_test_set_merge_wait(int(limit_ns), int(extra)), "pkv_test_set_merge_wait")
 
 
 # ---------------------------------------------------------------- allocator

@@ -2,6 +2,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -25,12 +26,19 @@ struct DeviceInfo {
   int num_sms = 0;
 };
 DeviceInfo g_devices[kMaxDevices];
+std::mutex g_devices_mutex;
+
+// Bounded-wait test hook (pkv_test_set_merge_wait): 0 = the normal bound.
+std::atomic<unsigned long long> g_merge_wait_limit_ns{0};
+std::atomic<uint32_t> g_merge_wait_extra{0};
 
 // Per-device set-up with that device current: the device address of the error
-// flag and the SM count.
+// flag and the SM count (under a lock: host threads may make their first call
+// on a device at the same time).
 pkv_status device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ECUDA;
+  std::lock_guard<std::mutex> lock(g_devices_mutex);
   DeviceInfo& d = g_devices[dev];
   if (!d.ready) {
     void* p = nullptr;
@@ -176,6 +184,9 @@ pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pk
     a.tmp_out = a.tmp_m = a.tmp_l = nullptr;
   }
   a.scale_log2 = scale * 1.4426950408889634f;
+  const unsigned long long hook_ns = g_merge_wait_limit_ns.load(std::memory_order_relaxed);
+  a.merge_wait_limit_ns = hook_ns ? hook_ns : kWaitLimitNs;
+  a.merge_wait_extra = g_merge_wait_extra.load(std::memory_order_relaxed);
   DeviceInfo* dev = nullptr;
   pkv_status st = device_info(&dev);
   if (st != PKV_OK) return st;
@@ -226,6 +237,29 @@ pkv_status validate_decode_tables(const int32_t* tables, const int32_t* lens, in
   return PKV_OK;
 }
 
+// PKV_VALIDATE=1 check of a copy list (host copy): every frame in range, and the
+// pairs independent of their order (all run concurrently): distinct
+// destinations, and no destination that is also the source of another pair.
+pkv_status validate_copy_pairs(const int64_t* pairs, int32_t n, int32_t num_blocks) {
+  std::vector<uint8_t> role(static_cast<size_t>(num_blocks), 0);  // bit 0: source, bit 1: destination
+  for (int32_t i = 0; i < n; ++i) {
+    const int64_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) return PKV_ERANGE;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    const int64_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+    if (src == dst) continue;  // no-op pair
+    role[static_cast<size_t>(src)] |= 1u;
+    if (role[static_cast<size_t>(dst)] & 2u) return PKV_EINVAL;  // two pairs write one frame
+    role[static_cast<size_t>(dst)] |= 2u;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    const int64_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+    if (src != dst && (role[static_cast<size_t>(dst)] & 1u)) return PKV_EINVAL;  // read and written
+  }
+  return PKV_OK;
+}
+
 }  // namespace
 }  // namespace pkv
 
@@ -256,6 +290,12 @@ pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t str
   if (clear && cudaMemsetAsync(dev->err, 0, sizeof h, stream) != cudaSuccess) return PKV_ECUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return PKV_ECUDA;
   *flags_out = h;
+  return PKV_OK;
+}
+
+pkv_status pkv_test_set_merge_wait(uint64_t limit_ns, uint32_t extra) {
+  g_merge_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+  g_merge_wait_extra.store(extra, std::memory_order_relaxed);
   return PKV_OK;
 }
 
@@ -384,6 +424,15 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_
   if (num_pairs == 0) return PKV_OK;
   if (!k_cache || !v_cache || !src_dst_pairs) return PKV_EINVAL;
   if (!aligned16(k_cache) || !aligned16(v_cache)) return PKV_EINVAL;
+  if (validate_env()) {
+    std::vector<int64_t> h(2 * static_cast<size_t>(num_pairs));
+    if (cudaMemcpyAsync(h.data(), src_dst_pairs, sizeof(int64_t) * h.size(), cudaMemcpyDeviceToHost,
+                        stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return PKV_ECUDA;
+    const pkv_status vs = validate_copy_pairs(h.data(), num_pairs, num_blocks);
+    if (vs != PKV_OK) return vs;
+  }
   DeviceInfo* dev = nullptr;
   pkv_status st = device_info(&dev);
   if (st != PKV_OK) return st;

@@ -26,6 +26,10 @@ __global__ void __launch_bounds__(kReshapeThreads) reshape_and_cache_kernel(
     uint4* __restrict__ v_cache, const int64_t* __restrict__ slots, int64_t num_tokens,
     int32_t num_kv_heads, int32_t vpr_shift, int32_t block_size, int64_t num_slots,
     unsigned int* err) {
+  // A kernel queued behind this one with programmatic dependent launch (the
+  // decode call's planning kernel) may become resident now; it waits for this
+  // grid to complete before it goes on.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int32_t per_token = num_kv_heads << vpr_shift;
   const int32_t col_mask = (1 << vpr_shift) - 1;
   const int64_t stride = 2 * static_cast<int64_t>(gridDim.x);
@@ -78,6 +82,7 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(uint4* __rest
                                                                    int64_t vec_per_block,
                                                                    int32_t num_blocks,
                                                                    unsigned int* err) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // as in the cache write
   for (int64_t item = blockIdx.x; item < 2 * static_cast<int64_t>(num_pairs); item += gridDim.x) {
     const int64_t pair = item >> 1;
     const int64_t src = __ldg(pairs + 2 * pair);

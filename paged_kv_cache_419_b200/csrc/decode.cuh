@@ -13,7 +13,8 @@
 //    is cut into n = ceil(L / part_tokens) near-equal partitions whose sizes are
 //    multiples of 64 tokens.  All G = Hq/Hkv query heads of the kv head share one
 //    K/V fetch.
-//  * plan_kernel (one CTA, plain stream order) lists the items, largest first,
+//  * plan_kernel (one CTA; it may become resident while the work before it on
+//    the stream finishes, and waits for that work in-kernel) lists the items, largest first,
 //    lists the contexts that span several partitions and zeroes their
 //    completion counters.  Partition 0 of the first grid/Hkv sequences is not
 //    listed: decode CTA c starts with it (sequence c / Hkv, kv head c % Hkv),
@@ -31,14 +32,16 @@
 //  * Consumer warp w owns tokens 16w..16w+15 of each stage with its own
 //    online-softmax state.  Scores: S^T = Q K^T as mma.sync m16n8k16 tiles (fp32
 //    accumulation), K fragments read with ldmatrix from the swizzled stage.  PV:
-//    O^T += V^T P^T, P^T taken from the score accumulators as they lie (rounded
-//    to the input type), V^T read with transposing ldmatrix.
+//    O^T += V^T P^T, P^T taken from the score accumulators as they lie (as two
+//    16-bit parts, hi + lo, so that the weights keep about 16 significant bits),
+//    V^T read with transposing ldmatrix.
 //  * Epilogue per item: the four warps merge through shared memory in a fixed
 //    order (bit-reproducible).  A one-partition context writes `out`; otherwise
 //    the partition's normalised output, max and sum go to the workspace.  Each
-//    CTA publishes its multi-partition items to per-(sequence, kv head)
-//    counters, and merge_kernel, which runs in the decode grid's tail, merges
-//    each such context (log-sum-exp) into `out` as soon as its count is complete.
+//    multi-partition item is published as soon as it is written (a release
+//    increment of its (sequence, kv head) counter), and merge_kernel, which runs
+//    in the decode grid's tail, merges each such context (log-sum-exp) into
+//    `out` as soon as its count is complete.
 //  * Scores are kept in base-2 units (scale * log2 e folded into one multiply),
 //    so the exponentials are single ex2 instructions.
 #pragma once
@@ -78,6 +81,11 @@ struct DecodeArgs {
   float* tmp_m;           // [S, Hq, max_parts]
   float* tmp_l;           // [S, Hq, max_parts]
   unsigned int* err;
+  // Bound of the merge grid's wait for a pair's partitions, and extra
+  // publications it waits for beyond the partition count (0 except under the
+  // bounded-wait test hook, which makes the wait run out on purpose).
+  unsigned long long merge_wait_limit_ns;
+  uint32_t merge_wait_extra;
 };
 
 constexpr int kConsumerWarps = 4;
@@ -87,9 +95,9 @@ constexpr int kPlanThreads = 1024;
 constexpr int kItemSlots = 2;
 constexpr int kRecSlots = 2;   // records of items k and k+1
 constexpr int kStageTokens = 64;
-// Multi-partition items a CTA finishes before it publishes them (one fence for
-// the lot) to the merge grid; a full list is published at the next item.
-constexpr int kPubSlots = 32;
+// Multi-partition items a CTA has finished and not yet published to the merge
+// grid: at most one (it is published at the start of the next item, or at exit).
+constexpr int kPubSlots = 2;
 // Work record of one (sequence, partition): int32 s, part, n_parts, t_begin,
 // n_tok, L, 0, 0.
 constexpr int kRecordBytes = 32;
@@ -206,9 +214,12 @@ constexpr int kPlanDirect = 8;   // partitions a thread writes itself
 constexpr int kPlanWide = 512;   // sequences listed for warp-wide record writing
 
 static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeArgs a) {
-  // This grid is launched in plain stream order, so its predecessor has
-  // completed.  The decode grid may start now: its static first items read only
-  // inputs, and it waits for this grid before it touches anything written here.
+  // This grid may be launched while its predecessor on the stream still runs
+  // (programmatic dependent launch): wait here until the predecessor has
+  // completed and its writes are visible.  Then the decode grid may start: its
+  // static first items read only inputs, and it waits for this grid before it
+  // touches anything written here.
+  grid_dependency_wait();
   allow_dependent_launch();
   const int n_static = static_first_seqs(a.num_seqs, a.grid_ctas, a.num_kv_heads);
   constexpr int kMaxClasses = kMaxPartTokens / 32 + 2;
@@ -463,9 +474,20 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
         blockIdx.x < static_cast<uint32_t>(static_first_seqs(a.num_seqs, a.grid_ctas, a.num_kv_heads)) * Hkv;
     uint32_t cur = 0;  // list index of the current item (items after a static first one)
     if (static_first) {
+      const int s = static_cast<int>(blockIdx.x / Hkv);
+      if constexpr (PAGED) {
+        // The table entries are requested together with the context length, one
+        // memory round trip for both: every entry partition 0 can use (at most
+        // part_tokens / B, and never past the row), whatever the length turns
+        // out to be.  Entries past the context are fetched but never used.
+        const int cap = min(a.part_tokens / B, a.max_blocks);
+        const int32_t* row = a.tables + static_cast<int64_t>(s) * a.max_blocks;
+        for (int e = lane; e < cap; e += 32) cp_async_4(s_tab + e, row + e);
+        cp_async_arrive_noinc(&tab_bar[0]);
+        tab_pending |= 1u;  // buffer 0, phase 0
+      }
       if (lane == 0) {  // record of partition 0 of sequence blockIdx.x / Hkv, in slot 0
         int32_t* r = reinterpret_cast<int32_t*>(smem + Tr::OFF_REC);
-        const int s = static_cast<int>(blockIdx.x / Hkv);
         const int L = clamp_len(a.lens[s], a.max_ctx);
         int n, size;
         partition_of(L, a.part_tokens, n, size);
@@ -480,7 +502,6 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
         mbar_arrive(&rec_bar[0]);
       }
       __syncwarp();
-      fetch_table(0);
     } else {
       plan_wait();
       if (lane == 0) cur = atomicAdd(a.work, 1u);
@@ -646,7 +667,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
   //           n-tiles, K read with ldmatrix straight from the swizzled stage;
   //   output  O^T (D x 8) += V^T (D x 16) P^T (16 x 8): V read with transposing
   //           ldmatrix, P^T taken from the score accumulators as they lie
-  //           (their C layout is the B layout of the next product).
+  //           (their C layout is the B layout of the next product), as a hi
+  //           and a lo 16-bit part, one product each.
   // Exits are decided together (barrier-OR over the consumer warps) so that no
   // warp is ever left waiting at a named barrier.
   const int quad = lane >> 2;  // score tile: head row; output tile: dim row
@@ -664,18 +686,17 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
   const uint32_t v_lane =
       static_cast<uint32_t>((w_tok0 + 8 * (mat >> 1) + mrow) * 128 + (((mat & 1) ^ mrow) << 4));
   uint32_t st = 0, ph = 0;  // ring slot and use parity of the next stage
-  // Publication (thread 0): partial results of multi-partition items are
-  // announced to the merge grid by one gpu-scope fence followed by one counter
-  // increment per item.  The fence is cumulative over the other consumer
-  // threads' writes, which a named barrier ordered before it; batching makes it
-  // one fence per kPubSlots items instead of one per item.
+  // Publication (thread 0): the partial result of a multi-partition item is
+  // announced to the merge grid by one gpu-scope release increment of its
+  // (sequence, kv head) counter, right after the named barrier at the start of
+  // the next item (or at exit), which orders every consumer thread's write-out
+  // of the item before it.  Publishing each item as soon as it is written lets
+  // the merge of a context start as soon as its last partition is done.
   // s_pub[kPubSlots] holds the count (thread 0 alone touches the list).
   if (threadIdx.x == 0) s_pub[kPubSlots] = 0u;
   auto publish = [&]() {
     const uint32_t n = s_pub[kPubSlots];
-    if (n == 0) return;
-    __threadfence();
-    for (uint32_t i = 0; i < n; ++i) atomicAdd(&a.pair_done[s_pub[i]], 1u);
+    for (uint32_t i = 0; i < n; ++i) red_add_release_gpu(&a.pair_done[s_pub[i]], 1u);
     s_pub[kPubSlots] = 0u;
   };
 
@@ -686,7 +707,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
     const ItemInfo info = items[slot];
     // Every consumer thread has finished the previous item's write-out here.
     if (named_barrier_or(1, NW * 32, !arrived || info.s < 0)) break;
-    if (threadIdx.x == 0 && s_pub[kPubSlots] == kPubSlots) publish();
+    if (threadIdx.x == 0) publish();
     const int h0 = info.kvh * G;
 
     // Q as the A operand: lane holds head `quad`, dims 16 ks + 2 qc (+1) and the
@@ -777,9 +798,16 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
             p[nt][e] = x[nt][e] == -CUDART_INF_F ? 0.f : fast_exp2(x[nt][e] - m_run);
           l_lane += p[nt][e];
         }
-      // P^T as the B operand: k = token, n = head (rounded to the input type)
+      // P^T as the B operand (k = token, n = head), split into two 16-bit parts:
+      // hi = p rounded to the input type, lo = the rest (p - hi, exact in fp32)
+      // rounded again.  Two products with the same V fragments then carry p to
+      // about 16 significant bits, so the weights that multiply V agree with the
+      // fp32 weights the normaliser sums.
       const uint32_t pb0 = pack2<T>(p[0][0], p[0][1]);
       const uint32_t pb1 = pack2<T>(p[1][0], p[1][1]);
+      const float2 h0 = unpack2<T>(pb0), h1 = unpack2<T>(pb1);
+      const uint32_t pl0 = pack2<T>(p[0][0] - h0.x, p[0][1] - h0.y);
+      const uint32_t pl1 = pack2<T>(p[1][0] - h1.x, p[1][1] - h1.y);
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_v[st], ph))) return false;
       if constexpr (!FULL) {
         // V rows past the end of the context hold whatever the pool or an
@@ -799,6 +827,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
         uint32_t va[4];
         ldmatrix_x4_trans(va, sV + (mt >> 2) * Tr::PANEL_BYTES + (v_lane ^ ((mt & 3) << 5)));
         mma_16816<T>(acc[mt], va, pb0, pb1);
+        mma_16816<T>(acc[mt], va, pl0, pl1);
       }
       // the zeroing stores must be ordered before the next bulk copy into this half
       if constexpr (!FULL) fence_proxy_async_smem();
@@ -967,11 +996,15 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
     // possibly stale L1 line.
     if (tid == 0) {
       s_ready = wait_counter_bounded(a.pair_done + static_cast<int64_t>(s) * Hkv + kvh,
-                                     static_cast<uint32_t>(np), a.err);
+                                     static_cast<uint32_t>(np) + a.merge_wait_extra, a.err,
+                                     a.merge_wait_limit_ns);
       if (!s_ready) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
     }
     __syncthreads();
-    if (!s_ready) continue;  // uniform: results of this pair stay unwritten
+    if (!s_ready) {  // uniform: results of this pair stay unwritten
+      __syncthreads();  // every thread has read s_ready before thread 0 rewrites it
+      continue;
+    }
 
     // ---- M and L per head (warp g reduces head g; online across chunks)
     float M = -CUDART_INF_F, L = 0.f;  // valid in warp g < G

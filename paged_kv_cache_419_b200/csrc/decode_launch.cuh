@@ -1,21 +1,26 @@
 // Host launchers for the decode kernels; included by one file per (dtype, head_dim).
 #pragma once
 
+#include <atomic>
+
 #include "decode.cuh"
 
 namespace pkv {
 
 // Persistent grid size of one decode instantiation on the current device:
 // SM count x resident CTAs per SM (set up once per device).
+// Two host threads making their first call at once may both run the set-up; it
+// is idempotent and the atomic store publishes the same value.
 template <typename T, int D, int G, int B, bool PAGED>
 cudaError_t decode_grid(int num_sms, int* grid) {
   using Tr = DecodeTraits<T, D, G, B, PAGED>;
-  static int blocks_per_sm[64] = {};
+  static std::atomic<int> blocks_per_sm[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (blocks_per_sm[dev] == 0) {
+  int per_sm = blocks_per_sm[dev].load(std::memory_order_acquire);
+  if (per_sm == 0) {
     auto kern = decode_kernel<T, D, G, B, PAGED>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -24,9 +29,10 @@ cudaError_t decode_grid(int num_sms, int* grid) {
     int n = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecodeThreads, Tr::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    blocks_per_sm[dev] = n > 0 ? n : 1;
+    per_sm = n > 0 ? n : 1;
+    blocks_per_sm[dev].store(per_sm, std::memory_order_release);
   }
-  *grid = num_sms * blocks_per_sm[dev];
+  *grid = num_sms * per_sm;
   return cudaSuccess;
 }
 
@@ -39,24 +45,24 @@ cudaError_t launch_decode_one(const DecodeArgs& args, const DecodeMaps& maps, in
   if (e != cudaSuccess) return e;
   DecodeArgs a = args;
   a.grid_ctas = grid;
-  // The plan grid is launched in plain stream order: it starts once everything
-  // before it on the stream has completed, so the kernels behind it may read
-  // their inputs as soon as they start.  Decode and merge use programmatic
-  // dependent launch: each may start while its predecessor runs and waits for
-  // it in-kernel before touching anything the predecessor writes.
+  // All three grids use programmatic dependent launch: each may become resident
+  // while its predecessor runs.  The plan waits in-kernel for its predecessor
+  // (whatever the caller queued before the call) to complete before it lets the
+  // decode grid launch, so the kernels behind it may read their inputs as soon
+  // as they start; decode and merge wait in-kernel for their predecessors before
+  // touching anything those write.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 0;
+  cfg.numAttrs = 1;
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(kPlanThreads);
   cfg.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&cfg, plan_kernel, a);
   if (e != cudaSuccess) return e;
-  cfg.numAttrs = 1;
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kDecodeThreads);
   cfg.dynamicSmemBytes = Tr::SMEM_BYTES;

@@ -95,17 +95,25 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
+// *p += v at gpu scope with release semantics: this thread's earlier writes, and
+// those of the threads a CTA barrier ordered before it, become visible to any
+// thread that reads the new value with acquire semantics.
+__device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Wait until *counter >= target (each read a gpu-scope acquire).  False after
-// kWaitLimitNs, or at once when another wait has already timed out
+// limit_ns, or at once when another wait has already timed out
 // (PKV_DEVERR_WAIT_TIMEOUT set in *err): the work it was waiting for will not come.
 __device__ __forceinline__ bool wait_counter_bounded(const uint32_t* counter, uint32_t target,
-                                                     const unsigned int* err) {
+                                                     const unsigned int* err,
+                                                     unsigned long long limit_ns) {
   if (ld_acquire_gpu(counter) >= target) return true;
   const unsigned long long t0 = global_timer_ns();
   for (;;) {
     __nanosleep(200);
     if (ld_acquire_gpu(counter) >= target) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
     if (err && (*reinterpret_cast<const volatile unsigned int*>(err) & PKV_DEVERR_WAIT_TIMEOUT))
       return false;
   }

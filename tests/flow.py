@@ -143,3 +143,24 @@ def max_abs_err(gpu_out: torch.Tensor, ref: np.ndarray, rows=None) -> float:
     if rows is not None:
         g, ref = g[rows], ref[rows]
     return float(np.abs(g - ref).max()) if g.size else 0.0
+
+
+def ulp_distance(out_bits: np.ndarray, ref_bits: np.ndarray) -> np.ndarray:
+    """Number of representable 16-bit values between two fp16 / bf16 bit patterns
+    (sign-magnitude mapped onto one ordered integer line; +0 and -0 coincide)."""
+    def line(b):
+        b = b.astype(np.int64)
+        mag = b & 0x7FFF
+        return np.where(b & 0x8000, -mag, mag)
+    return np.abs(line(out_bits) - line(ref_bits))
+
+
+def rounded_oracle_stats(gpu_out: torch.Tensor, ref: np.ndarray, dtype) -> dict:
+    """Error of the GPU output against the oracle rounded to the output type (round
+    to nearest even, one rounding from fp64): share of bit-identical elements,
+    share within one ulp, and the largest distance in ulps."""
+    got = from_dev(gpu_out).reshape(-1)
+    want = oracle.round_to_dtype(ref, dtype).reshape(-1)
+    d = ulp_distance(got, want)
+    return {"elements": int(d.size), "identical": float(np.mean(d == 0)),
+            "within_1_ulp": float(np.mean(d <= 1)), "max_ulp": int(d.max()) if d.size else 0}

@@ -28,6 +28,11 @@ MUTATIONS = {
                           "v = ldexp((double)(f | 0x400), e - 24);"),
     "scatter_offset": ("int64_t frame = slot / B, off = slot % B;",
                        "int64_t frame = slot / B, off = (B - 1) - slot % B;"),
+    "round_ties_away_from_zero": ("if (r > 0.5 || (r == 0.5 && fmod(f, 2.0) != 0.0)) f += 1.0;",
+                                  "if (r >= 0.5) f += 1.0;"),
+    "round_truncates": ("if (r > 0.5 || (r == 0.5 && fmod(f, 2.0) != 0.0)) f += 1.0;",
+                        "(void)r;"),
+    "round_no_carry": ("      f = ldexp(1.0, frac_bits);\n      e += 1;", "      f = ldexp(1.0, sig) - 1.0;"),
     "prefill_not_causal": ("attend(out + ((int64_t)i * Hq + h) * D, NULL, x, qd, K, V, (int64_t)p0 + i + 1, D, scale);",
                            "attend(out + ((int64_t)i * Hq + h) * D, NULL, x, qd, K, V, n, D, scale);"),
     "prefill_excludes_self": ("attend(out + ((int64_t)i * Hq + h) * D, NULL, x, qd, K, V, (int64_t)p0 + i + 1, D, scale);",

@@ -405,3 +405,99 @@ def test_kv_bytes_per_token_13b_closed_form():
     assert abs(request / 1e9 - g["request_gigabytes"]) < 0.1  # 1.678e9 B, printed as 1.6 GB
     # the kernel's per-layer view of the same shape: 40 heads x 128 = 5120
     assert 2 * 40 * 128 * elt * layers == per_token
+
+
+# --------------------------------------------------------------------------
+# rounding of results to the storage type (round to nearest, ties to even)
+# --------------------------------------------------------------------------
+
+def _format_values(dtype):
+    """All finite values of fp16 / bf16 in increasing order, with their bit patterns
+    (numpy / torch decoders, independent of the oracle)."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    if dtype == wl.F16:
+        vals = bits.view(np.float16).astype(np.float64)
+    else:
+        vals = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    keep = np.isfinite(vals) & ~((vals == 0) & (bits >= 0x8000))  # one zero (+0)
+    order = np.argsort(vals[keep], kind="stable")
+    return vals[keep][order], bits[keep][order]
+
+
+def _nearest_even_reference(x, vals, bits):
+    """Nearest representable value to x by exact rational comparison with its two
+    bracketing neighbours; a tie goes to the pattern whose last bit is 0; beyond
+    the largest finite value the halfway point to the next power step decides
+    between the maximum and infinity."""
+    top, top_bits = vals[-1], int(bits[-1])
+    inf_bits = 0x7C00 if top < 1e6 else 0x7F80
+    ax = abs(x)
+    sign = 0x8000 if x < 0 or (x == 0 and math.copysign(1.0, x) < 0) else 0
+    if ax > top:
+        ulp = top - vals[-2]
+        return sign | (inf_bits if Fraction(ax) >= Fraction(top) + Fraction(ulp) / 2 else top_bits)
+    i = int(np.searchsorted(vals, ax, side="left"))
+    if vals[i] == ax:
+        return sign | int(bits[i])
+    lo, hi = i - 1, i
+    dlo = Fraction(ax) - Fraction(vals[lo])
+    dhi = Fraction(vals[hi]) - Fraction(ax)
+    if dlo < dhi:
+        pick = lo
+    elif dhi < dlo:
+        pick = hi
+    else:
+        pick = lo if int(bits[lo]) % 2 == 0 else hi
+    return sign | int(bits[pick])
+
+
+@pytest.mark.parametrize("dtype", [wl.F16, wl.BF16])
+def test_round_to_dtype_is_identity_on_every_representable_value(dtype):
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = oracle.to_double(bits, dtype)
+    finite = np.isfinite(vals)
+    assert np.array_equal(oracle.round_to_dtype(vals[finite], dtype), bits[finite])
+    inf = np.isinf(vals)
+    assert np.array_equal(oracle.round_to_dtype(vals[inf], dtype), bits[inf])
+
+
+@pytest.mark.parametrize("dtype", [wl.F16, wl.BF16])
+def test_round_to_dtype_midpoints_go_to_even_and_neighbours_to_the_nearer(dtype):
+    vals, bits = _format_values(dtype)
+    pos = vals > 0
+    v, b = vals[pos], bits[pos]
+    mid = (v[:-1] + v[1:]) / 2           # exact in fp64 (a few more bits than the format)
+    got = oracle.round_to_dtype(mid, dtype)
+    even = np.where(b[:-1] % 2 == 0, b[:-1], b[1:])
+    assert np.array_equal(got, even)
+    assert np.array_equal(oracle.round_to_dtype(np.nextafter(mid, np.inf), dtype), b[1:])
+    assert np.array_equal(oracle.round_to_dtype(np.nextafter(mid, -np.inf), dtype), b[:-1])
+    # the same on the negative side, with the sign bit set
+    assert np.array_equal(oracle.round_to_dtype(-mid, dtype), even | 0x8000)
+
+
+@pytest.mark.parametrize("dtype", [wl.F16, wl.BF16])
+def test_round_to_dtype_matches_exact_nearest_search(dtype):
+    vals, bits = _format_values(dtype)
+    rng = np.random.default_rng(11 + dtype)
+    top = vals[-1]
+    tiny = vals[vals > 0][0]
+    x = np.concatenate([
+        rng.standard_normal(1500),
+        np.exp(rng.uniform(np.log(tiny / 4), np.log(top * 1.01), 1500)) * rng.choice([-1, 1], 1500),
+        rng.uniform(0, 4 * tiny, 300),                       # subnormal range
+        np.array([top, top * (1 + 2.0 ** -12), top * 1.5, -top * 1.5, 0.0, -0.0]),
+    ])
+    got = oracle.round_to_dtype(x, dtype)
+    want = np.array([_nearest_even_reference(float(t), vals, bits) for t in x], dtype=np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_round_to_f16_matches_numpy_conversion():
+    # numpy converts float64 -> float16 with one round-to-nearest-even step
+    rng = np.random.default_rng(12)
+    x = np.concatenate([rng.standard_normal(200000) * 10.0 ** rng.integers(-9, 5, 200000),
+                        rng.uniform(-70000, 70000, 20000)])
+    with np.errstate(over="ignore"):
+        want = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(oracle.round_to_dtype(x, wl.F16), want)
