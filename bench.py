@@ -80,8 +80,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["decode", "cache-ops"], default="decode",
-                    help="cache-ops: time reshape_and_cache and copy_blocks alone at HBM-bound sizes")
+    ap.add_argument("--op", choices=["decode", "cache-ops", "prefill"], default="decode",
+                    help="cache-ops: time reshape_and_cache and copy_blocks alone at HBM-bound sizes; "
+                         "prefill: time the chunked-prefill batch alone")
     ap.add_argument("--workload", default="gqa8b", choices=["tiny", "mha13b", "gqa8b", "long"])
     ap.add_argument("--l2-flush", choices=["clean", "dirty"], default="clean",
                     help="L2 eviction before each timed step: 256 MiB write then read (clean) or write only")
@@ -139,6 +140,77 @@ def job_throughput(step_ms, step_bytes: float, step_seqs: float, device=None):
 def barrier():
     if torch.distributed.is_available() and torch.distributed.is_initialized():
         torch.distributed.barrier()
+
+
+def measured_tensor_peak(sustained: bool = False):
+    """Dense bf16 tensor-core TFLOP/s measured on this machine (MEASURED_PEAKS.json:
+    the burst figure for a kernel timed alone, the sustained one for a kernel
+    inside a long loop), else the recorded fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    try:
+        with open(path) as f:
+            return float(json.load(f)[key]), "measured"
+    except Exception:
+        return (1400.0 if sustained else 1590.0), "fallback"
+
+
+def prefill_flops(inp: wl.PrefillInputs) -> int:
+    """Algorithmic flops of causal prefill attention: each new token i of a
+    sequence scores and weights p0 + i + 1 keys, 2 flops per multiply-add in
+    q.K and in P.V, per query head and head dimension."""
+    w = inp.w
+    per_row_key = 4 * w.head_dim * w.num_heads
+    total = 0
+    for p0, T in zip(inp.cached.astype(np.int64), inp.chunk.astype(np.int64)):
+        total += int(T * p0 + T * (T + 1) // 2)
+    return per_row_key * total
+
+
+def time_prefill(args, flush, device):
+    """Chunked prefill over the paged cache (the prefill workload): every token's
+    K/V written with the cache write, then the prefill call timed alone as a CUDA
+    graph (events as graph nodes), the L2 flushed before each call."""
+    from paged_kv_cache_419_b200 import binding as pkv
+
+    inp = wl.make_prefill_inputs("prefill")
+    w = inp.w
+    td = torch.float16 if w.dtype == wl.F16 else torch.bfloat16
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(td).to(device)
+
+    a = pkv.BlockAllocator(w.num_blocks, w.block_size, inp.frame_order)
+    slots = np.concatenate([a.add_seq(s, int(inp.context_lens[s])) for s in range(w.num_seqs)])
+    table, lens = a.block_table(np.arange(w.num_seqs, dtype=np.int32), w.max_blocks_per_seq)
+    a.close()
+    shape = (w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+    kc = torch.zeros(shape, dtype=td, device=device)
+    vc = torch.zeros(shape, dtype=td, device=device)
+    pkv.reshape_and_cache(dev(inp.k_stream), dev(inp.v_stream), kc, vc, torch.from_numpy(slots).to(device))
+    q = dev(inp.q)
+    out = torch.empty_like(q)
+    tab_d, lens_d = torch.from_numpy(table).to(device), torch.from_numpy(lens).to(device)
+    qs_d = torch.from_numpy(inp.query_start).to(device)
+    max_q = int(inp.chunk.max())
+
+    def call():
+        pkv.paged_prefill(out, q, kc, vc, tab_d, qs_d, lens_d, w.scale, max_q)
+
+    ms = graph_time_ms(call, flush, args.l2_flush, max(args.steps, 5))
+    if pkv.device_error():
+        raise RuntimeError("device error flags set by the prefill")
+    flops = prefill_flops(inp)
+    peak, kind = measured_tensor_peak()
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"ms": round(ms, 5), "tflops": round(tflops, 1), "flops": int(flops),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak, "peak_kind": kind,
+                         "unit": "TFLOP/s", "frac": round(tflops / peak, 4)},
+            "workload": (f"{w.num_seqs} sequences, {w.num_heads}/{w.num_kv_heads} heads, D={w.head_dim}, "
+                         f"B={w.block_size}, {wl.DTYPE_NAMES[w.dtype]}; chunks of "
+                         f"{int(inp.chunk.min())}-{int(inp.chunk.max())} new tokens after "
+                         f"{int(inp.cached.min())}-{int(inp.cached.max())} cached ones"),
+            "new_tokens": int(inp.chunk.sum()), "context_tokens": int(inp.context_lens.sum())}
 
 
 def measured_hbm_peak():
@@ -377,8 +449,8 @@ def merge_alone_ms(call, K):
         ev[1].record()
     torch.cuda.current_stream().wait_stream(side)
     graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
-    _, n = ok(rt.cudaGraphGetNodes(graph, numNodes=0))
-    nodes, n = ok(rt.cudaGraphGetNodes(graph, numNodes=n))
+    _, n = ok(rt.cudaGraphGetNodes(graph, 0))
+    nodes, n = ok(rt.cudaGraphGetNodes(graph, n))
     kinds = [ok(rt.cudaGraphNodeGetType(nd))[0] for nd in nodes]
     kernels = [nd for nd, k in zip(nodes, kinds) if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel]
     records = [nd for nd, k in zip(nodes, kinds) if k == rt.cudaGraphNodeType.cudaGraphNodeTypeEventRecord]
@@ -387,10 +459,10 @@ def merge_alone_ms(call, K):
                            f"{len(kernels)} kernels and {len(records)} events")
 
     def deps(nd):
-        _, _, m = ok(rt.cudaGraphNodeGetDependencies_v2(nd, numDependencies=0))
+        _, _, m = ok(rt.cudaGraphNodeGetDependencies_v2(nd, 0))
         if m == 0:
             return []
-        found, _, m = ok(rt.cudaGraphNodeGetDependencies_v2(nd, numDependencies=m))
+        found, _, m = ok(rt.cudaGraphNodeGetDependencies_v2(nd, m))
         return [int(x) for x in found[:m]]
 
     first = [r for r in records if not deps(r)]
@@ -601,6 +673,11 @@ def config_sweep(args, flush, device, peak):
                                  pass2=True)
     res["long"] = r
     del b, ws
+    torch.cuda.empty_cache()
+    try:  # the prefill leg never costs the decode figures
+        res["prefill"] = time_prefill(args, flush, device)
+    except Exception as e:
+        res["prefill"] = {"error": f"{type(e).__name__}: {e}"}
     torch.cuda.empty_cache()
     return res
 
@@ -1261,6 +1338,12 @@ def main(argv=None):
     elif args.op == "cache-ops":
         if rank == 0:
             run_cache_ops(args, local)
+    elif args.op == "prefill":
+        if rank == 0:
+            torch.cuda.set_device(local)
+            device = torch.device("cuda", local)
+            flush = torch.zeros(2 * L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+            print(json.dumps({"op": "prefill", **time_prefill(args, flush, device)}), flush=True)
     else:
         run_ours(args, world, rank, local)
 

@@ -102,7 +102,8 @@ pkv_status pkv_test_set_merge_wait(uint64_t limit_ns, uint32_t extra);
  * 32 * num_seqs * P bytes of work records (one per context partition), and, when
  * P > 1, the partition results num_seqs * num_heads * P * (head_dim + 2) * 4
  * bytes; each piece rounded up to 256 bytes, with
- * P = ceil(max_context_len / partition_size).  partition_size 0 = default (1024).
+ * P = ceil(max_context_len / partition_size), partition_size 0 (the default
+ * policy) counting as 512.
  * Returns 0 for invalid arguments; the decode call then rejects them.
  */
 size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
@@ -132,10 +133,17 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t h
  *                kernel may read further entries of the row, up to one partition's
  *                worth, without using them, so the whole row must be readable)
  *   context_lens device int32 [num_seqs], 0 <= context_lens[s] <= max_blocks_per_seq * block_size
- *   partition_size maximum tokens per context partition (0 = 1024); a multiple of 64
- *                in [64, 2048].  A context of L tokens is split into ceil(L / partition_size)
+ *   partition_size maximum tokens per context partition, a multiple of 64 in
+ *                [64, 2048]: a context of L tokens is split into ceil(L / partition_size)
  *                near-equal partitions (multiples of 64 tokens) that run on different
  *                CTAs and are merged with a log-sum-exp in the same launch sequence.
+ *                0 = the default policy: partitions of up to 1024 tokens; but when the
+ *                batch has fewer (sequence, kv head) pairs than the decode grid has
+ *                CTAs (a few long contexts), partitions are sized per call so that
+ *                the batch's token-heads make about k whole waves of the grid, k =
+ *                max(1, round(token-heads / (CTAs x 1024))): a context of L tokens
+ *                gets about L k CTAs / token-heads partitions (64 to 2048 tokens each,
+ *                at most ceil(L / 512) of them).
  *   workspace    device scratch of pkv_decode_workspace_bytes(num_seqs, num_heads,
  *                head_dim, max_blocks_per_seq * block_size, partition_size) bytes,
  *                16-byte aligned; contents need no initialisation and are garbage
@@ -209,6 +217,50 @@ pkv_status pkv_contiguous_attention_decode(void* out, const void* q, const void*
                                            int32_t num_kv_heads, int32_t head_dim, pkv_dtype dtype,
                                            int32_t partition_size, void* workspace,
                                            size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Paged prefill attention (slide 3: the prompt is processed in parallel before
+ * decoding; dataarena note section 4, step 3: a scheduled request runs its
+ * prefill; slides 9-10: attention block by block through the block table).
+ *
+ * Sequence s brings T_s = query_start[s+1] - query_start[s] new tokens at
+ * positions p0_s .. p0_s + T_s - 1, p0_s = context_lens[s] - T_s (p0 = 0: a
+ * whole prompt; p0 > 0: a later chunk of one).  Their keys and values are
+ * already in the cache (written with pkv_reshape_and_cache).  New token i of
+ * sequence s, query head h (kv head g = h / (num_heads/num_kv_heads)):
+ *   out[query_start[s] + i, h, :] =
+ *       sum_{t <= p0_s + i} softmax_t(scale * q[query_start[s] + i, h, :] . K_s[t,:]) V_s[t,:]
+ * with K_s, V_s gathered through the block table as in the decode (causal:
+ * each new token sees the cached context and the new tokens up to itself).
+ * Runs on the tensor cores with fp32 accumulation; the softmax weights enter the
+ * PV product rounded to `dtype` and the normaliser sums those rounded weights,
+ * so each output row is an exact convex combination of V rows up to fp32
+ * rounding; out is rounded to `dtype`.  Max-abs error against exact arithmetic
+ * stays within 2e-3 (fp16) / 1e-2 (bf16) for inputs of unit scale.
+ *
+ *   out, q       device [total_query_tokens, num_heads, head_dim] dtype (rows of
+ *                sequence s at query_start[s] ..); rows outside every chunk are
+ *                not written
+ *   query_start  device int32 [num_seqs + 1], non-decreasing, within
+ *                [0, total_query_tokens]; every T_s <= max_query_len
+ *   context_lens device int32 [num_seqs], T_s <= context_lens[s] <= max_blocks_per_seq * block_size
+ *   block_tables, k_cache, v_cache, num_blocks, block_size as in the decode; the
+ *                first ceil(context_lens[s] / block_size) entries of row s are used
+ *   max_query_len host int, the longest chunk (sets the grid)
+ * Supported: head_dim 64 or 128, block_size 8, 16 or 32, any num_heads that is a
+ * multiple of num_kv_heads (up to 65535 heads and 65535 sequences).  Allocates
+ * nothing and needs no workspace.  A chunk that does not fit (longer than
+ * max_query_len or than the table, outside the query rows) is skipped and
+ * a context length below T_s or above the table's capacity is clamped; both set
+ * PKV_DEVERR_CONTEXT_LEN.  One kernel launch on `stream`.
+ */
+pkv_status pkv_paged_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* query_start,
+                             const int32_t* context_lens, int32_t num_seqs, int32_t max_query_len,
+                             int32_t total_query_tokens, int32_t max_blocks_per_seq,
+                             int32_t num_blocks, float scale, int32_t num_heads,
+                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                             pkv_dtype dtype, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Cache write and copy-on-write block copy                                 */

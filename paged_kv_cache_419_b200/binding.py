@@ -29,7 +29,7 @@ EXPORTS = (
     "pkv_copy_blocks", "pkv_alloc_create", "pkv_alloc_destroy", "pkv_alloc_add_seq",
     "pkv_alloc_fork", "pkv_alloc_append", "pkv_alloc_append_batch", "pkv_alloc_free_seq",
     "pkv_alloc_beam_step", "pkv_alloc_block_table", "pkv_alloc_refcount", "pkv_alloc_stats",
-    "pkv_alloc_add_seq_cached", "pkv_block_hash", "pkv_test_set_merge_wait",
+    "pkv_alloc_add_seq_cached", "pkv_block_hash", "pkv_test_set_merge_wait", "pkv_paged_prefill",
 )
 
 
@@ -102,6 +102,8 @@ def lib() -> ctypes.CDLL:
             "pkv_alloc_refcount": ([P, i32, P], ctypes.c_int),
             "pkv_alloc_stats": ([P, ctypes.POINTER(AllocStats)], ctypes.c_int),
             "pkv_test_set_merge_wait": ([ctypes.c_uint64, ctypes.c_uint32], ctypes.c_int),
+            "pkv_paged_prefill": ([P, P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
+                                   ctypes.c_int, P], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -206,6 +208,26 @@ def contiguous_attention_decode(out, q, k, v, context_lens, scale: float, partit
 
 
 # ---------------------------------------------------------- cache write / copy
+def paged_prefill(out, q, k_cache, v_cache, block_tables, query_start, context_lens, scale: float,
+                  max_query_len: int, stream=None):
+    """Causal attention of each sequence's new tokens (q rows query_start[s] ..
+    query_start[s+1]) over its paged context of context_lens[s] tokens
+    (pkv_paged_prefill).  q, out: [total_tokens, Hq, D]; caches [N, Hkv, B, D]."""
+    total, Hq, D = q.shape
+    N, Hkv, Bs, D2 = k_cache.shape
+    if D2 != D or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch between q, out and the caches")
+    S = context_lens.shape[0]
+    if query_start.shape[0] != S + 1:
+        raise ValueError("query_start must hold num_seqs + 1 offsets")
+    _check(lib().pkv_paged_prefill(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), _dev(query_start, "query_start", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32), S, int(max_query_len), total,
+        block_tables.shape[1], N, float(scale), Hq, Hkv, D, Bs, _dtype_code(q), _stream(stream)),
+        "pkv_paged_prefill")
+
+
 def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
     """Scatter key/value [T, Hkv, D] into the caches [N, Hkv, B, D] at slot_mapping (int64 [T])."""
     T, Hkv, D = key.shape

@@ -9,6 +9,7 @@
 #include "cache_ops.cuh"
 #include "decode.cuh"
 #include "pkv.h"
+#include "prefill.cuh"
 
 namespace pkv {
 
@@ -19,6 +20,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kDefaultPartition = 1024;
+constexpr int kBalancedMinPartition = 512;
 
 struct DeviceInfo {
   bool ready = false;
@@ -67,6 +69,13 @@ bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
 
 int resolve_partition(int32_t partition_size) {
   return partition_size == 0 ? kDefaultPartition : partition_size;
+}
+
+// Partition size that bounds the workspace: the requested one, or for the
+// default (0) the smallest size the per-call balanced policy picks when a
+// context spans several partitions.
+int workspace_partition(int32_t partition_size) {
+  return partition_size == 0 ? kBalancedMinPartition : partition_size;
 }
 
 bool valid_partition(int p) { return p >= kStageTokens && p <= kMaxPartTokens && p % kStageTokens == 0; }
@@ -162,11 +171,15 @@ pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pk
   if (a.num_seqs == 0) return PKV_OK;
   const int part = resolve_partition(partition_size);
   if (!valid_partition(part)) return PKV_EINVAL;
+  const int ws_part = workspace_partition(partition_size);
   const int group = a.num_heads / a.num_kv_heads;
   a.part_tokens = part;
-  a.max_parts = (a.max_ctx + part - 1) / part;
+  // default size: the launcher switches to the balanced policy when the batch
+  // has fewer (sequence, kv head) pairs than decode CTAs
+  a.balanced = partition_size == 0 ? 1 : 0;
+  a.max_parts = (a.max_ctx + ws_part - 1) / ws_part;
   if (a.max_parts < 1) a.max_parts = 1;
-  const WorkspaceLayout lay = workspace_layout(a.num_seqs, a.num_heads, head_dim, a.max_ctx, part);
+  const WorkspaceLayout lay = workspace_layout(a.num_seqs, a.num_heads, head_dim, a.max_ctx, ws_part);
   if (!workspace || ws_bytes < static_cast<size_t>(lay.total) || !aligned16(workspace))
     return PKV_EINVAL;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -260,6 +273,54 @@ pkv_status validate_copy_pairs(const int64_t* pairs, int32_t n, int32_t num_bloc
   return PKV_OK;
 }
 
+// Map of q viewed as [total_q][Hq][head_dim] 16-bit elements: boxes of one
+// 128-byte panel x 1 head x 128 query rows, 128-byte swizzle (the K-major
+// layout the tensor cores read), zero fill past the last row.
+pkv_status encode_query_map(CUtensorMap* m, const void* q, pkv_dtype dtype, int head_dim,
+                            int64_t num_heads, int64_t total_q) {
+  const EncodeTiledFn fn = encode_tiled();
+  if (!fn) return PKV_ECUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_heads),
+                              static_cast<cuuint64_t>(total_q > 0 ? total_q : 1)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                 static_cast<cuuint64_t>(num_heads) * head_dim * 2};
+  const cuuint32_t box[3] = {64u, 1u, static_cast<cuuint32_t>(kPrefillTileM)};
+  const cuuint32_t elem_strides[3] = {1u, 1u, 1u};
+  const CUresult r =
+      fn(m, dtype == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+         const_cast<void*>(q), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_EINVAL;
+}
+
+// PKV_VALIDATE=1 check of a prefill batch (host copies of the query offsets,
+// context lengths and block tables).
+pkv_status validate_prefill(const int32_t* query_start, const int32_t* lens, const int32_t* tables,
+                            int32_t S, int32_t max_query_len, int32_t total_q, int32_t MB,
+                            int32_t N, int32_t B, cudaStream_t stream) {
+  std::vector<int32_t> qs(static_cast<size_t>(S) + 1), h_lens(S), h_tab(static_cast<size_t>(S) * MB);
+  if (cudaMemcpyAsync(qs.data(), query_start, sizeof(int32_t) * qs.size(), cudaMemcpyDeviceToHost,
+                      stream) != cudaSuccess ||
+      cudaMemcpyAsync(h_lens.data(), lens, sizeof(int32_t) * S, cudaMemcpyDeviceToHost, stream) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(h_tab.data(), tables, sizeof(int32_t) * h_tab.size(), cudaMemcpyDeviceToHost,
+                      stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return PKV_ECUDA;
+  for (int32_t s = 0; s < S; ++s) {
+    const int64_t T = static_cast<int64_t>(qs[s + 1]) - qs[s];
+    const int64_t L = h_lens[s];
+    if (qs[s] < 0 || T < 0 || qs[s + 1] > total_q || T > max_query_len) return PKV_ERANGE;
+    if (L < T || L > static_cast<int64_t>(MB) * B) return PKV_ERANGE;
+    for (int64_t j = 0; j < (L + B - 1) / B; ++j) {
+      const int32_t p = h_tab[static_cast<size_t>(s) * MB + j];
+      if (p < 0 || p >= N) return PKV_ERANGE;
+    }
+  }
+  return PKV_OK;
+}
+
 }  // namespace
 }  // namespace pkv
 
@@ -305,7 +366,8 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t h
   if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
       !valid_partition(part))
     return 0;
-  return workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, part);
+  return workspace_bytes(num_seqs, num_heads, head_dim, max_context_len,
+                         workspace_partition(partition_size));
 }
 
 pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
@@ -382,6 +444,68 @@ pkv_status pkv_contiguous_attention_decode(void* out, const void* q, const void*
   a.max_ctx = max_context_len;
   return decode_common(a, head_dim, 32, dtype, partition_size, workspace, workspace_bytes, false,
                        scale, stream);
+}
+
+pkv_status pkv_paged_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* query_start,
+                             const int32_t* context_lens, int32_t num_seqs, int32_t max_query_len,
+                             int32_t total_query_tokens, int32_t max_blocks_per_seq,
+                             int32_t num_blocks, float scale, int32_t num_heads,
+                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                             pkv_dtype dtype, cudaStream_t stream) {
+  if (num_seqs < 0 || max_query_len < 0 || total_query_tokens < 0 || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0 || num_heads <= 0 || num_kv_heads <= 0)
+    return PKV_EINVAL;
+  if (dtype != PKV_F16 && dtype != PKV_BF16) return PKV_EUNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PKV_EUNSUPPORTED;
+  if (num_heads % num_kv_heads != 0) return PKV_EUNSUPPORTED;
+  if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_EUNSUPPORTED;
+  if (num_seqs > 65535 || num_heads > 65535) return PKV_EUNSUPPORTED;
+  if (static_cast<int64_t>(max_blocks_per_seq) * block_size > (1 << 30)) return PKV_EUNSUPPORTED;
+  if (num_seqs == 0 || max_query_len == 0 || total_query_tokens == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !query_start || !context_lens)
+    return PKV_EINVAL;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_EINVAL;
+  if (validate_env()) {
+    const pkv_status vs = validate_prefill(query_start, context_lens, block_tables, num_seqs,
+                                           max_query_len, total_query_tokens, max_blocks_per_seq,
+                                           num_blocks, block_size, stream);
+    if (vs != PKV_OK) return vs;
+  }
+  DeviceInfo* dev = nullptr;
+  pkv_status st = device_info(&dev);
+  if (st != PKV_OK) return st;
+  PrefillArgs a{};
+  a.out = out;
+  a.tables = block_tables;
+  a.query_start = query_start;
+  a.lens = context_lens;
+  a.num_seqs = num_seqs;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.block_size = block_size;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.total_q = total_query_tokens;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.err = dev->err;
+  PrefillMaps maps;
+  if ((st = encode_query_map(&maps.q, q, dtype, head_dim, num_heads, total_query_tokens)) != PKV_OK)
+    return st;
+  const int64_t rows = static_cast<int64_t>(num_kv_heads) * block_size;
+  if ((st = encode_cache_map(&maps.k, k_cache, dtype, head_dim, rows, num_blocks, block_size)) != PKV_OK)
+    return st;
+  if ((st = encode_cache_map(&maps.v, v_cache, dtype, head_dim, rows, num_blocks, block_size)) != PKV_OK)
+    return st;
+  cudaError_t e;
+  if (dtype == PKV_F16)
+    e = head_dim == 64 ? launch_prefill<__half, 64>(a, maps, max_query_len, stream)
+                       : launch_prefill<__half, 128>(a, maps, max_query_len, stream);
+  else
+    e = head_dim == 64 ? launch_prefill<__nv_bfloat16, 64>(a, maps, max_query_len, stream)
+                       : launch_prefill<__nv_bfloat16, 128>(a, maps, max_query_len, stream);
+  return from_cuda(e);
 }
 
 pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,

@@ -70,10 +70,12 @@ struct DecodeArgs {
   int32_t num_kv_heads;
   int32_t max_ctx;        // capacity in tokens: MB * B (paged) or the contiguous stride
   int32_t part_tokens;    // maximum tokens per partition (multiple of 64)
-  int32_t max_parts;      // ceil(max_ctx / part_tokens): upper bound of partitions per context
+  int32_t max_parts;      // upper bound of partitions per context (workspace stride)
+  int32_t balanced;       // 1: partitions sized per call from the batch's total work
   float scale_log2;       // scale * log2(e)
   int32_t grid_ctas;      // decode CTAs; item c (c < grid_ctas) is CTA c's first item
-  uint32_t* work;         // [0] next item, [1] item count, [2] multi-partition sequences
+  uint32_t* work;         // [0] next item, [1] item count, [2] multi-partition sequences,
+                          // [4..5] (balanced) the batch's token-heads U as a uint64
   uint32_t* pair_done;    // [S * Hkv] partitions published per (sequence, kv head)
   int32_t* merge_seqs;    // [S] sequences whose context spans more than one partition
   uint8_t* records;       // [S * max_parts] work records, largest partition first (32 B each)
@@ -114,6 +116,45 @@ __device__ __forceinline__ void partition_of(int L, int part_tokens, int& n, int
   const int n0 = (L + part_tokens - 1) / part_tokens;
   size = ((L + n0 - 1) / n0 + kStageTokens - 1) & ~(kStageTokens - 1);
   n = (L + size - 1) / size;
+}
+
+// Balanced partitioning, for batches with fewer (sequence, kv head) pairs than
+// decode CTAs: there, fixed-size partitions leave a last wave of a few items
+// on an otherwise idle grid.  The batch's U = Hkv x sum L token-heads are cut
+// into about k x grid items of near-equal size, k = max(1, round(U / (grid x
+// 1024))): a context of L tokens gets n = round(L k grid / U) partitions (at
+// least ceil(L / kMaxPartTokens), at most max_parts and ceil(L / 64)) of equal
+// size rounded up to a multiple of 64 (the last one shorter).  Integer
+// arithmetic only: the plan, the statically started CTAs and the merge agree.
+__device__ __forceinline__ void partition_balanced(int L, unsigned long long U, int grid,
+                                                   int max_parts, int& n, int& size) {
+  if (L <= 0 || U == 0) {
+    n = 1;
+    size = L > 0 ? L : 0;
+    return;
+  }
+  const long long g = grid;
+  long long k = (static_cast<long long>(U) + g * 512) / (g * 1024);
+  if (k < 1) k = 1;
+  long long nn = (static_cast<long long>(L) * k * g + static_cast<long long>(U / 2)) /
+                 static_cast<long long>(U);
+  const long long lo = (L + kMaxPartTokens - 1) / kMaxPartTokens;
+  const long long hi = min(static_cast<long long>(max_parts), static_cast<long long>((L + 63) / 64));
+  nn = nn < lo ? lo : nn;
+  nn = nn > hi ? hi : nn;
+  if (nn < 1) nn = 1;
+  size = ((L + static_cast<int>(nn) - 1) / static_cast<int>(nn) + kStageTokens - 1) & ~(kStageTokens - 1);
+  n = (L + size - 1) / size;
+}
+
+// Partitions of a context of L tokens under this call's policy (U: the batch's
+// token-heads, used by the balanced policy only).
+__device__ __forceinline__ void partition_for(int L, const DecodeArgs& a, unsigned long long U,
+                                              int& n, int& size) {
+  if (a.balanced)
+    partition_balanced(L, U, a.grid_ctas, a.max_parts, n, size);
+  else
+    partition_of(L, a.part_tokens, n, size);
 }
 
 // Sequences whose partition 0 runs as a static first item: decode CTA c
@@ -228,11 +269,26 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
   __shared__ uint32_t total, n_multi, n_wide;
   __shared__ int4 s_wide[kPlanWide];  // (sequence, first full-size slot, last slot, first listed partition)
   __shared__ int s_len[kPlanSmemSeqs];
+  __shared__ unsigned long long s_U;
   const int classes = a.part_tokens / 32 + 2;  // class c: size in (part - 32(c+1), part - 32c]; last: empty
   const bool cached = a.num_seqs <= kPlanSmemSeqs;
   for (int c = threadIdx.x; c < classes; c += blockDim.x) count[c] = 0;
-  if (threadIdx.x == 0) total = n_multi = n_wide = 0;
+  if (threadIdx.x == 0) {
+    total = n_multi = n_wide = 0;
+    s_U = 0ull;
+  }
   __syncthreads();
+  // Balanced policy: the batch's token-heads first (the merge grid reads them too).
+  unsigned long long U = 0;
+  if (a.balanced) {
+    unsigned long long mine = 0;
+    for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x)
+      mine += static_cast<unsigned long long>(clamp_len(a.lens[s], a.max_ctx));
+    atomicAdd(&s_U, mine);
+    __syncthreads();
+    U = s_U * static_cast<unsigned long long>(a.num_kv_heads);
+    if (threadIdx.x == 0) *reinterpret_cast<unsigned long long*>(a.work + 4) = U;
+  }
   auto size_class = [&](int sz) { return sz == 0 ? classes - 1 : (a.part_tokens - sz) / 32; };
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int raw = a.lens[s];
@@ -240,7 +296,7 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
     const int L = clamp_len(raw, a.max_ctx);
     if (cached) s_len[s] = L;
     int n, size;
-    partition_of(L, a.part_tokens, n, size);
+    partition_for(L, a, U, n, size);
     // listed partitions: skip .. n-1 (partition 0 of a static sequence is not
     // listed); partitions below n-1 have `size` tokens, the last one the rest
     const int skip = s < n_static ? 1 : 0;
@@ -304,7 +360,7 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int L = cached ? s_len[s] : clamp_len(a.lens[s], a.max_ctx);
     int n, size;
-    partition_of(L, a.part_tokens, n, size);
+    partition_for(L, a, U, n, size);
     const int last = L - (n - 1) * size;
     const int skip = s < n_static ? 1 : 0;
     const int n_full = n - 1 - skip;
@@ -329,7 +385,7 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
       const int s = e.x;
       const int L = cached ? s_len[s] : clamp_len(a.lens[s], a.max_ctx);
       int n, size;
-      partition_of(L, a.part_tokens, n, size);
+      partition_for(L, a, U, n, size);
       for (int p = e.w + lane; p < n; p += 32)
         write_record(s, p, n, size, L,
                      p < n - 1 ? static_cast<uint32_t>(e.y + p - e.w) : static_cast<uint32_t>(e.z));
@@ -486,11 +542,21 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
         cp_async_arrive_noinc(&tab_bar[0]);
         tab_pending |= 1u;  // buffer 0, phase 0
       }
+      // Balanced policy: the batch's token-heads, summed by the warp (a batch
+      // with static items for every sequence has fewer than grid / Hkv of them).
+      unsigned long long U = 0;
+      if (a.balanced) {
+        for (int t = lane; t < a.num_seqs; t += 32)
+          U += static_cast<unsigned long long>(clamp_len(a.lens[t], a.max_ctx));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) U += __shfl_xor_sync(0xffffffffu, U, o);
+        U *= static_cast<unsigned long long>(a.num_kv_heads);
+      }
       if (lane == 0) {  // record of partition 0 of sequence blockIdx.x / Hkv, in slot 0
         int32_t* r = reinterpret_cast<int32_t*>(smem + Tr::OFF_REC);
         const int L = clamp_len(a.lens[s], a.max_ctx);
         int n, size;
-        partition_of(L, a.part_tokens, n, size);
+        partition_for(L, a, U, n, size);
         r[0] = s;
         r[1] = 0;
         r[2] = n;
@@ -983,12 +1049,14 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
   const uint32_t Hkv = static_cast<uint32_t>(a.num_kv_heads);
   // The plan finished before the decode grid let this grid launch.
   const uint32_t n_tasks = __ldcg(a.work + 2) * Hkv;
+  const unsigned long long U =
+      a.balanced ? __ldcg(reinterpret_cast<const unsigned long long*>(a.work + 4)) : 0ull;
   for (uint32_t t = blockIdx.x; t < n_tasks; t += gridDim.x) {
     const int s = __ldcg(a.merge_seqs + t / Hkv);
     const int kvh = static_cast<int>(t % Hkv);
     const int h0 = kvh * G;
     int np, psize;
-    partition_of(clamp_len(a.lens[s], a.max_ctx), a.part_tokens, np, psize);
+    partition_for(clamp_len(a.lens[s], a.max_ctx), a, U, np, psize);
     const int64_t base0 = (static_cast<int64_t>(s) * a.num_heads + h0) * a.max_parts;
     auto cell = [&](int g, int p) { return base0 + static_cast<int64_t>(g) * a.max_parts + p; };
     // Wait (bounded) until the decode grid has published all np partitions of
@@ -1041,8 +1109,11 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int c0 = 0; c0 < np; c0 += kMergeChunk) {
       const int cn = min(kMergeChunk, np - c0);
-      if (c0 > 0) {
-        __syncthreads();  // the previous chunk's weights are no longer read
+      // One chunk: its statistics are still in s_m / s_w from the pass above.
+      // Several: that pass left the last chunk there, so every chunk (the first
+      // included) is loaded again.
+      if (np > kMergeChunk) {
+        if (c0 > 0) __syncthreads();  // the previous chunk's weights are no longer read
         for (int i = tid; i < G * cn; i += kMergeThreads) {
           const int g = i / cn, p = i % cn;
           s_m[g][p] = __ldcg(a.tmp_m + cell(g, c0 + p));

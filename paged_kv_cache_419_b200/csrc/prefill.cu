@@ -1,0 +1,485 @@
+// Paged prefill attention for sm_100a (tcgen05 tensor cores, TMEM accumulators).
+//
+// Method (vLLM and PagedAttention slide 3: the prompt is processed in parallel
+// before decoding starts; dataarena note section 4, step 3: a scheduled request
+// runs its prefill; slides 9-10: attention reads keys and values block by block
+// through the block table).  A sequence s gets T new tokens at positions
+// p0 .. p0 + T - 1 (a whole prompt when p0 = 0, a later chunk of it otherwise);
+// their keys and values are already in the paged cache, written by the cache
+// write.  New token i attends causally over positions 0 .. p0 + i:
+//   out[i, h, :] = sum_{t <= p0 + i} softmax_t(scale q[i, h, :] . K[t, :]) V[t, :]
+// with kv head h / (Hq / Hkv).  Unlike the single-query decode, this is a dense
+// contraction (T x D by D x L), so it runs on the tensor cores.
+//
+// Kernel design (B200).
+//  * One CTA per (sequence, 128-query tile, query head); 192 threads, one CTA
+//    per SM (192 KB of shared memory at head_dim 128).
+//  * Warp 0 loads: the tile's Q rows once (TMA, 128-byte swizzle), then the
+//    K and V tiles of 128 keys through a ring of two stages, one TMA box per
+//    cache block and 128-byte panel, with the frames taken from the block table.
+//  * Warp 1 holds the tensor memory (512 columns: two 128-column score buffers
+//    and the output accumulator) and one of its threads issues the tcgen05.mma
+//    instructions: S_j = Q K_j^T into score buffer j % 2, then O += P_{j-1}
+//    V_{j-1}, so the scores of tile j are computed while the softmax of tile
+//    j - 1 runs.  Q, K and P are K-major operands; V is used as it lies in the
+//    cache tiles, as an MN-major operand.  Completion is signalled to
+//    mbarriers with tcgen05.commit.
+//  * Warps 2-5 own one query row per thread (tensor-memory lane = row): they
+//    read the row's scores from tensor memory, apply the causal mask by select
+//    (so garbage keys past the context never reach a sum), keep the running
+//    max and sum (base-2 units), rescale the output row in tensor memory when
+//    the max grows, and write P (rounded to the input type) into shared memory
+//    for the next product.  The sum is taken over the rounded weights, so the
+//    output is an exact convex combination of V rows.  In the last key tile
+//    they zero the V rows past the context (0 x NaN would be NaN).
+//  * Epilogue: out = O / l, rounded to the input type, written per row.
+//  * Every mbarrier wait is bounded; on expiry the kernel sets
+//    PKV_DEVERR_WAIT_TIMEOUT, waits (bounded) for its own copies and tensor-core
+//    work, frees its tensor memory and returns.
+#include "prefill.cuh"
+
+namespace pkv {
+
+// ------------------------------------------------------------ tcgen05 helpers
+// Shared-memory matrix descriptor (sm_100 format): start address, leading and
+// stride byte offsets (all >> 4), version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16 with fp32 accumulation: A and B of the
+// same 16-bit type (f16 = 0, bf16 = 1), A K-major, B K-major (0) or MN-major
+// (1), shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(uint32_t ab_format, uint32_t b_mn_major,
+                                                      uint32_t M, uint32_t N) {
+  return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (b_mn_major << 16) |
+         ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+      : "memory");
+}
+
+// Arrive on `bar` once every tcgen05 operation this thread issued so far is done.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31, %32};"
+      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+        "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+        "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+        "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+        "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+        "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+        "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+        "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ------------------------------------------------------------ kernel
+template <typename T, int D>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    prefill_kernel(const PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
+  using Tr = PrefillTraits<D>;
+  constexpr int ND = Tr::ND;
+  constexpr int KSTEPS = D / 16;          // k-steps of S = Q K^T
+  constexpr int PV_STEPS = kPrefillTileN / 16;
+  constexpr uint32_t AB_FMT = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+  constexpr uint32_t IDESC_S = umma_idesc_f16(AB_FMT, 0u, kPrefillTileM, kPrefillTileN);
+  constexpr uint32_t IDESC_O = umma_idesc_f16(AB_FMT, 1u, kPrefillTileM, D);
+
+  // ---- which tile: x = query head (the G heads of a kv head are neighbours,
+  // so their CTAs share K/V tiles in L2), y = query tile (largest first), z = sequence
+  const int h = blockIdx.x;
+  const int s = blockIdx.z;
+  const int q0 = __ldg(a.query_start + s);
+  const int n_new = __ldg(a.query_start + s + 1) - q0;  // T, the chunk's tokens
+  const int i0 = static_cast<int>(gridDim.y - 1 - blockIdx.y) * kPrefillTileM;
+  // A chunk that does not fit the launch (longer than max_query_len, outside
+  // the query rows, or longer than the table can hold) is skipped and flagged.
+  const int cap = a.max_blocks * a.block_size;
+  if (q0 < 0 || n_new < 0 || q0 + n_new > a.total_q ||
+      n_new > static_cast<int>(gridDim.y) * kPrefillTileM || n_new > cap) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) set_error(a.err, PKV_DEVERR_CONTEXT_LEN);
+    return;
+  }
+  if (i0 >= n_new) return;  // uniform over the CTA, before any set-up
+  int L = __ldg(a.lens + s);
+  if (L < n_new || L > cap) {  // the context must hold the chunk and fit the table: clamped
+    if (threadIdx.x == 0) set_error(a.err, PKV_DEVERR_CONTEXT_LEN);
+    L = L < n_new ? n_new : cap;
+  }
+  const int p0 = L - n_new;
+  const int kvh = h / (a.num_heads / a.num_kv_heads);
+  // keys this tile needs: 0 .. p0 + min(i0 + 127, T - 1)
+  const int last_key = p0 + min(i0 + kPrefillTileM - 1, n_new - 1);
+  const int n_kv = last_key / kPrefillTileN + 1;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Tr::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + kPrefillStages;
+  uint64_t* k_empty = v_full + kPrefillStages;
+  uint64_t* v_empty = k_empty + kPrefillStages;
+  uint64_t* s_full = v_empty + kPrefillStages;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* o_done = p_full + 1;
+  uint64_t* mma_done = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_TMEM);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < kPrefillStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);  // one arrival per softmax warp
+    }
+    mbar_init(p_full, 4);
+    mbar_init(o_done, 1);
+    mbar_init(mma_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {  // the whole warp allocates the tensor memory
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kPrefillTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tmem_fence_before_sync();
+  __syncthreads();
+  tmem_fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  const uint32_t sQ = smem_addr(smem + Tr::OFF_Q);
+  const uint32_t sK = smem_addr(smem + Tr::OFF_K);
+  const uint32_t sV = smem_addr(smem + Tr::OFF_V);
+  const uint32_t sP = smem_addr(smem + Tr::OFF_P);
+
+  if (warp == 0) {
+    // ============================================================ loads
+    const int B = a.block_size;
+    const int32_t* row = a.tables + static_cast<int64_t>(s) * a.max_blocks;
+    bool ok = true;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(Tr::TILE));
+#pragma unroll
+      for (int pn = 0; pn < ND; ++pn)
+        tma_load_3d(smem + Tr::OFF_Q + pn * Tr::PANEL, &maps.q, pn * 64, h, q0 + i0, q_full);
+    }
+    int issued_k = 0, issued_v = 0;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int st = j % kPrefillStages;
+      const int k_lo = j * kPrefillTileN;
+      const int k_hi = min(k_lo + kPrefillTileN, L);           // keys of the context in this tile
+      const int nb = (k_hi - k_lo + B - 1) / B;                 // blocks to load
+      const int blk = lane / ND, pn = lane % ND;                // this lane's block and panel
+      int frame = 0;
+      const bool copier = blk < nb;
+      if (copier) {
+        frame = __ldg(row + k_lo / B + blk);
+        if (frame < 0 || frame >= a.num_blocks) {
+          set_error(a.err, PKV_DEVERR_TABLE_ENTRY);
+          frame = 0;
+        }
+      }
+      const uint32_t bytes = static_cast<uint32_t>(nb * ND * B * 128);
+      const int off = pn * Tr::PANEL + blk * B * 128;
+      // K half of the stage
+      if (lane == 0 && j >= kPrefillStages &&
+          !mbar_wait_bounded(&k_empty[st], ((j / kPrefillStages) - 1) & 1)) {
+        set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+        ok = false;
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      if (lane == 0) mbar_arrive_expect_tx(&k_full[st], bytes);
+      __syncwarp();
+      if (copier)
+        tma_load_3d(smem + Tr::OFF_K + st * Tr::TILE + off, &maps.k, pn * 64, kvh * B, frame, &k_full[st]);
+      ++issued_k;
+      // V half
+      if (lane == 0 && j >= kPrefillStages &&
+          !mbar_wait_bounded(&v_empty[st], ((j / kPrefillStages) - 1) & 1)) {
+        set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+        ok = false;
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      if (lane == 0) mbar_arrive_expect_tx(&v_full[st], bytes);
+      __syncwarp();
+      if (copier)
+        tma_load_3d(smem + Tr::OFF_V + st * Tr::TILE + off, &maps.v, pn * 64, kvh * B, frame, &v_full[st]);
+      ++issued_v;
+    }
+    // Leave no copy in flight: wait (bounded) for the last load into each stage.
+    if (lane == 0) {
+      if (!mbar_wait_bounded(q_full, 0)) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+      for (int j = max(0, issued_k - kPrefillStages); j < issued_k; ++j)
+        if (!mbar_wait_bounded(&k_full[j % kPrefillStages], (j / kPrefillStages) & 1))
+          set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+      for (int j = max(0, issued_v - kPrefillStages); j < issued_v; ++j)
+        if (!mbar_wait_bounded(&v_full[j % kPrefillStages], (j / kPrefillStages) & 1))
+          set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    // ============================================================ tensor cores
+    if (lane == 0) {
+      bool ok = mbar_wait_bounded(q_full, 0);
+      auto issue_pv = [&](int i) {  // O += P_i V_i
+        const int st = i % kPrefillStages;
+        if (!mbar_wait_bounded(p_full, i & 1) ||
+            !mbar_wait_bounded(&v_full[st], (i / kPrefillStages) & 1))
+          return false;
+        tmem_fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < PV_STEPS; ++k) {
+          // A = P, K-major: keys k*16.. in panel k / 4, 32 bytes per k-step inside it
+          const uint64_t ad = umma_desc(sP + (k >> 2) * Tr::PANEL + (k & 3) * 32, 16, 1024);
+          // B = V, MN-major: 16 keys = two 8-row groups of 1024 bytes; panels of 64
+          // dims Tr::PANEL apart
+          const uint64_t bd = umma_desc(sV + st * Tr::TILE + k * 2048, Tr::PANEL, 1024);
+          umma_f16(tmem + Tr::COL_O, ad, bd, IDESC_O, i > 0 || k > 0);
+        }
+        umma_commit(o_done);
+        umma_commit(&v_empty[st]);
+        return true;
+      };
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int st = j % kPrefillStages, b = j & 1;
+        if (!mbar_wait_bounded(&k_full[st], (j / kPrefillStages) & 1) ||
+            (j >= 2 && !mbar_wait_bounded(&s_empty[b], ((j - 2) >> 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tmem_fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < KSTEPS; ++k) {
+          const uint32_t koff = (k >> 2) * Tr::PANEL + (k & 3) * 32;
+          umma_f16(tmem + Tr::COL_S + b * kPrefillTileN, umma_desc(sQ + koff, 16, 1024),
+                   umma_desc(sK + st * Tr::TILE + koff, 16, 1024), IDESC_S, k > 0);
+        }
+        umma_commit(&s_full[b]);
+        umma_commit(&k_empty[st]);
+        if (j >= 1 && !issue_pv(j - 1)) ok = false;
+      }
+      if (ok && !issue_pv(n_kv - 1)) ok = false;
+      if (!ok) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+      // every issued tensor-core operation has finished before the CTA frees
+      // the tensor memory or its shared memory
+      umma_commit(mma_done);
+      if (!mbar_wait_bounded(mma_done, 0)) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ softmax rows
+    const int quarter = warp & 3;                 // tensor-memory lanes 32 quarter ..
+    const int r = quarter * 32 + lane;            // this thread's query row
+    const int i = i0 + r;                         // its token index in the chunk
+    const bool valid = i < n_new;
+    const int limit = valid ? p0 + i : L - 1;     // last key this row may see
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    float m = -CUDART_INF_F, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int b = j & 1;
+      const int k_lo = j * kPrefillTileN;
+      ok = ok && mbar_wait_bounded(&s_full[b], (j >> 1) & 1);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tmem_fence_after_sync();
+      float x[kPrefillTileN];
+#pragma unroll
+      for (int c = 0; c < kPrefillTileN / 32; ++c) {
+        float v[32];
+        tmem_ld32(lane_base + Tr::COL_S + b * kPrefillTileN + c * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[c * 32 + e] = v[e];
+      }
+      tmem_wait_ld();
+      tmem_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[b]);
+      // scale to base-2 units; keys past this row's limit become -inf (select)
+      float mx = -CUDART_INF_F;
+      if (k_lo + kPrefillTileN - 1 <= limit) {
+#pragma unroll
+        for (int t = 0; t < kPrefillTileN; ++t) {
+          x[t] *= a.scale_log2;
+          mx = fmaxf(mx, x[t]);
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < kPrefillTileN; ++t) {
+          x[t] = k_lo + t <= limit ? x[t] * a.scale_log2 : -CUDART_INF_F;
+          mx = fmaxf(mx, x[t]);
+        }
+      }
+      const float m_new = fmaxf(m, mx);
+      const float alpha = m == -CUDART_INF_F ? 0.f : fast_exp2(m - m_new);
+      // P row, rounded to the input type; the sum is over the rounded weights
+      uint32_t pk[kPrefillTileN / 2];
+      float sum = 0.f;
+#pragma unroll
+      for (int t = 0; t < kPrefillTileN; t += 2) {
+        const float e0 = x[t] == -CUDART_INF_F ? 0.f : fast_exp2(x[t] - m_new);
+        const float e1 = x[t + 1] == -CUDART_INF_F ? 0.f : fast_exp2(x[t + 1] - m_new);
+        pk[t / 2] = pack2<T>(e0, e1);
+        const float2 rounded = unpack2<T>(pk[t / 2]);
+        sum += rounded.x + rounded.y;
+      }
+      l = l * alpha + sum;
+      // the previous product has finished reading P and writing O
+      if (j >= 1) ok = ok && mbar_wait_bounded(o_done, (j - 1) & 1);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tmem_fence_after_sync();
+      if (j >= 1 && m_new > m) {  // rescale this row of O
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(lane_base + Tr::COL_O + c * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] *= alpha;
+          tmem_st32(lane_base + Tr::COL_O + c * 32, v);
+        }
+        tmem_wait_st();
+      }
+      m = m_new;
+      // P row r into the K-major, 128-byte swizzled P tile: keys 64 pn .. in
+      // panel pn, 16-byte chunk c of the row at chunk c ^ (r % 8)
+      uint8_t* prow = smem + Tr::OFF_P + r * 128;
+#pragma unroll
+      for (int c = 0; c < kPrefillTileN / 8; ++c) {
+        const int pn = c >> 3, ch = (c & 7) ^ (r & 7);
+        *reinterpret_cast<uint4*>(prow + pn * Tr::PANEL + ch * 16) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      // The tile that reaches past the context: zero the V rows of the keys
+      // past it (whatever the stage held there, 0 x it must be 0).
+      if (k_lo + kPrefillTileN > L) {
+        const int st = j % kPrefillStages;
+        ok = ok && mbar_wait_bounded(&v_full[st], (j / kPrefillStages) & 1);
+        if (ok && k_lo + r >= L) {
+          uint8_t* vrow = smem + Tr::OFF_V + st * Tr::TILE + r * 128;
+#pragma unroll
+          for (int pn = 0; pn < ND; ++pn)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+              *reinterpret_cast<uint4*>(vrow + pn * Tr::PANEL + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();  // generic writes of P (and V) before the tensor cores read them
+      tmem_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    // ---- epilogue: out = O / l
+    ok = ok && mbar_wait_bounded(o_done, (n_kv - 1) & 1);
+    if (__all_sync(0xffffffffu, ok)) {
+      tmem_fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      T* orow = static_cast<T*>(a.out) + (static_cast<int64_t>(q0 + i) * a.num_heads + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float v[32];
+        tmem_ld32(lane_base + Tr::COL_O + c * 32, v);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            const uint4 w = make_uint4(pack2<T>(v[e] * inv, v[e + 1] * inv), pack2<T>(v[e + 2] * inv, v[e + 3] * inv),
+                                       pack2<T>(v[e + 4] * inv, v[e + 5] * inv), pack2<T>(v[e + 6] * inv, v[e + 7] * inv));
+            *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
+          }
+        }
+      }
+    } else if (lane == 0) {
+      set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+    }
+  }
+  tmem_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tmem_fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kPrefillTmemCols)
+                 : "memory");
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_prefill(const PrefillArgs& a, const PrefillMaps& m, int max_query_len,
+                           cudaStream_t stream) {
+  using Tr = PrefillTraits<D>;
+  auto kern = prefill_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>(a.num_heads),
+                  static_cast<unsigned>((max_query_len + kPrefillTileM - 1) / kPrefillTileM),
+                  static_cast<unsigned>(a.num_seqs));
+  kern<<<grid, kPrefillThreads, Tr::SMEM_BYTES, stream>>>(a, m);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_prefill<__half, 64>(const PrefillArgs&, const PrefillMaps&, int, cudaStream_t);
+template cudaError_t launch_prefill<__half, 128>(const PrefillArgs&, const PrefillMaps&, int, cudaStream_t);
+template cudaError_t launch_prefill<__nv_bfloat16, 64>(const PrefillArgs&, const PrefillMaps&, int, cudaStream_t);
+template cudaError_t launch_prefill<__nv_bfloat16, 128>(const PrefillArgs&, const PrefillMaps&, int, cudaStream_t);
+
+}  // namespace pkv

@@ -34,7 +34,8 @@ def test_status_strings():
         assert B.status_string(code).startswith("PKV_")
 
 
-def _layout_bytes(S, Hq, D, ctx, part=1024):
+def _layout_bytes(S, Hq, D, ctx, part=512):
+    # partition_size 0 (the default policy) bounds the workspace as 512-token partitions
     r = lambda x: (x + 255) // 256 * 256
     P = max(1, -(-ctx // part))
     rec = 32
@@ -43,11 +44,12 @@ def _layout_bytes(S, Hq, D, ctx, part=1024):
 
 def test_workspace_bytes_formula():
     # one partition per context: counters and the work list only
-    assert B.decode_workspace_bytes(256, 32, 128, 1024) == _layout_bytes(256, 32, 128, 1024)
-    assert B.decode_workspace_bytes(256, 32, 128, 1024) < 1 << 20
-    # 4096 tokens in the default 1024-token partitions: P = 4 cells of (D + 2) floats
+    assert B.decode_workspace_bytes(256, 32, 128, 512) == _layout_bytes(256, 32, 128, 512)
+    assert B.decode_workspace_bytes(256, 32, 128, 512) < 1 << 20
+    assert B.decode_workspace_bytes(256, 32, 128, 1024, 1024) < 1 << 20
+    # 4096 tokens under the default policy: P = 8 cells of (D + 2) floats
     assert B.decode_workspace_bytes(256, 32, 128, 4096) == _layout_bytes(256, 32, 128, 4096)
-    assert B.decode_workspace_bytes(256, 32, 128, 4096) > 256 * 32 * 4 * 130 * 4
+    assert B.decode_workspace_bytes(256, 32, 128, 4096) > 256 * 32 * 8 * 130 * 4
     # an explicit 512: P = 8
     assert B.decode_workspace_bytes(256, 32, 128, 4096, 512) == _layout_bytes(256, 32, 128, 4096, 512)
     assert B.decode_workspace_bytes(4, 32, 128, 32768, 1024) == _layout_bytes(4, 32, 128, 32768, 1024)

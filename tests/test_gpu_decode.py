@@ -104,11 +104,49 @@ def test_gqa8b_full_size_all_sequences(part):
 
 @pytest.mark.parametrize("part", [64, 512, 0, 2048])
 def test_long_context_partitions(part):
-    """4 x 16K-32K tokens; partition 0 is the default (1024), the benchmark's."""
+    """4 x 16K-32K tokens; partition 0 is the default (1024), the benchmark's.
+    At 64 tokens a context has up to 512 partitions, so the merge runs over
+    several chunks of partition statistics.  Besides the max-abs bound, nearly
+    every element must equal the oracle rounded to bf16: these outputs are small
+    (|out| ~ 0.01), so a wrong merge weight can hide inside the absolute
+    tolerance but not in this count."""
     inp = wl.make_decode_inputs("long")
     out, ref, err, _, _ = run_and_compare(inp, partition_size=part, check_cache=False)
-    print(f"long partition {part}: max-abs error {err:.3e}, vs rounded oracle "
-          f"{rounded_oracle_stats(out, ref, wl.BF16)}")
+    st = rounded_oracle_stats(out, ref, wl.BF16)
+    print(f"long partition {part}: max-abs error {err:.3e}, vs rounded oracle {st}")
+    assert st["within_1_ulp"] >= 0.99, st
+
+
+def test_default_policy_balances_few_long_contexts():
+    """A batch with fewer (sequence, kv head) pairs than decode CTAs, at the
+    default partition size: partitions are sized per call from the batch's total
+    (lengths from one token to 20K, so some contexts get one partition and some
+    dozens).  Same bar as every other case, and bit-identical to the contiguous
+    cache under the same policy."""
+    B = _bin()
+    lens = np.array([1, 63, 64, 65, 700, 5000, 20001, 12000], np.int32)
+    bs = 32
+    max_blocks = -(-int(lens.max()) // bs)
+    w = wl.Workload("few", 12, len(lens), 8, 2, 128, bs, max_blocks * len(lens) + 3, wl.BF16,
+                    max_blocks, 1.0 / np.sqrt(128), lengths=("uniform", 1, 2))
+    inp = wl.make_decode_inputs(w, lengths=lens)
+    out, ref, err, b, _ = run_and_compare(inp, check_cache=False)
+    st = rounded_oracle_stats(out, ref, wl.BF16)
+    print(f"few long contexts, default policy: max-abs {err:.3e}, vs rounded oracle {st}")
+    assert st["within_1_ulp"] >= 0.99, st
+    max_ctx = max_blocks * bs
+    k = torch.zeros(w.num_seqs, w.num_kv_heads, max_ctx, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros_like(k)
+    ks, vs = to_dev(inp.k_stream, w.dtype), to_dev(inp.v_stream, w.dtype)
+    for s in range(w.num_seqs):
+        a, e = int(inp.offsets[s]), int(inp.offsets[s + 1])
+        k[s, :, : e - a] = ks[a:e].transpose(0, 1)
+        v[s, :, : e - a] = vs[a:e].transpose(0, 1)
+    out_c = torch.empty_like(b.q)
+    B.contiguous_attention_decode(out_c, b.q, k, v, b.lens, w.scale)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    assert torch.equal(out_c, out)
 
 
 # ------------------------------------------------------------ normalisation pins

@@ -1,0 +1,32 @@
+"""Host-side pieces of the prefill path (no GPU): the seeded batch layout and
+the benchmark's flop count, checked by brute force."""
+import numpy as np
+
+import bench
+import workloads as wl
+
+
+def test_prefill_batch_layout():
+    inp = wl.make_prefill_inputs("prefill")
+    w = inp.w
+    assert (inp.cached[:4] == 0).all() and (inp.cached <= 4096).all()
+    assert ((inp.chunk >= 256) & (inp.chunk <= 2048)).all()
+    assert inp.query_start[0] == 0 and np.array_equal(np.diff(inp.query_start), inp.chunk)
+    assert inp.q.shape == (int(inp.chunk.sum()), w.num_heads, w.head_dim)
+    assert np.array_equal(np.diff(inp.offsets), inp.context_lens)
+    assert inp.k_stream.shape == (int(inp.context_lens.sum()), w.num_kv_heads, w.head_dim)
+    # the pool holds every sequence's blocks and the table every row
+    assert sum(-(-int(L) // w.block_size) for L in inp.context_lens) <= w.num_blocks
+    assert int(inp.context_lens.max()) <= w.max_blocks_per_seq * w.block_size
+
+
+def test_prefill_flops_count_every_causal_pair_once():
+    w = wl.Workload("tiny-prefill", 3, 3, 4, 2, 64, 16, 64, wl.BF16, 16, 0.125,
+                    lengths=("prefill", 0, 1, 1, 0))
+    inp = wl.make_prefill_inputs(w, cached=[0, 7, 30], chunk=[5, 1, 12])
+    pairs = 0
+    for p0, T in zip(inp.cached, inp.chunk):
+        for i in range(int(T)):
+            pairs += len(range(0, int(p0) + i + 1))  # keys 0 .. p0 + i
+    # q.K and P.V: one multiply-add (2 flops) per head dimension each, per query head
+    assert bench.prefill_flops(inp) == pairs * 2 * 2 * w.head_dim * w.num_heads

@@ -20,6 +20,9 @@ Workloads follow the five decode batches used throughout the project:
                1000 tokens, 0..200 private tokens per sample, 65536 frames
 * ``long``     4 seqs, 32/8 heads, D=128, B=32, bf16, 8192 frames,
                L ~ U{16384..32768}
+* ``prefill``  16 seqs, 32/8 heads, D=128, B=16, bf16, 8192 frames: each a chunk
+               of T ~ U{256..2048} new tokens after p0 ~ U{0..4096} cached ones
+               (p0 = 0 for the first 4: whole prompts)
 
 Draw order inside one workload: context lengths, the physical frame order of
 the pool, q, K, V (for ``shared``: generated lengths, frame order, q, prompt K,
@@ -97,6 +100,11 @@ WORKLOADS = {
     # beam search over a block tree: one 1000-token prompt, 4 beams, 200 steps
     "beam": Workload("beam", 5, 4, 32, 8, 128, 16, 4096, BF16, 76, 1.0 / math.sqrt(128),
                      lengths=("beam", 1000, 200)),
+    # chunked prefill, Llama-3-8B-shaped GQA: 16 sequences, each a chunk of
+    # U{256..2048} new tokens after U{0..4096} cached ones (the first 4 whole
+    # prompts, nothing cached)
+    "prefill": Workload("prefill", 7, 16, 32, 8, 128, 16, 8192, BF16, 384, 1.0 / math.sqrt(128),
+                        lengths=("prefill", 4096, 256, 2048, 4)),
 }
 
 
@@ -345,3 +353,52 @@ def random_pool(rng_seed: int, num_blocks: int, num_kv_heads: int, block_size: i
     rng = np.random.default_rng(rng_seed)
     shape = (num_blocks, num_kv_heads, block_size, head_dim)
     return _normal_bits(rng, shape, dtype), _normal_bits(rng, shape, dtype)
+
+
+@dataclasses.dataclass
+class PrefillInputs:
+    """One prefill batch.  Sequence s has ``cached[s]`` tokens already in the
+    cache and ``chunk[s]`` new ones after them.  ``k_stream``/``v_stream`` hold
+    all of its cached + new tokens in logical order (rows
+    ``offsets[s]:offsets[s+1]``); ``q`` holds the new tokens' queries, sequence
+    after sequence (rows ``query_start[s]:query_start[s+1]``)."""
+    w: Workload
+    cached: np.ndarray        # int32 [S]
+    chunk: np.ndarray         # int32 [S]
+    frame_order: np.ndarray   # int32 [N]
+    q: np.ndarray             # uint16 [sum chunk, Hq, D]
+    k_stream: np.ndarray      # uint16 [sum (cached + chunk), Hkv, D]
+    v_stream: np.ndarray
+    offsets: np.ndarray       # int64 [S + 1]
+    query_start: np.ndarray   # int32 [S + 1]
+
+    @property
+    def context_lens(self) -> np.ndarray:
+        return (self.cached + self.chunk).astype(np.int32)
+
+
+def make_prefill_inputs(name_or_w="prefill", seed: int | None = None, cached=None,
+                        chunk=None) -> PrefillInputs:
+    """Seeded prefill batch.  Draw order: cached lengths, chunk lengths, frame
+    order, q, K, V.  ``cached`` / ``chunk`` override the drawn lengths (tests)."""
+    w = WORKLOADS[name_or_w] if isinstance(name_or_w, str) else name_or_w
+    rng = np.random.default_rng(w.seed if seed is None else seed)
+    _, max_cached, lo, hi, n_whole = w.lengths
+    p0 = rng.integers(0, max_cached, size=w.num_seqs, endpoint=True).astype(np.int32)
+    p0[:n_whole] = 0
+    T = rng.integers(lo, hi, size=w.num_seqs, endpoint=True).astype(np.int32)
+    if cached is not None or chunk is not None:
+        p0 = np.asarray(cached if cached is not None else p0, np.int32)
+        T = np.asarray(chunk if chunk is not None else T, np.int32)
+        w = dataclasses.replace(w, num_seqs=int(T.shape[0]))
+    frame_order = rng.permutation(w.num_blocks).astype(np.int32)
+    total_q = int(T.astype(np.int64).sum())
+    q = _normal_bits(rng, (total_q, w.num_heads, w.head_dim), w.dtype)
+    lens = (p0 + T).astype(np.int64)
+    k = _normal_bits(rng, (int(lens.sum()), w.num_kv_heads, w.head_dim), w.dtype, w.k_scale)
+    v = _normal_bits(rng, (int(lens.sum()), w.num_kv_heads, w.head_dim), w.dtype)
+    offsets = np.zeros(w.num_seqs + 1, dtype=np.int64)
+    np.cumsum(lens, out=offsets[1:])
+    qs = np.zeros(w.num_seqs + 1, dtype=np.int32)
+    np.cumsum(T, out=qs[1:])
+    return PrefillInputs(w, p0, T, frame_order, q, k, v, offsets, qs)
