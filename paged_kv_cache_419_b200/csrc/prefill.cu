@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
       const float m_new = fmaxf(m, mx);
-      const float alpha = m == -CUDART_INF_F ? 0.f : fast_exp2(m - m_new);
+      const float alpha = m == -CUDART_INF_F ? 0.f : (m_new == m ? 1.f : fast_exp2(m - m_new));
       // P row, rounded to the input type; the sum is over the rounded weights
       uint32_t pk[kPrefillTileN / 2];
       float sum = 0.f;
@@ -388,7 +388,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (j >= 1) ok = ok && mbar_wait_bounded(o_done, (j - 1) & 1);
       if (!__all_sync(0xffffffffu, ok)) break;
       tmem_fence_after_sync();
-      if (j >= 1 && m_new > m) {  // rescale this row of O
+      // Rescale the rows of O whose max grew.  tcgen05.ld / st are warp-wide
+      // (.sync.aligned): the whole warp takes the branch when any of its rows
+      // needs it, and rows whose max did not grow multiply by alpha = 1 exactly.
+      if (j >= 1 && __any_sync(0xffffffffu, m_new > m)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float v[32];
