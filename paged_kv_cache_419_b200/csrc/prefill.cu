@@ -12,30 +12,40 @@
 // contraction (T x D by D x L), so it runs on the tensor cores.
 //
 // Kernel design (B200).
-//  * One CTA per (sequence, 128-query tile, query head); 192 threads, one CTA
-//    per SM (192 KB of shared memory at head_dim 128).
-//  * Warp 0 loads: the tile's Q rows once (TMA, 128-byte swizzle), then the
-//    K and V tiles of 128 keys through a ring of two stages, one TMA box per
+//  * One CTA per pair of 128-row query tiles of one sequence: two heads of a
+//    kv group on the same rows when Hq / Hkv is even (both tiles read the same
+//    K/V tiles and do the same work), else two consecutive row tiles of one
+//    head.  320 threads, one CTA per SM (192 KB of shared memory at head_dim
+//    128).  Query tiles with more keys are scheduled first.
+//  * Warp 0 loads: both tiles' Q rows once (TMA, 128-byte swizzle), then the K
+//    and V tiles of 128 keys through a ring of two stages, one TMA box per
 //    cache block and 128-byte panel, with the frames taken from the block table.
-//  * Warp 1 holds the tensor memory (512 columns: two 128-column score buffers
-//    and the output accumulator) and one of its threads issues the tcgen05.mma
-//    instructions: S_j = Q K_j^T into score buffer j % 2, then O += P_{j-1}
-//    V_{j-1}, so the scores of tile j are computed while the softmax of tile
-//    j - 1 runs.  Q, K and P are K-major operands; V is used as it lies in the
-//    cache tiles, as an MN-major operand.  Completion is signalled to
+//  * Warp 1 holds the tensor memory (512 columns: per query tile a 128-column
+//    score buffer and a D-column output accumulator) and one of its threads
+//    issues the tcgen05.mma instructions.  Per key tile j and query tile t:
+//    S_t(j) = Q_t K_j^T (Q, K K-major in shared memory), then O_t += P_t(j) V_j
+//    with P_t(j) read from tensor memory and V used as it lies in the cache
+//    tile, as an MN-major operand.  While the softmax of one query tile runs,
+//    the tensor cores work on the other tile.  Completion is signalled to
 //    mbarriers with tcgen05.commit.
-//  * Warps 2-5 own one query row per thread (tensor-memory lane = row): they
-//    read the row's scores from tensor memory, apply the causal mask by select
-//    (so garbage keys past the context never reach a sum), keep the running
-//    max and sum (base-2 units), rescale the output row in tensor memory when
-//    the max grows, and write P (rounded to the input type) into shared memory
-//    for the next product.  The sum is taken over the rounded weights, so the
-//    output is an exact convex combination of V rows.  In the last key tile
-//    they zero the V rows past the context (0 x NaN would be NaN).
+//  * Warps 2-5 (tile 0) and 6-9 (tile 1) own one query row per thread
+//    (tensor-memory lane = row).  Pass 1 reads the row's scores and takes the
+//    max, with the causal mask applied by select (so garbage keys past the
+//    context never reach a sum); the row of O is rescaled in tensor memory when
+//    the max grows.  Pass 2 turns the scores into P (base-2 exponentials,
+//    rounded to the input type, two per 32-bit column) and stores it over the
+//    first 64 columns of the tile's own score buffer.  The sum is taken over the
+//    rounded weights, so the output is an exact convex combination of V rows.
+//    In the last key tile they zero the V rows past the context (0 x NaN would
+//    be NaN).
+//  * The next scores of a tile overwrite its P, so they are issued only after
+//    the product reading P has completed (tcgen05.mma orders only products
+//    into the same accumulator).
 //  * Epilogue: out = O / l, rounded to the input type, written per row.
 //  * Every mbarrier wait is bounded; on expiry the kernel sets
-//    PKV_DEVERR_WAIT_TIMEOUT, waits (bounded) for its own copies and tensor-core
-//    work, frees its tensor memory and returns.
+//    PKV_DEVERR_WAIT_TIMEOUT and moves on.  Before the tensor memory is freed,
+//    the MMA thread's last tcgen05.commit (which covers every product it issued)
+//    is waited for, and every copy the loader issued has landed.
 #include "prefill.cuh"
 
 namespace pkv {
@@ -120,47 +130,77 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 
+// 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+        "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15])
+      : "memory");
+}
+
+// A from tensor memory, B from shared memory (kind::f16, fp32 accumulation).
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------ kernel
+// Query tile t in {0, 1} of a CTA: head h_t, rows i0_t .. i0_t + 127 of the
+// chunk.  Two heads of one kv group share the rows when Hq / Hkv is even (the
+// tiles read the same K/V tiles and do the same work); otherwise one head
+// takes two consecutive row tiles.
 template <typename T, int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
   using Tr = PrefillTraits<D>;
   constexpr int ND = Tr::ND;
-  constexpr int KSTEPS = D / 16;          // k-steps of S = Q K^T
-  constexpr int PV_STEPS = kPrefillTileN / 16;
+  constexpr int KSTEPS = D / 16;               // k-steps of S = Q K^T
+  constexpr int PV_STEPS = kPrefillTileN / 16; // k-steps of O += P V
   constexpr uint32_t AB_FMT = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t IDESC_S = umma_idesc_f16(AB_FMT, 0u, kPrefillTileM, kPrefillTileN);
   constexpr uint32_t IDESC_O = umma_idesc_f16(AB_FMT, 1u, kPrefillTileM, D);
 
-  // ---- which tile: x = query head (the G heads of a kv head are neighbours,
-  // so their CTAs share K/V tiles in L2), y = query tile (largest first), z = sequence
-  const int h = blockIdx.x;
+  const int G = a.num_heads / a.num_kv_heads;
+  const bool head_pair = (G & 1) == 0;
   const int s = blockIdx.z;
   const int q0 = __ldg(a.query_start + s);
   const int n_new = __ldg(a.query_start + s + 1) - q0;  // T, the chunk's tokens
-  const int i0 = static_cast<int>(gridDim.y - 1 - blockIdx.y) * kPrefillTileM;
-  // A chunk that does not fit the launch (longer than max_query_len, outside
-  // the query rows, or longer than the table can hold) is skipped and flagged.
+  const int rows_per_cta = head_pair ? kPrefillTileM : 2 * kPrefillTileM;
   const int cap = a.max_blocks * a.block_size;
   if (q0 < 0 || n_new < 0 || q0 + n_new > a.total_q ||
-      n_new > static_cast<int>(gridDim.y) * kPrefillTileM || n_new > cap) {
+      n_new > static_cast<int>(gridDim.y) * rows_per_cta || n_new > cap) {
     if (threadIdx.x == 0 && blockIdx.y == 0) set_error(a.err, PKV_DEVERR_CONTEXT_LEN);
     return;
   }
-  if (i0 >= n_new) return;  // uniform over the CTA, before any set-up
+  const int base_row = static_cast<int>(gridDim.y - 1 - blockIdx.y) * rows_per_cta;
+  if (base_row >= n_new) return;  // uniform over the CTA, before any set-up
   int L = __ldg(a.lens + s);
-  if (L < n_new || L > cap) {  // the context must hold the chunk and fit the table: clamped
+  if (L < n_new || L > cap) {
     if (threadIdx.x == 0) set_error(a.err, PKV_DEVERR_CONTEXT_LEN);
     L = L < n_new ? n_new : cap;
   }
   const int p0 = L - n_new;
-  const int kvh = h / (a.num_heads / a.num_kv_heads);
-  // keys this tile needs: 0 .. p0 + min(i0 + 127, T - 1)
-  const int last_key = p0 + min(i0 + kPrefillTileM - 1, n_new - 1);
-  const int n_kv = last_key / kPrefillTileN + 1;
+  int h_t[2], i0_t[2], nkv_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    h_t[t] = head_pair ? 2 * static_cast<int>(blockIdx.x) + t : static_cast<int>(blockIdx.x);
+    i0_t[t] = head_pair ? base_row : base_row + t * kPrefillTileM;
+    // key tiles this query tile needs (0 when its rows are past the chunk)
+    nkv_t[t] = i0_t[t] < n_new ? (p0 + min(i0_t[t] + kPrefillTileM - 1, n_new - 1)) / kPrefillTileN + 1 : 0;
+  }
+  const int n_kv = max(nkv_t[0], nkv_t[1]);
+  const int kvh = h_t[0] / G;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -170,11 +210,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t* v_full = k_full + kPrefillStages;
   uint64_t* k_empty = v_full + kPrefillStages;
   uint64_t* v_empty = k_empty + kPrefillStages;
-  uint64_t* s_full = v_empty + kPrefillStages;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* mma_done = o_done + 1;
+  uint64_t* s_full = v_empty + kPrefillStages;   // [2]: scores of tile t ready
+  uint64_t* p_full = s_full + 2;                 // [2]: P of tile t in tensor memory
+  uint64_t* pv_done = p_full + 2;                // [2]: O_t += P_t V done (P_t may be overwritten)
+  uint64_t* o_final = pv_done + 2;               // every product done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_TMEM);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,16 +225,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(&k_empty[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);  // one arrival per softmax warp
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 4);  // one arrival per softmax warp of the tile
+      mbar_init(&pv_done[t], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(o_done, 1);
-    mbar_init(mma_done, 1);
+    mbar_init(o_final, 1);
     fence_barrier_init();
   }
-  if (warp == 1) {  // the whole warp allocates the tensor memory
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kPrefillTmemCols)
@@ -210,7 +248,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t sQ = smem_addr(smem + Tr::OFF_Q);
   const uint32_t sK = smem_addr(smem + Tr::OFF_K);
   const uint32_t sV = smem_addr(smem + Tr::OFF_V);
-  const uint32_t sP = smem_addr(smem + Tr::OFF_P);
 
   if (warp == 0) {
     // ============================================================ loads
@@ -218,18 +255,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int32_t* row = a.tables + static_cast<int64_t>(s) * a.max_blocks;
     bool ok = true;
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(Tr::TILE));
+      mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(2 * Tr::TILE));
 #pragma unroll
-      for (int pn = 0; pn < ND; ++pn)
-        tma_load_3d(smem + Tr::OFF_Q + pn * Tr::PANEL, &maps.q, pn * 64, h, q0 + i0, q_full);
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int pn = 0; pn < ND; ++pn)
+          tma_load_3d(smem + Tr::OFF_Q + t * Tr::TILE + pn * Tr::PANEL, &maps.q, pn * 64, h_t[t],
+                      q0 + i0_t[t], q_full);
     }
     int issued_k = 0, issued_v = 0;
     for (int j = 0; j < n_kv && ok; ++j) {
       const int st = j % kPrefillStages;
       const int k_lo = j * kPrefillTileN;
-      const int k_hi = min(k_lo + kPrefillTileN, L);           // keys of the context in this tile
-      const int nb = (k_hi - k_lo + B - 1) / B;                 // blocks to load
-      const int blk = lane / ND, pn = lane % ND;                // this lane's block and panel
+      const int k_hi = min(k_lo + kPrefillTileN, L);
+      const int nb = (k_hi - k_lo + B - 1) / B;
+      const int blk = lane / ND, pn = lane % ND;
       int frame = 0;
       const bool copier = blk < nb;
       if (copier) {
@@ -241,7 +281,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       const uint32_t bytes = static_cast<uint32_t>(nb * ND * B * 128);
       const int off = pn * Tr::PANEL + blk * B * 128;
-      // K half of the stage
       if (lane == 0 && j >= kPrefillStages &&
           !mbar_wait_bounded(&k_empty[st], ((j / kPrefillStages) - 1) & 1)) {
         set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
@@ -254,7 +293,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (copier)
         tma_load_3d(smem + Tr::OFF_K + st * Tr::TILE + off, &maps.k, pn * 64, kvh * B, frame, &k_full[st]);
       ++issued_k;
-      // V half
       if (lane == 0 && j >= kPrefillStages &&
           !mbar_wait_bounded(&v_empty[st], ((j / kPrefillStages) - 1) & 1)) {
         set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
@@ -268,7 +306,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tma_load_3d(smem + Tr::OFF_V + st * Tr::TILE + off, &maps.v, pn * 64, kvh * B, frame, &v_full[st]);
       ++issued_v;
     }
-    // Leave no copy in flight: wait (bounded) for the last load into each stage.
     if (lane == 0) {
       if (!mbar_wait_bounded(q_full, 0)) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
       for (int j = max(0, issued_k - kPrefillStages); j < issued_k; ++j)
@@ -280,142 +317,144 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else if (warp == 1) {
     // ============================================================ tensor cores
+    // Order of the products: S_0(0), S_1(0); then for each key tile j:
+    // O_0 += P_0(j) V_j, S_0(j+1), O_1 += P_1(j) V_j, S_1(j+1).  P_t(j) lives in
+    // tensor memory over the first 64 columns of S_t(j), so S_t(j+1) is issued
+    // only once the product that reads P_t(j) has completed (products with
+    // different accumulators are not ordered by the hardware).  While one
+    // tile's softmax runs, the tensor cores work on the other tile.
     if (lane == 0) {
-      bool ok = mbar_wait_bounded(q_full, 0);
-      auto issue_pv = [&](int i) {  // O += P_i V_i
-        const int st = i % kPrefillStages;
-        if (!mbar_wait_bounded(p_full, i & 1) ||
-            !mbar_wait_bounded(&v_full[st], (i / kPrefillStages) & 1))
-          return false;
-        tmem_fence_after_sync();
-#pragma unroll
-        for (int k = 0; k < PV_STEPS; ++k) {
-          // A = P, K-major: keys k*16.. in panel k / 4, 32 bytes per k-step inside it
-          const uint64_t ad = umma_desc(sP + (k >> 2) * Tr::PANEL + (k & 3) * 32, 16, 1024);
-          // B = V, MN-major: 16 keys = two 8-row groups of 1024 bytes; panels of 64
-          // dims Tr::PANEL apart
-          const uint64_t bd = umma_desc(sV + st * Tr::TILE + k * 2048, Tr::PANEL, 1024);
-          umma_f16(tmem + Tr::COL_O, ad, bd, IDESC_O, i > 0 || k > 0);
-        }
-        umma_commit(o_done);
-        umma_commit(&v_empty[st]);
-        return true;
-      };
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j % kPrefillStages, b = j & 1;
-        if (!mbar_wait_bounded(&k_full[st], (j / kPrefillStages) & 1) ||
-            (j >= 2 && !mbar_wait_bounded(&s_empty[b], ((j - 2) >> 1) & 1))) {
-          ok = false;
-          break;
-        }
-        tmem_fence_after_sync();
+      bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&k_full[0], 0);
+      auto issue_s = [&](int t, int st) {  // S_t = Q_t K^T of the key tile in stage st
 #pragma unroll
         for (int k = 0; k < KSTEPS; ++k) {
           const uint32_t koff = (k >> 2) * Tr::PANEL + (k & 3) * 32;
-          umma_f16(tmem + Tr::COL_S + b * kPrefillTileN, umma_desc(sQ + koff, 16, 1024),
+          umma_f16(tmem + Tr::colS(t), umma_desc(sQ + t * Tr::TILE + koff, 16, 1024),
                    umma_desc(sK + st * Tr::TILE + koff, 16, 1024), IDESC_S, k > 0);
         }
-        umma_commit(&s_full[b]);
-        umma_commit(&k_empty[st]);
-        if (j >= 1 && !issue_pv(j - 1)) ok = false;
+        umma_commit(&s_full[t]);
+      };
+      if (ok) {
+        tmem_fence_after_sync();
+        for (int t = 0; t < 2; ++t)
+          if (nkv_t[t] > 0) issue_s(t, 0);
+        umma_commit(&k_empty[0]);
       }
-      if (ok && !issue_pv(n_kv - 1)) ok = false;
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int st = j % kPrefillStages, st1 = (j + 1) % kPrefillStages;
+        const bool more = j + 1 < n_kv;
+        if (!mbar_wait_bounded(&v_full[st], (j / kPrefillStages) & 1) ||
+            (more && !mbar_wait_bounded(&k_full[st1], ((j + 1) / kPrefillStages) & 1))) {
+          ok = false;
+          break;
+        }
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= nkv_t[t]) continue;
+          if (!mbar_wait_bounded(&p_full[t], j & 1)) {
+            ok = false;
+            break;
+          }
+          tmem_fence_after_sync();
+#pragma unroll
+          for (int k = 0; k < PV_STEPS; ++k)
+            umma_f16_ts(tmem + Tr::colO(t), tmem + Tr::colS(t) + k * 8,
+                        umma_desc(sV + st * Tr::TILE + k * 2048, Tr::PANEL, 1024), IDESC_O,
+                        j > 0 || k > 0);
+          umma_commit(&pv_done[t]);
+          if (j + 1 < nkv_t[t]) {
+            if (!mbar_wait_bounded(&pv_done[t], j & 1)) {
+              ok = false;
+              break;
+            }
+            tmem_fence_after_sync();
+            issue_s(t, st1);
+          }
+        }
+        umma_commit(&v_empty[st]);
+        if (more) umma_commit(&k_empty[st1]);
+      }
       if (!ok) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
-      // every issued tensor-core operation has finished before the CTA frees
-      // the tensor memory or its shared memory
-      umma_commit(mma_done);
-      if (!mbar_wait_bounded(mma_done, 0)) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+      // o_final: every product issued above (all of them on the normal path)
+      // has finished; the softmax warps read O after it, and the CTA frees the
+      // tensor and shared memory only after it.
+      umma_commit(o_final);
     }
     __syncwarp();
   } else {
     // ============================================================ softmax rows
+    const int t = (warp - 2) >> 2;                // query tile of this warp group
     const int quarter = warp & 3;                 // tensor-memory lanes 32 quarter ..
-    const int r = quarter * 32 + lane;            // this thread's query row
-    const int i = i0 + r;                         // its token index in the chunk
+    const int r = quarter * 32 + lane;            // this thread's query row of the tile
+    const int i = i0_t[t] + r;                    // its token index in the chunk
     const bool valid = i < n_new;
     const int limit = valid ? p0 + i : L - 1;     // last key this row may see
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t cS = lane_base + Tr::colS(t), cO = lane_base + Tr::colO(t);
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int b = j & 1;
+    for (int j = 0; j < nkv_t[t]; ++j) {
       const int k_lo = j * kPrefillTileN;
-      ok = ok && mbar_wait_bounded(&s_full[b], (j >> 1) & 1);
+      ok = ok && mbar_wait_bounded(&s_full[t], j & 1);
       if (!__all_sync(0xffffffffu, ok)) break;
       tmem_fence_after_sync();
-      float x[kPrefillTileN];
+      const bool full = k_lo + kPrefillTileN - 1 <= limit;
+      // pass 1: the row max (keys past the limit are -inf, by select)
+      float mx = -CUDART_INF_F;
 #pragma unroll
       for (int c = 0; c < kPrefillTileN / 32; ++c) {
         float v[32];
-        tmem_ld32(lane_base + Tr::COL_S + b * kPrefillTileN + c * 32, v);
+        tmem_ld32(cS + c * 32, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[c * 32 + e] = v[e];
+        for (int e = 0; e < 32; ++e)
+          if (full || k_lo + c * 32 + e <= limit) mx = fmaxf(mx, v[e]);
       }
-      tmem_wait_ld();
-      tmem_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[b]);
-      // scale to base-2 units; keys past this row's limit become -inf (select)
-      float mx = -CUDART_INF_F;
-      if (k_lo + kPrefillTileN - 1 <= limit) {
-#pragma unroll
-        for (int t = 0; t < kPrefillTileN; ++t) {
-          x[t] *= a.scale_log2;
-          mx = fmaxf(mx, x[t]);
-        }
-      } else {
-#pragma unroll
-        for (int t = 0; t < kPrefillTileN; ++t) {
-          x[t] = k_lo + t <= limit ? x[t] * a.scale_log2 : -CUDART_INF_F;
-          mx = fmaxf(mx, x[t]);
-        }
-      }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = m == -CUDART_INF_F ? 0.f : (m_new == m ? 1.f : fast_exp2(m - m_new));
-      // P row, rounded to the input type; the sum is over the rounded weights
-      uint32_t pk[kPrefillTileN / 2];
-      float sum = 0.f;
-#pragma unroll
-      for (int t = 0; t < kPrefillTileN; t += 2) {
-        const float e0 = x[t] == -CUDART_INF_F ? 0.f : fast_exp2(x[t] - m_new);
-        const float e1 = x[t + 1] == -CUDART_INF_F ? 0.f : fast_exp2(x[t + 1] - m_new);
-        pk[t / 2] = pack2<T>(e0, e1);
-        const float2 rounded = unpack2<T>(pk[t / 2]);
-        sum += rounded.x + rounded.y;
-      }
-      l = l * alpha + sum;
-      // the previous product has finished reading P and writing O
-      if (j >= 1) ok = ok && mbar_wait_bounded(o_done, (j - 1) & 1);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tmem_fence_after_sync();
-      // Rescale the rows of O whose max grew.  tcgen05.ld / st are warp-wide
-      // (.sync.aligned): the whole warp takes the branch when any of its rows
-      // needs it, and rows whose max did not grow multiply by alpha = 1 exactly.
-      if (j >= 1 && __any_sync(0xffffffffu, m_new > m)) {
+      const float m_new = fmaxf(m, mx * a.scale_log2);
+      // The product of the previous tile ran before S_t(j): O_t is final for it.
+      // tcgen05.ld / st are warp-wide (.sync.aligned): the whole warp rescales
+      // when any of its rows' max grew; the others multiply by alpha = 1 exactly.
+      if (j > 0 && __any_sync(0xffffffffu, m_new > m)) {
+        const float alpha = m_new == m ? 1.f : fast_exp2(m - m_new);
+        l *= alpha;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float v[32];
-          tmem_ld32(lane_base + Tr::COL_O + c * 32, v);
+          tmem_ld32(cO + c * 32, v);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= alpha;
-          tmem_st32(lane_base + Tr::COL_O + c * 32, v);
+          tmem_st32(cO + c * 32, v);
         }
-        tmem_wait_st();
       }
       m = m_new;
-      // P row r into the K-major, 128-byte swizzled P tile: keys 64 pn .. in
-      // panel pn, 16-byte chunk c of the row at chunk c ^ (r % 8)
-      uint8_t* prow = smem + Tr::OFF_P + r * 128;
+      // pass 2: P = 2^(x - m) rounded to the input type, packed two keys per
+      // column over the first 64 columns of S (a chunk's P columns precede
+      // the scores read after it); the sum is over the rounded weights
+      float sum = 0.f;
 #pragma unroll
-      for (int c = 0; c < kPrefillTileN / 8; ++c) {
-        const int pn = c >> 3, ch = (c & 7) ^ (r & 7);
-        *reinterpret_cast<uint4*>(prow + pn * Tr::PANEL + ch * 16) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      for (int c = 0; c < kPrefillTileN / 32; ++c) {
+        float v[32];
+        tmem_ld32(cS + c * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int kk = k_lo + c * 32 + e;
+          const float e0 = (full || kk <= limit) ? fast_exp2(v[e] * a.scale_log2 - m) : 0.f;
+          const float e1 = (full || kk + 1 <= limit) ? fast_exp2(v[e + 1] * a.scale_log2 - m) : 0.f;
+          pk[e / 2] = pack2<T>(e0, e1);
+          const float2 rd = unpack2<T>(pk[e / 2]);
+          sum += rd.x + rd.y;
+        }
+        tmem_st16(cS + c * 16, pk);
       }
-      // The tile that reaches past the context: zero the V rows of the keys
-      // past it (whatever the stage held there, 0 x it must be 0).
-      if (k_lo + kPrefillTileN > L) {
+      l += sum;
+      tmem_wait_st();
+      // The key tile that reaches past the context: zero the V rows of the keys
+      // past it (whatever the stage held there, 0 x it must be 0).  The first
+      // tile whose product reads this key tile does it (tile 0, unless its rows
+      // end before this key tile).
+      if ((t == 0 || j >= nkv_t[0]) && k_lo + kPrefillTileN > L) {
         const int st = j % kPrefillStages;
         ok = ok && mbar_wait_bounded(&v_full[st], (j / kPrefillStages) & 1);
         if (ok && k_lo + r >= L) {
@@ -426,29 +465,31 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             for (int ch = 0; ch < 8; ++ch)
               *reinterpret_cast<uint4*>(vrow + pn * Tr::PANEL + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();  // generic writes of P (and V) before the tensor cores read them
       tmem_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
     // ---- epilogue: out = O / l
-    ok = ok && mbar_wait_bounded(o_done, (n_kv - 1) & 1);
+    ok = ok && (nkv_t[t] == 0 || mbar_wait_bounded(o_final, 0));
     if (__all_sync(0xffffffffu, ok)) {
-      tmem_fence_after_sync();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      T* orow = static_cast<T*>(a.out) + (static_cast<int64_t>(q0 + i) * a.num_heads + h) * D;
+      if (nkv_t[t] > 0) {
+        tmem_fence_after_sync();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        T* orow = static_cast<T*>(a.out) + (static_cast<int64_t>(q0 + i) * a.num_heads + h_t[t]) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float v[32];
-        tmem_ld32(lane_base + Tr::COL_O + c * 32, v);
-        tmem_wait_ld();
-        if (valid) {
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(cO + c * 32, v);
+          tmem_wait_ld();
+          if (valid) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            const uint4 w = make_uint4(pack2<T>(v[e] * inv, v[e + 1] * inv), pack2<T>(v[e + 2] * inv, v[e + 3] * inv),
-                                       pack2<T>(v[e + 4] * inv, v[e + 5] * inv), pack2<T>(v[e + 6] * inv, v[e + 7] * inv));
-            *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
+            for (int e = 0; e < 32; e += 8) {
+              const uint4 w = make_uint4(pack2<T>(v[e] * inv, v[e + 1] * inv), pack2<T>(v[e + 2] * inv, v[e + 3] * inv),
+                                         pack2<T>(v[e + 4] * inv, v[e + 5] * inv), pack2<T>(v[e + 6] * inv, v[e + 7] * inv));
+              *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
+            }
           }
         }
       }
@@ -456,6 +497,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
     }
   }
+  // Nothing of the tensor cores or the copies is in flight past here: the MMA
+  // thread's final commit covers every product, and it is waited for below
+  // before the tensor memory is freed.
+  if (warp == 1 && lane == 0 && !mbar_wait_bounded(o_final, 0)) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
   tmem_fence_before_sync();
   __syncthreads();
   if (warp == 1) {
@@ -473,8 +518,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, const PrefillMaps& m, int max_q
   auto kern = prefill_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(a.num_heads),
-                  static_cast<unsigned>((max_query_len + kPrefillTileM - 1) / kPrefillTileM),
+  const bool head_pair = ((a.num_heads / a.num_kv_heads) & 1) == 0;
+  const int rows = head_pair ? kPrefillTileM : 2 * kPrefillTileM;
+  const dim3 grid(static_cast<unsigned>(head_pair ? a.num_heads / 2 : a.num_heads),
+                  static_cast<unsigned>((max_query_len + rows - 1) / rows),
                   static_cast<unsigned>(a.num_seqs));
   kern<<<grid, kPrefillThreads, Tr::SMEM_BYTES, stream>>>(a, m);
   return cudaGetLastError();

@@ -33,7 +33,7 @@ struct PrefillMaps {
   CUtensorMap q, k, v;
 };
 
-constexpr int kPrefillThreads = 192;
+constexpr int kPrefillThreads = 320;  // TMA, MMA, 2 x 4 softmax warps
 constexpr int kPrefillTileM = 128;  // query rows per CTA
 constexpr int kPrefillTileN = 128;  // keys per tile
 constexpr int kPrefillStages = 2;
@@ -44,30 +44,30 @@ struct PrefillTraits {
   static constexpr int ND = D / 64;                       // 128-byte panels per row
   static constexpr int PANEL = kPrefillTileM * 128;       // one panel of 128 rows
   static constexpr int TILE = ND * PANEL;                 // Q, K or V tile
-  static constexpr int P_TILE = 2 * PANEL;                // P: 128 rows x 128 keys
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE;
+  static constexpr int OFF_Q = 0;                         // two query tiles
+  static constexpr int OFF_K = OFF_Q + 2 * TILE;
   static constexpr int OFF_V = OFF_K + kPrefillStages * TILE;
-  static constexpr int OFF_P = OFF_V + kPrefillStages * TILE;
-  static constexpr int OFF_BAR = OFF_P + P_TILE;
-  // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], s_empty[2], p_full, o_done, mma_done
-  static constexpr int NUM_BARS = 1 + 4 * kPrefillStages + 4 + 3;
+  static constexpr int OFF_BAR = OFF_V + kPrefillStages * TILE;
+  // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], p_full[2], pv_done[2], o_final
+  static constexpr int NUM_BARS = 1 + 4 * kPrefillStages + 6 + 1;
   static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_TMEM + 16;
   // SMEM_USED + 1024 bytes of slack for the 1024-byte aligned base, and never
   // less than 117 KB: two CTAs never share an SM, so the second never waits in
   // tcgen05.alloc for the first one's 512 tensor-memory columns.
   static constexpr int SMEM_BYTES = SMEM_USED + 1024 > 117 * 1024 ? SMEM_USED + 1024 : 117 * 1024;
-  // tensor memory columns
-  static constexpr uint32_t COL_S = 0;     // two score buffers of 128 columns
-  static constexpr uint32_t COL_O = 256;   // the output accumulator, D columns
+  // tensor memory: query tile t has its scores at colS(t) (128 columns; its P
+  // over the first 64 of them) and its output accumulator at colO(t) (D columns)
+  static constexpr uint32_t colS(int t) { return 256u * static_cast<uint32_t>(t); }
+  static constexpr uint32_t colO(int t) { return 256u * static_cast<uint32_t>(t) + 128u; }
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
 // Launch of the prefill grid (instantiated in prefill.cu for fp16 / bf16 and
-// head_dim 64 / 128): (query heads) x (query tiles of the longest chunk) x
-// (sequences) CTAs.
+// head_dim 64 / 128): per sequence, one CTA per pair of 128-row query tiles
+// (two heads of a kv group on the same rows when Hq / Hkv is even, else two
+// consecutive row tiles of one head).
 template <typename T, int D>
 cudaError_t launch_prefill(const PrefillArgs& a, const PrefillMaps& m, int max_query_len,
                            cudaStream_t stream);

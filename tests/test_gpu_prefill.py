@@ -16,7 +16,7 @@ import torch
 import oracle
 from oracle.allocator_model import AllocatorModel
 import workloads as wl
-from flow import TOL, POISON, to_dev, from_dev, torch_dtype, rounded_oracle_stats
+from flow import TOL, POISON, to_dev, from_dev, torch_dtype, rounded_oracle_stats, stored_tolerance
 
 pytestmark = pytest.mark.gpu
 
@@ -101,6 +101,17 @@ def max_err(out, ref, rows=None):
     return float(np.abs(g - ref).max())
 
 
+def assert_within_tolerance(out, ref, dtype, rows=None):
+    """Every element within the tolerance, or within half an ulp of the exact
+    value in the output type where that is larger (stored_tolerance)."""
+    g = out.double().cpu().numpy()
+    if rows is not None:
+        g, ref = g[rows], ref[rows]
+    bound = stored_tolerance(ref, dtype)
+    worst = float((np.abs(g - ref) - bound).max())
+    assert worst <= 0.0, (worst, float(np.abs(g - ref).max()))
+
+
 # Cached prefixes of 0 (a whole prompt), a few tokens and several tiles; chunks
 # of 1 token, across tile and block boundaries, and several query tiles.
 CACHED = [0, 5, 40, 300, 129]
@@ -122,7 +133,7 @@ def test_prefill_matches_oracle(dtype, D, G, bs):
     assert np.array_equal(tables, table)
     assert torch.isfinite(out).all()
     err = max_err(out, ref)
-    assert err <= TOL[dtype], err
+    assert_within_tolerance(out, ref, dtype)
     if dtype == wl.BF16 and D == 128 and G == 4 and bs == 16:
         print(f"prefill vs rounded oracle: {rounded_oracle_stats(out, ref, dtype)}, max-abs {err:.3e}")
 
@@ -206,7 +217,8 @@ def test_prefill_last_token_agrees_with_decode():
     B.paged_attention_decode(dec, q_last, kc, vc, torch.from_numpy(table).cuda(),
                              torch.from_numpy(lens).cuda(), w.scale)
     torch.cuda.synchronize()
-    assert (dec.double() - out[last].double()).abs().max().item() <= TOL[wl.BF16]
+    # both within the tolerance of the exact value: within twice it of each other
+    assert (dec.double() - out[last].double()).abs().max().item() <= 2 * TOL[wl.BF16]
 
 
 def test_prefill_bad_lengths_set_flags_without_faulting():
@@ -248,5 +260,4 @@ def test_prefill_full_size_batch_sampled_rows():
                          set(rng.choice(T, size=20, replace=False).tolist()))
     ref, _ = oracle_prefill_batch(inp, rows=rows)
     idx = np.concatenate([inp.query_start[s] + np.array(r) for s, r in rows.items()])
-    err = max_err(out, ref, idx)
-    assert err <= TOL[wl.BF16], err
+    assert_within_tolerance(out, ref, wl.BF16, idx)

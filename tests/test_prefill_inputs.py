@@ -30,3 +30,15 @@ def test_prefill_flops_count_every_causal_pair_once():
             pairs += len(range(0, int(p0) + i + 1))  # keys 0 .. p0 + i
     # q.K and P.V: one multiply-add (2 flops) per head dimension each, per query head
     assert bench.prefill_flops(inp) == pairs * 2 * 2 * w.head_dim * w.num_heads
+
+
+def test_stored_tolerance_is_half_an_ulp_above_the_absolute_bound():
+    from flow import stored_tolerance, TOL
+
+    ref = np.array([0.0, 0.3, 2.5, 3.99, 4.0, 5.0, -6.0, 100.0])
+    got = stored_tolerance(ref, wl.BF16)
+    # bf16 spacing is 2^(e-7) in [2^e, 2^(e+1)); half of it from magnitude 4 up
+    assert np.allclose(got, [TOL[wl.BF16]] * 4 + [2.0 ** -6, 2.0 ** -6, 2.0 ** -6, 2.0 ** -2])
+    # fp16 spacing is 2^(e-10): half of it passes 2e-3 from magnitude 8 up
+    assert np.allclose(stored_tolerance(np.array([1.0, 4.0, 8.0, 64.0]), wl.F16),
+                       [TOL[wl.F16], TOL[wl.F16], 2.0 ** -8, 2.0 ** -5])
