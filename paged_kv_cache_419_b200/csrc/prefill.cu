@@ -155,6 +155,10 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Lag of a row's reference max behind its true running max (base-2 units)
+// before the output row is rescaled: weights stay below 2^8.
+constexpr float kLazy = 8.f;
+
 // ------------------------------------------------------------ kernel
 // Query tile t in {0, 1} of a CTA: head h_t, rows i0_t .. i0_t + 127 of the
 // chunk.  Two heads of one kv group share the rows when Hq / Hkv is even (the
@@ -317,12 +321,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
   } else if (warp == 1) {
     // ============================================================ tensor cores
-    // Order of the products: S_0(0), S_1(0); then for each key tile j:
-    // O_0 += P_0(j) V_j, S_0(j+1), O_1 += P_1(j) V_j, S_1(j+1).  P_t(j) lives in
+    // Two chains of products, one per query tile t: S_t(j) = Q_t K_j^T, the
+    // softmax of tile t, O_t += P_t(j) V_j, then S_t(j+1).  P_t(j) lives in
     // tensor memory over the first 64 columns of S_t(j), so S_t(j+1) is issued
-    // only once the product that reads P_t(j) has completed (products with
-    // different accumulators are not ordered by the hardware).  While one
-    // tile's softmax runs, the tensor cores work on the other tile.
+    // only once the product that reads P_t(j) has completed (the hardware orders
+    // a thread's products into the same accumulator, not these).  The issuing
+    // thread polls both chains without blocking and issues whichever step is
+    // ready, so while one chain waits (for its softmax, or for its product to
+    // complete) the tensor cores work on the other one.  A K (V) stage is
+    // released once every chain that uses it has issued its scores (product).
     if (lane == 0) {
       bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&k_full[0], 0);
       auto issue_s = [&](int t, int st) {  // S_t = Q_t K^T of the key tile in stage st
@@ -334,44 +341,69 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         umma_commit(&s_full[t]);
       };
+      auto users = [&](int j) { return (nkv_t[0] > j ? 1 : 0) + (nkv_t[1] > j ? 1 : 0); };
       if (ok) {
         tmem_fence_after_sync();
         for (int t = 0; t < 2; ++t)
           if (nkv_t[t] > 0) issue_s(t, 0);
         umma_commit(&k_empty[0]);
       }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j % kPrefillStages, st1 = (j + 1) % kPrefillStages;
-        const bool more = j + 1 < n_kv;
-        if (!mbar_wait_bounded(&v_full[st], (j / kPrefillStages) & 1) ||
-            (more && !mbar_wait_bounded(&k_full[st1], ((j + 1) / kPrefillStages) & 1))) {
-          ok = false;
-          break;
-        }
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= nkv_t[t]) continue;
-          if (!mbar_wait_bounded(&p_full[t], j & 1)) {
-            ok = false;
-            break;
-          }
-          tmem_fence_after_sync();
+      int jt[2] = {0, 0};          // key tile of chain t's next product
+      bool want_s[2] = {false, false};  // chain t's next step is S_t(jt + 1)
+      int s_cnt[kPrefillStages] = {0, 0}, v_cnt[kPrefillStages] = {0, 0};
+      unsigned long long last = global_timer_ns();
+      int idle = 0;
+      while (ok) {
+        bool busy = false, progressed = false;
 #pragma unroll
-          for (int k = 0; k < PV_STEPS; ++k)
-            umma_f16_ts(tmem + Tr::colO(t), tmem + Tr::colS(t) + k * 8,
-                        umma_desc(sV + st * Tr::TILE + k * 2048, Tr::PANEL, 1024), IDESC_O,
-                        j > 0 || k > 0);
-          umma_commit(&pv_done[t]);
-          if (j + 1 < nkv_t[t]) {
-            if (!mbar_wait_bounded(&pv_done[t], j & 1)) {
-              ok = false;
-              break;
+        for (int t = 0; t < 2; ++t) {
+          const int j = jt[t];
+          if (j >= nkv_t[t]) continue;
+          busy = true;
+          if (!want_s[t]) {  // O_t += P_t(j) V_j once P_t(j) and V_j are there
+            const int st = j % kPrefillStages;
+            if (!mbar_try_wait(&p_full[t], j & 1) ||
+                !mbar_try_wait(&v_full[st], (j / kPrefillStages) & 1))
+              continue;
+            tmem_fence_after_sync();
+#pragma unroll
+            for (int k = 0; k < PV_STEPS; ++k)
+              umma_f16_ts(tmem + Tr::colO(t), tmem + Tr::colS(t) + k * 8,
+                          umma_desc(sV + st * Tr::TILE + k * 2048, Tr::PANEL, 1024), IDESC_O,
+                          j > 0 || k > 0);
+            umma_commit(&pv_done[t]);
+            if (++v_cnt[st] == users(j)) {
+              umma_commit(&v_empty[st]);
+              v_cnt[st] = 0;
             }
+            if (j + 1 < nkv_t[t])
+              want_s[t] = true;
+            else
+              jt[t] = nkv_t[t];  // chain t is done
+          } else {  // S_t(j+1) once the product reading P_t(j) is done and K_{j+1} is there
+            const int st1 = (j + 1) % kPrefillStages;
+            if (!mbar_try_wait(&pv_done[t], j & 1) ||
+                !mbar_try_wait(&k_full[st1], ((j + 1) / kPrefillStages) & 1))
+              continue;
             tmem_fence_after_sync();
             issue_s(t, st1);
+            if (++s_cnt[st1] == users(j + 1)) {
+              umma_commit(&k_empty[st1]);
+              s_cnt[st1] = 0;
+            }
+            want_s[t] = false;
+            jt[t] = j + 1;
           }
+          progressed = true;
         }
-        umma_commit(&v_empty[st]);
-        if (more) umma_commit(&k_empty[st1]);
+        if (!busy) break;
+        if (progressed) {
+          idle = 0;
+          last = global_timer_ns();
+        } else if (++idle >= 64) {  // bounded: no chain has moved for kWaitLimitNs
+          idle = 0;
+          if (global_timer_ns() - last > kWaitLimitNs) ok = false;
+        }
       }
       if (!ok) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
       // o_final: every product issued above (all of them on the normal path)
@@ -390,6 +422,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int limit = valid ? p0 + i : L - 1;     // last key this row may see
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t cS = lane_base + Tr::colS(t), cO = lane_base + Tr::colO(t);
+    // Running state of the row, in base-2 units: m is the max the weights are
+    // taken against (at most kLazy below the true running max, see below) and
+    // l the sum of the rounded weights.
+    const float sl = a.scale_log2;
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv_t[t]; ++j) {
@@ -397,24 +433,48 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       ok = ok && mbar_wait_bounded(&s_full[t], j & 1);
       if (!__all_sync(0xffffffffu, ok)) break;
       tmem_fence_after_sync();
-      const bool full = k_lo + kPrefillTileN - 1 <= limit;
-      // pass 1: the row max (keys past the limit are -inf, by select)
-      float mx = -CUDART_INF_F;
+      // Pass 1: the row's 128 scores, all requested before one wait, and their
+      // max in base-2 units.  Keys past this row's limit count as -inf (by
+      // select); only tiles on the diagonal (or past the context) need that,
+      // and a warp takes the masked path only when one of its rows needs it.
+      const bool masked = __any_sync(0xffffffffu, k_lo + kPrefillTileN - 1 > limit);
+      float mx;
+      {
+        float x[kPrefillTileN];
 #pragma unroll
-      for (int c = 0; c < kPrefillTileN / 32; ++c) {
-        float v[32];
-        tmem_ld32(cS + c * 32, v);
+        for (int c = 0; c < kPrefillTileN / 32; ++c) {
+          float v[32];
+          tmem_ld32(cS + c * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[c * 32 + e] = v[e];
+        }
         tmem_wait_ld();
+        if (masked) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (full || k_lo + c * 32 + e <= limit) mx = fmaxf(mx, v[e]);
+          for (int e = 0; e < kPrefillTileN; ++e) x[e] = k_lo + e <= limit ? x[e] * sl : -CUDART_INF_F;
+        } else {
+#pragma unroll
+          for (int e = 0; e < kPrefillTileN; ++e) x[e] *= sl;
+        }
+        float mx4[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+        for (int e = 4; e < kPrefillTileN; e += 4) {
+          mx4[0] = fmaxf(mx4[0], x[e]);
+          mx4[1] = fmaxf(mx4[1], x[e + 1]);
+          mx4[2] = fmaxf(mx4[2], x[e + 2]);
+          mx4[3] = fmaxf(mx4[3], x[e + 3]);
+        }
+        mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       }
-      const float m_new = fmaxf(m, mx * a.scale_log2);
-      // The product of the previous tile ran before S_t(j): O_t is final for it.
-      // tcgen05.ld / st are warp-wide (.sync.aligned): the whole warp rescales
-      // when any of its rows' max grew; the others multiply by alpha = 1 exactly.
-      if (j > 0 && __any_sync(0xffffffffu, m_new > m)) {
-        const float alpha = m_new == m ? 1.f : fast_exp2(m - m_new);
+      // Lazy rescale: the weights are 2^(x - m) with m allowed to lag the true
+      // running max by up to kLazy (weights up to 2^kLazy, exact in the input
+      // type's range and in fp32), so O and l are rescaled only when the max
+      // outgrows that.  The product of the previous key tile ran before S_t(j),
+      // so O_t holds it.  tcgen05.ld / st are warp-wide (.sync.aligned): the
+      // whole warp takes the branch, rows that need no rescale multiply by 1.
+      const bool grow = mx > m + kLazy;
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        const float alpha = grow ? fast_exp2(m - mx) : 1.f;
         l *= alpha;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -426,35 +486,56 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_st32(cO + c * 32, v);
         }
       }
-      m = m_new;
-      // pass 2: P = 2^(x - m) rounded to the input type, packed two keys per
-      // column over the first 64 columns of S (a chunk's P columns precede
-      // the scores read after it); the sum is over the rounded weights
-      float sum = 0.f;
+      if (grow) m = mx;
+      // Pass 2, in two halves of 64 scores (two loads, one wait each): P =
+      // 2^(x - m) rounded to the input type, two keys per 32-bit column, over
+      // the first 64 columns of S (the columns a half writes were read by the
+      // halves before it); the sum is over the rounded weights, in four
+      // independent partial sums.
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kPrefillTileN / 32; ++c) {
-        float v[32];
-        tmem_ld32(cS + c * 32, v);
-        tmem_wait_ld();
-        uint32_t pk[16];
+      for (int hh = 0; hh < 2; ++hh) {
+        float x[64];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int kk = k_lo + c * 32 + e;
-          const float e0 = (full || kk <= limit) ? fast_exp2(v[e] * a.scale_log2 - m) : 0.f;
-          const float e1 = (full || kk + 1 <= limit) ? fast_exp2(v[e + 1] * a.scale_log2 - m) : 0.f;
-          pk[e / 2] = pack2<T>(e0, e1);
-          const float2 rd = unpack2<T>(pk[e / 2]);
-          sum += rd.x + rd.y;
+        for (int c = 0; c < 2; ++c) {
+          float v[32];
+          tmem_ld32(cS + hh * 64 + c * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[c * 32 + e] = v[e];
         }
-        tmem_st16(cS + c * 16, pk);
+        tmem_wait_ld();
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          const int kk = k_lo + hh * 64 + e;
+          float p0v, p1v;
+          if (masked) {
+            p0v = kk <= limit ? fast_exp2(x[e] * sl - m) : 0.f;
+            p1v = kk + 1 <= limit ? fast_exp2(x[e + 1] * sl - m) : 0.f;
+          } else {
+            p0v = fast_exp2(x[e] * sl - m);
+            p1v = fast_exp2(x[e + 1] * sl - m);
+          }
+          pk[e / 2] = pack2<T>(p0v, p1v);
+          const float2 rd = unpack2<T>(pk[e / 2]);
+          sum4[(e >> 1) & 3] += rd.x + rd.y;
+        }
+        uint32_t lo[16], hi[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          lo[e] = pk[e];
+          hi[e] = pk[16 + e];
+        }
+        tmem_st16(cS + hh * 32, lo);
+        tmem_st16(cS + hh * 32 + 16, hi);
       }
-      l += sum;
+      l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       tmem_wait_st();
       // The key tile that reaches past the context: zero the V rows of the keys
-      // past it (whatever the stage held there, 0 x it must be 0).  The first
-      // tile whose product reads this key tile does it (tile 0, unless its rows
-      // end before this key tile).
-      if ((t == 0 || j >= nkv_t[0]) && k_lo + kPrefillTileN > L) {
+      // past it (whatever the stage held there, 0 x it must be 0).  Each chain
+      // does it before its own product (the two products may run in either
+      // order); the second chain writes zeros over zeros.
+      if (k_lo + kPrefillTileN > L) {
         const int st = j % kPrefillStages;
         ok = ok && mbar_wait_bounded(&v_full[st], (j / kPrefillStages) & 1);
         if (ok && k_lo + r >= L) {
