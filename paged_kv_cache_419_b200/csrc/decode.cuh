@@ -157,6 +157,17 @@ __device__ __forceinline__ void partition_for(int L, const DecodeArgs& a, unsign
     partition_of(L, a.part_tokens, n, size);
 }
 
+// Round-robin schedule: under the balanced policy the items are near-equal by
+// construction, so no largest-first list is needed.  With at most
+// kRoundRobinSeqs sequences (two per lane of a warp), each decode CTA c takes
+// items c, c + grid, c + 2 grid, ... of the enumeration (sequence, partition,
+// kv head), kv head fastest, which it computes from the context lengths alone:
+// no CTA waits for the planning kernel's list.
+constexpr int kRoundRobinSeqs = 64;
+__device__ __forceinline__ bool round_robin(const DecodeArgs& a) {
+  return a.balanced && a.num_seqs <= kRoundRobinSeqs;
+}
+
 // Sequences whose partition 0 runs as a static first item: decode CTA c
 // (c < this * Hkv) starts with partition 0 of sequence c / Hkv, kv head c % Hkv,
 // computed from the inputs alone, so it does not wait for the plan; the plan
@@ -310,6 +321,14 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
     }
   }
   __syncthreads();
+  if (round_robin(a)) {  // every item is taken statically: no list to write
+    if (threadIdx.x == 0) {
+      a.work[0] = 0u;
+      a.work[1] = 0u;
+      a.work[2] = n_multi;
+    }
+    return;
+  }
   if (threadIdx.x < 32) {  // exclusive scan of the class counts, one warp
     const int lane = threadIdx.x;
     constexpr int kPerLane = (kMaxClasses + 31) / 32;
@@ -472,7 +491,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
       if (!plan_done) {
         grid_dependency_wait();
         allow_dependent_launch();
-        n_items = *reinterpret_cast<volatile uint32_t*>(a.work + 1);
+        if (!round_robin(a)) n_items = *reinterpret_cast<volatile uint32_t*>(a.work + 1);
         plan_done = true;
       }
     };
@@ -526,10 +545,87 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
     };
 
     bool ok = true;
+    const bool rr = round_robin(a);
+    // Round-robin schedule (see round_robin): lane l describes sequences l and
+    // l + 32: length, partitions, partition size and the index of its first
+    // (sequence, partition) pair in the enumeration.
+    int rr_L[2] = {0, 0}, rr_n[2] = {0, 0}, rr_size[2] = {0, 0}, rr_first[2] = {0, 0};
+    auto rr_record = [&](uint32_t j, uint32_t idx) {  // whole warp; record of item idx -> slot j % 2
+      const int pair = static_cast<int>(idx / Hkv);
+      int own = -1;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        if (pair >= rr_first[h] && pair < rr_first[h] + rr_n[h]) own = h;
+      const uint32_t mask = __ballot_sync(0xffffffffu, own >= 0);
+      const int src = __ffs(mask) - 1;  // exactly one lane owns the pair
+      const int h = __shfl_sync(0xffffffffu, own, src);
+      const int L = __shfl_sync(0xffffffffu, h ? rr_L[1] : rr_L[0], src);
+      const int n = __shfl_sync(0xffffffffu, h ? rr_n[1] : rr_n[0], src);
+      const int size = __shfl_sync(0xffffffffu, h ? rr_size[1] : rr_size[0], src);
+      const int first = __shfl_sync(0xffffffffu, h ? rr_first[1] : rr_first[0], src);
+      if (lane == 0) {
+        int32_t* r = reinterpret_cast<int32_t*>(smem + Tr::OFF_REC + (j & 1) * kRecordBytes);
+        const int p = pair - first, t_begin = p * size;
+        r[0] = src + 32 * h;
+        r[1] = p;
+        r[2] = n;
+        r[3] = t_begin;
+        r[4] = min(size, L - t_begin);
+        r[5] = L;
+        // complete the slot's barrier phase as a copy would have
+        mbar_arrive(&rec_bar[j & 1]);
+      }
+      __syncwarp();
+    };
+    if (rr) {
+      unsigned long long U = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = lane + 32 * h;
+        rr_L[h] = t < a.num_seqs ? clamp_len(a.lens[t], a.max_ctx) : 0;
+        U += static_cast<unsigned long long>(rr_L[h]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) U += __shfl_xor_sync(0xffffffffu, U, o);
+      U *= static_cast<unsigned long long>(a.num_kv_heads);
+      int n_lane[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = lane + 32 * h;
+        partition_for(rr_L[h], a, U, rr_n[h], rr_size[h]);
+        n_lane[h] = t < a.num_seqs ? rr_n[h] : 0;
+      }
+      // exclusive prefix of the partition counts in sequence order
+      // (sequences 0..31 on lanes 0..31, then 32..63)
+      int incl0 = n_lane[0], incl1 = n_lane[1];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int a0 = __shfl_up_sync(0xffffffffu, incl0, o);
+        const int a1 = __shfl_up_sync(0xffffffffu, incl1, o);
+        if (lane >= o) {
+          incl0 += a0;
+          incl1 += a1;
+        }
+      }
+      const int total0 = __shfl_sync(0xffffffffu, incl0, 31);
+      rr_first[0] = incl0 - n_lane[0];
+      rr_first[1] = total0 + incl1 - n_lane[1];
+      rr_n[0] = n_lane[0];  // 0 past the last sequence: no pair maps there
+      rr_n[1] = n_lane[1];
+      n_items = static_cast<uint32_t>(total0 + __shfl_sync(0xffffffffu, incl1, 31)) * Hkv;
+    }
     const bool static_first =
+        !rr &&
         blockIdx.x < static_cast<uint32_t>(static_first_seqs(a.num_seqs, a.grid_ctas, a.num_kv_heads)) * Hkv;
     uint32_t cur = 0;  // list index of the current item (items after a static first one)
-    if (static_first) {
+    if (rr) {
+      cur = blockIdx.x;
+      if (cur < n_items) {
+        rr_record(0, cur);
+        ok = wait_record(0);
+        if (ok) fetch_table(0);
+      }
+    } else if (static_first) {
       const int s = static_cast<int>(blockIdx.x / Hkv);
       if constexpr (PAGED) {
         // The table entries are requested together with the context length, one
@@ -599,7 +695,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
       if (!wait_table(k)) break;  // fetched while the previous item streamed
       const int32_t* rec = rec_slot(k);
       const int s = rec[0], part = rec[1], n_parts = rec[2], t_begin = rec[3], n_tok = rec[4];
-      const int kvh = static_cast<int>((is_static ? blockIdx.x : cur) % Hkv);
+      const int kvh = static_cast<int>((is_static ? blockIdx.x : cur) % Hkv);  // rr: cur = item
       if (lane == 0) {
         ItemInfo& info = items[slot];
         info.s = s;
@@ -619,12 +715,17 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
       bool next_ready = false;    // its record waited for and its table requested
       auto prepare_next = [&](int step) {
         if (step == 0) {
-          plan_wait();
-          if (lane == 0) {
-            nxt = atomicAdd(a.work, 1u);
-            if (nxt < n_items) copy_record(k + 1, nxt);
+          if (!rr) plan_wait();
+          if (rr) {
+            nxt = cur + gridDim.x;
+            if (nxt < n_items) rr_record(k + 1, nxt);
+          } else {
+            if (lane == 0) {
+              nxt = atomicAdd(a.work, 1u);
+              if (nxt < n_items) copy_record(k + 1, nxt);
+            }
+            nxt = __shfl_sync(0xffffffffu, nxt, 0);
           }
-          nxt = __shfl_sync(0xffffffffu, nxt, 0);
         } else if (!next_ready) {
           next_ready = true;
           if (nxt < n_items) {
@@ -703,6 +804,11 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
       if (!ok) break;  // the consumers time out on their next wait and stop too
       if (n_stages == 0 && !prepare_next(0)) break;
       if (!prepare_next(1)) break;  // one-stage (or empty) items: finish preparing now
+      // The next item (or the end of the work) is handed over only after the
+      // plan has finished: its counter reset precedes every publication.  (On
+      // the list schedule prepare_next waited already; the round-robin schedule
+      // reaches here first with its first item's stages in flight.)
+      plan_wait();
       cur = nxt;
     }
     // Never leave the CTA with copies in flight: wait (bounded) until the last

@@ -328,7 +328,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // a thread's products into the same accumulator, not these).  The issuing
     // thread polls both chains without blocking and issues whichever step is
     // ready, so while one chain waits (for its softmax, or for its product to
-    // complete) the tensor cores work on the other one.  A K (V) stage is
+    // complete) the tensor cores work on the other one.  The polls use
+    // mbarrier.test_wait, which never suspends the thread.  A K (V) stage is
     // released once every chain that uses it has issued its scores (product).
     if (lane == 0) {
       bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&k_full[0], 0);
@@ -362,8 +363,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           busy = true;
           if (!want_s[t]) {  // O_t += P_t(j) V_j once P_t(j) and V_j are there
             const int st = j % kPrefillStages;
-            if (!mbar_try_wait(&p_full[t], j & 1) ||
-                !mbar_try_wait(&v_full[st], (j / kPrefillStages) & 1))
+            if (!mbar_test_wait(&p_full[t], j & 1) ||
+                !mbar_test_wait(&v_full[st], (j / kPrefillStages) & 1))
               continue;
             tmem_fence_after_sync();
 #pragma unroll
@@ -382,8 +383,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               jt[t] = nkv_t[t];  // chain t is done
           } else {  // S_t(j+1) once the product reading P_t(j) is done and K_{j+1} is there
             const int st1 = (j + 1) % kPrefillStages;
-            if (!mbar_try_wait(&pv_done[t], j & 1) ||
-                !mbar_try_wait(&k_full[st1], ((j + 1) / kPrefillStages) & 1))
+            if (!mbar_test_wait(&pv_done[t], j & 1) ||
+                !mbar_test_wait(&k_full[st1], ((j + 1) / kPrefillStages) & 1))
               continue;
             tmem_fence_after_sync();
             issue_s(t, st1);
