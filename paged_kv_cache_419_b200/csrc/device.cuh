@@ -63,20 +63,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Non-blocking test of the phase with the given parity (returns at once; for
-// polling several barriers from one thread).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
 // try_wait that lets the hardware suspend the thread for up to `hint_ns` while
 // the phase is still open (no busy spinning on the issue slots).
 __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity,
