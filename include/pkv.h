@@ -72,6 +72,16 @@ typedef enum { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
 /* Human-readable name of a status code (static storage). */
 const char* pkv_status_string(pkv_status status);
 
+/* Why the last call on this host thread that returned PKV_ECUDA did so: the
+ * cudaError_t of the CUDA runtime call that failed (a launch with too many
+ * resources, a sticky fault of earlier work, ...), as an int; 0 if no call on
+ * this thread has returned PKV_ECUDA.  Later successful calls leave it as is. */
+int pkv_last_cuda_error(void);
+
+/* Name of a cudaError_t value, e.g. "cudaErrorLaunchOutOfResources" (static
+ * storage; the runtime's own name table). */
+const char* pkv_cuda_error_name(int error);
+
 /* Reads the device error flags of the current device into *flags_out after the
  * work queued on `stream` has finished (synchronises `stream`); clears them
  * when `clear` != 0. */

@@ -23,7 +23,8 @@ DEVERR_TABLE_ENTRY, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_COPY_PAIR, DEVERR_WA
 
 # Every function include/pkv.h declares.
 EXPORTS = (
-    "pkv_status_string", "pkv_device_error", "pkv_decode_workspace_bytes",
+    "pkv_status_string", "pkv_last_cuda_error", "pkv_cuda_error_name", "pkv_device_error",
+    "pkv_decode_workspace_bytes",
     "pkv_paged_attention_decode", "pkv_paged_attention_decode_static",
     "pkv_contiguous_attention_decode", "pkv_reshape_and_cache",
     "pkv_copy_blocks", "pkv_alloc_create", "pkv_alloc_destroy", "pkv_alloc_add_seq",
@@ -34,9 +35,16 @@ EXPORTS = (
 
 
 class PkvError(RuntimeError):
+    """A pkv_* call returned an error status; for PKV_ECUDA the message names the
+    CUDA error behind it (``cuda_error``, the cudaError_t value)."""
+
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)}")
+        self.cuda_error = last_cuda_error() if status == PKV_ECUDA else 0
+        msg = f"{what}: {status_string(status)}"
+        if status == PKV_ECUDA:
+            msg += f" ({cuda_error_name(self.cuda_error)})"
+        super().__init__(msg)
 
 
 class AllocStats(ctypes.Structure):
@@ -102,6 +110,8 @@ def lib() -> ctypes.CDLL:
             "pkv_alloc_refcount": ([P, i32, P], ctypes.c_int),
             "pkv_alloc_stats": ([P, ctypes.POINTER(AllocStats)], ctypes.c_int),
             "pkv_test_set_merge_wait": ([ctypes.c_uint64, ctypes.c_uint32], ctypes.c_int),
+            "pkv_last_cuda_error": ([], ctypes.c_int),
+            "pkv_cuda_error_name": ([ctypes.c_int], ctypes.c_char_p),
             "pkv_paged_prefill": ([P, P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
                                    ctypes.c_int, P], ctypes.c_int),
         }
@@ -115,6 +125,15 @@ def lib() -> ctypes.CDLL:
 
 def status_string(status: int) -> str:
     return lib().pkv_status_string(status).decode()
+
+
+def last_cuda_error() -> int:
+    """cudaError_t behind the last PKV_ECUDA of this thread (0 if none)."""
+    return int(lib().pkv_last_cuda_error())
+
+
+def cuda_error_name(error: int) -> str:
+    return lib().pkv_cuda_error_name(error).decode()
 
 
 def _check(status: int, what: str):

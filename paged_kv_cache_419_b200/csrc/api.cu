@@ -34,20 +34,39 @@ std::mutex g_devices_mutex;
 std::atomic<unsigned long long> g_merge_wait_limit_ns{0};
 std::atomic<uint32_t> g_merge_wait_extra{0};
 
+// The error of the last CUDA call that made a pkv_* call of this host thread
+// return PKV_ECUDA (pkv_last_cuda_error).
+thread_local int g_last_cuda_error = 0;
+
+// Records why a call returns PKV_ECUDA: the runtime's pending error of this
+// thread (taken, so that it is not blamed on a later launch), else `fallback`.
+pkv_status cuda_fail(cudaError_t fallback = cudaErrorUnknown) {
+  cudaError_t e = cudaGetLastError();
+  g_last_cuda_error = static_cast<int>(e != cudaSuccess ? e : fallback);
+  return PKV_ECUDA;
+}
+
+pkv_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return PKV_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return PKV_ECUDA;
+}
+
 // Per-device set-up with that device current: the device address of the error
 // flag and the SM count (under a lock: host threads may make their first call
 // on a device at the same time).
 pkv_status device_info(DeviceInfo** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_ECUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail();
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice);
   std::lock_guard<std::mutex> lock(g_devices_mutex);
   DeviceInfo& d = g_devices[dev];
   if (!d.ready) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return PKV_ECUDA;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return cuda_fail();
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return PKV_ECUDA;
+      return cuda_fail();
     d.err = static_cast<unsigned int*>(p);
     d.num_sms = sms;
     d.ready = true;
@@ -63,7 +82,7 @@ bool validate_env() {
   return v && v[0] && strcmp(v, "0") != 0;
 }
 
-pkv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ECUDA; }
+
 
 bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
 
@@ -134,7 +153,7 @@ EncodeTiledFn encode_tiled() {
 pkv_status encode_cache_map(CUtensorMap* m, const void* base, pkv_dtype dtype, int head_dim,
                             int64_t rows, int64_t planes, int box_rows) {
   const EncodeTiledFn fn = encode_tiled();
-  if (!fn) return PKV_ECUDA;
+  if (!fn) return cuda_fail(cudaErrorNotSupported);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim),
                               static_cast<cuuint64_t>(rows > 0 ? rows : 1),
                               static_cast<cuuint64_t>(planes > 0 ? planes : 1)};
@@ -238,7 +257,7 @@ pkv_status validate_decode_tables(const int32_t* tables, const int32_t* lens, in
       cudaMemcpyAsync(h_tab.data(), tables, sizeof(int32_t) * h_tab.size(), cudaMemcpyDeviceToHost,
                       stream) != cudaSuccess ||
       cudaStreamSynchronize(stream) != cudaSuccess)
-    return PKV_ECUDA;
+    return cuda_fail();
   for (int32_t s = 0; s < S; ++s) {
     const int64_t L = h_lens[s];
     if (L < 0 || L > static_cast<int64_t>(MB) * B) return PKV_ERANGE;
@@ -279,7 +298,7 @@ pkv_status validate_copy_pairs(const int64_t* pairs, int32_t n, int32_t num_bloc
 pkv_status encode_query_map(CUtensorMap* m, const void* q, pkv_dtype dtype, int head_dim,
                             int64_t num_heads, int64_t total_q) {
   const EncodeTiledFn fn = encode_tiled();
-  if (!fn) return PKV_ECUDA;
+  if (!fn) return cuda_fail(cudaErrorNotSupported);
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_heads),
                               static_cast<cuuint64_t>(total_q > 0 ? total_q : 1)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
@@ -307,7 +326,7 @@ pkv_status validate_prefill(const int32_t* query_start, const int32_t* lens, con
       cudaMemcpyAsync(h_tab.data(), tables, sizeof(int32_t) * h_tab.size(), cudaMemcpyDeviceToHost,
                       stream) != cudaSuccess ||
       cudaStreamSynchronize(stream) != cudaSuccess)
-    return PKV_ECUDA;
+    return cuda_fail();
   for (int32_t s = 0; s < S; ++s) {
     const int64_t T = static_cast<int64_t>(qs[s + 1]) - qs[s];
     const int64_t L = h_lens[s];
@@ -340,6 +359,12 @@ const char* pkv_status_string(pkv_status status) {
   return "unknown pkv_status";
 }
 
+int pkv_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* pkv_cuda_error_name(int error) {
+  return cudaGetErrorName(static_cast<cudaError_t>(error));
+}
+
 pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t stream) {
   if (!flags_out) return PKV_EINVAL;
   DeviceInfo* dev = nullptr;
@@ -347,9 +372,9 @@ pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t str
   if (st != PKV_OK) return st;
   unsigned int h = 0;
   if (cudaMemcpyAsync(&h, dev->err, sizeof h, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
-    return PKV_ECUDA;
-  if (clear && cudaMemsetAsync(dev->err, 0, sizeof h, stream) != cudaSuccess) return PKV_ECUDA;
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return PKV_ECUDA;
+    return cuda_fail();
+  if (clear && cudaMemsetAsync(dev->err, 0, sizeof h, stream) != cudaSuccess) return cuda_fail();
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return cuda_fail();
   *flags_out = h;
   return PKV_OK;
 }
@@ -428,7 +453,7 @@ pkv_status pkv_contiguous_attention_decode(void* out, const void* q, const void*
     if (cudaMemcpyAsync(h.data(), context_lens, sizeof(int32_t) * num_seqs,
                         cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
         cudaStreamSynchronize(stream) != cudaSuccess)
-      return PKV_ECUDA;
+      return cuda_fail();
     for (int32_t L : h)
       if (L < 0 || L > max_context_len) return PKV_ERANGE;
   }
@@ -527,7 +552,7 @@ pkv_status pkv_reshape_and_cache(const void* key, const void* value, void* k_cac
     if (cudaMemcpyAsync(h.data(), slot_mapping, sizeof(int64_t) * num_tokens,
                         cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
         cudaStreamSynchronize(stream) != cudaSuccess)
-      return PKV_ECUDA;
+      return cuda_fail();
     for (int64_t s : h)
       if (s >= static_cast<int64_t>(num_blocks) * block_size) return PKV_ERANGE;
   }
@@ -553,7 +578,7 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* src_dst_
     if (cudaMemcpyAsync(h.data(), src_dst_pairs, sizeof(int64_t) * h.size(), cudaMemcpyDeviceToHost,
                         stream) != cudaSuccess ||
         cudaStreamSynchronize(stream) != cudaSuccess)
-      return PKV_ECUDA;
+      return cuda_fail();
     const pkv_status vs = validate_copy_pairs(h.data(), num_pairs, num_blocks);
     if (vs != PKV_OK) return vs;
   }

@@ -15,7 +15,7 @@
 //  * One CTA per pair of 128-row query tiles of one sequence: two heads of a
 //    kv group on the same rows when Hq / Hkv is even (both tiles read the same
 //    K/V tiles and do the same work), else two consecutive row tiles of one
-//    head.  320 threads, one CTA per SM (192 KB of shared memory at head_dim
+//    head.  576 threads, one CTA per SM (197 KB of shared memory at head_dim
 //    128).  Query tiles with more keys are scheduled first.
 //  * Warp 0 loads: both tiles' Q rows once (TMA, 128-byte swizzle), then the K
 //    and V tiles of 128 keys through a ring of two stages, one TMA box per
@@ -28,16 +28,18 @@
 //    tile, as an MN-major operand.  While the softmax of one query tile runs,
 //    the tensor cores work on the other tile.  Completion is signalled to
 //    mbarriers with tcgen05.commit.
-//  * Warps 2-5 (tile 0) and 6-9 (tile 1) own one query row per thread
-//    (tensor-memory lane = row).  Pass 1 reads the row's scores and takes the
-//    max, with the causal mask applied by select (so garbage keys past the
-//    context never reach a sum); the row of O is rescaled in tensor memory when
-//    the max grows.  Pass 2 turns the scores into P (base-2 exponentials,
-//    rounded to the input type, two per 32-bit column) and stores it over the
-//    first 64 columns of the tile's own score buffer.  The sum is taken over the
-//    rounded weights, so the output is an exact convex combination of V rows.
-//    In the last key tile they zero the V rows past the context (0 x NaN would
-//    be NaN).
+//  * Warps 2-9 (tile 0) and 10-17 (tile 1) hold two threads per query row
+//    (tensor-memory lane = row), each with half of the tile's 128 keys in
+//    registers.  Each half takes its max, with the causal mask applied by
+//    select (so garbage keys past the context never reach a sum); the halves
+//    exchange maxima through shared memory at a named barrier of the tile's
+//    256 threads, and each rescales its half of the row of O in tensor memory
+//    when the max grows.  Then each turns its scores into P (base-2
+//    exponentials, rounded to the input type, two per 32-bit column) and
+//    stores it over the first 64 columns of the tile's own score buffer.  The
+//    sum is taken over the rounded weights, so the output is an exact convex
+//    combination of V rows.  In the last key tile they zero the V rows past
+//    the context (0 x NaN would be NaN).
 //  * The next scores of a tile overwrite its P, so they are issued only after
 //    the product reading P has completed (tcgen05.mma orders only products
 //    into the same accumulator).
@@ -130,7 +132,30 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]);
+
 // 16 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st16f(uint32_t taddr, const float (&v)[16]) {
+  uint32_t u[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[i]);
+  tmem_st16(taddr, u);
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
@@ -205,8 +230,11 @@ constexpr float kLazy = 8.f;
 // chunk.  Two heads of one kv group share the rows when Hq / Hkv is even (the
 // tiles read the same K/V tiles and do the same work); otherwise one head
 // takes two consecutive row tiles.
+// 96 registers: the register file is split between the SM's four schedulers
+// (16 K registers each) and 18 warps put five on two of them, 5 x 32 x 96 <=
+// 16 K; more registers per thread and the launch fails for lack of resources.
 template <typename T, int D>
-__global__ void __launch_bounds__(kPrefillThreads, 1)
+__global__ void __maxnreg__(96)
     prefill_kernel(const PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
   using Tr = PrefillTraits<D>;
   constexpr int ND = Tr::ND;
@@ -272,7 +300,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 4);  // one arrival per softmax warp of the tile
+      mbar_init(&p_full[t], 8);  // one arrival per softmax warp of the tile
       mbar_init(&pv_done[t], 1);
     }
     mbar_init(o_final, 1);
@@ -374,7 +402,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (lane == 0) {
       bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&k_full[0], 0);
       auto issue_s = [&](int t, int st) {  // S_t = Q_t K^T of the key tile in stage st
-#pragma unroll
+#pragma unroll 2
         for (int k = 0; k < KSTEPS; ++k) {
           const uint32_t koff = (k >> 2) * Tr::PANEL + (k & 3) * 32;
           umma_f16(tmem + Tr::colS(t), umma_desc(sQ + t * Tr::TILE + koff, 16, 1024),
@@ -403,7 +431,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             break;
           }
           tmem_fence_after_sync();
-#pragma unroll
+#pragma unroll 2
           for (int k = 0; k < PV_STEPS; ++k)
             umma_f16_ts(tmem + Tr::colO(t), tmem + Tr::colS(t) + k * 8,
                         umma_desc(sV + st * Tr::TILE + k * 2048, Tr::PANEL, 1024), IDESC_O,
@@ -430,134 +458,141 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     __syncwarp();
   } else {
     // ============================================================ softmax rows
-    const int t = (warp - 2) >> 2;                // query tile of this warp group
+    // Query tile t has 8 warps, two threads per query row (tensor-memory lane =
+    // row): half hf holds keys 64 hf .. 64 hf + 63 of every key tile, and output
+    // columns hf D/2 .. hf D/2 + D/2 - 1.  The two halves of a row combine their
+    // maxima (and, at the end, their sums) through shared memory at a named
+    // barrier of the tile's 256 threads; a failed wait anywhere in the tile is
+    // carried by that barrier, so all of the tile's threads stop together.
+    const int t = (warp - 2) >> 3;                // query tile of this warp group
+    const int hf = ((warp - 2) >> 2) & 1;         // half of the keys / output columns
     const int quarter = warp & 3;                 // tensor-memory lanes 32 quarter ..
     const int r = quarter * 32 + lane;            // this thread's query row of the tile
     const int i = i0_t[t] + r;                    // its token index in the chunk
     const bool valid = i < n_new;
     const int limit = valid ? p0 + i : L - 1;     // last key this row may see
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t cS = lane_base + Tr::colS(t), cO = lane_base + Tr::colO(t);
+    const uint32_t cS = lane_base + Tr::colS(t) + 64 * hf;          // this half's scores
+    const uint32_t cP = lane_base + Tr::colS(t) + 32 * hf;          // its P columns
+    const uint32_t cO = lane_base + Tr::colO(t) + hf * (D / 2);     // its output columns
+    float* red = reinterpret_cast<float*>(smem + Tr::OFF_RED) + t * 2 * kPrefillTileM;
+    float* red_l = reinterpret_cast<float*>(smem + Tr::OFF_RED) + (4 + t * 2) * kPrefillTileM;
+    const int bar_id = 1 + t;
     // Running state of the row, in base-2 units: m is the max the weights are
     // taken against (at most kLazy below the true running max, see below) and
-    // l the sum of the rounded weights.
+    // l this half's sum of the rounded weights.
     const float sl = a.scale_log2;
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv_t[t]; ++j) {
-      const int k_lo = j * kPrefillTileN;
+      const int k0 = j * kPrefillTileN + 64 * hf;  // first key of this half
       ok = ok && mbar_wait_bounded(&s_full[t], j & 1);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      const bool wok = __all_sync(0xffffffffu, ok);
       tmem_fence_after_sync();
-      // Pass 1: the row's 128 scores, all requested before one wait, and their
-      // max in base-2 units.  Keys past this row's limit count as -inf (by
-      // select); only tiles on the diagonal (or past the context) need that,
-      // and a warp takes the masked path only when one of its rows needs it.
-      const bool masked = __any_sync(0xffffffffu, k_lo + kPrefillTileN - 1 > limit);
-      float mx;
-      {
-        float x[kPrefillTileN];
+      // This half's 64 scores (one wait), kept in registers for both passes.
+      float x[64];
+      if (wok) {
 #pragma unroll
-        for (int c = 0; c < kPrefillTileN / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           float v[32];
           tmem_ld32(cS + c * 32, v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) x[c * 32 + e] = v[e];
         }
         tmem_wait_ld();
-        // The max of scale * s is scale * max s for scale >= 0 (scale * min s
-        // otherwise): reduce the raw scores, three at a time, and scale once.
-        if (sl >= 0.f) {
-          if (masked) {
-#pragma unroll
-            for (int e = 0; e < kPrefillTileN; ++e) x[e] = k_lo + e <= limit ? x[e] : -CUDART_INF_F;
-          }
-          mx = max3_tree<kPrefillTileN>(x) * sl;
-        } else {
-          if (masked) {
-#pragma unroll
-            for (int e = 0; e < kPrefillTileN; ++e) x[e] = k_lo + e <= limit ? x[e] : CUDART_INF_F;
-          }
-          mx = min3_tree<kPrefillTileN>(x) * sl;
-        }
       }
+      // Keys past this row's limit count as -inf (by select); only tiles on
+      // the diagonal (or past the context) need that, and a warp takes the
+      // masked path only when one of its rows needs it.  The max of scale * s
+      // is scale * max s for scale >= 0 (scale * min s otherwise).
+      const bool masked = __any_sync(0xffffffffu, k0 + 63 > limit);
+      const bool pos = sl >= 0.f;
+      float part;
+      if (!wok) {
+        part = pos ? -CUDART_INF_F : CUDART_INF_F;
+      } else if (pos) {
+        if (masked) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) x[e] = k0 + e <= limit ? x[e] : -CUDART_INF_F;
+        }
+        part = max3_tree<64>(x);
+      } else {
+        if (masked) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) x[e] = k0 + e <= limit ? x[e] : CUDART_INF_F;
+        }
+        part = min3_tree<64>(x);
+      }
+      red[hf * kPrefillTileM + r] = part;
+      // Both halves of every row have read their scores after this barrier, so
+      // the P writes below (over score columns) cannot race with a read.
+      if (named_barrier_or(bar_id, 2 * kPrefillTileM, !wok)) {
+        ok = false;
+        break;
+      }
+      const float other = red[(1 - hf) * kPrefillTileM + r];
+      const float mx = (pos ? fmaxf(part, other) : fminf(part, other)) * sl;
       // Lazy rescale: the weights are 2^(x - m) with m allowed to lag the true
       // running max by up to kLazy (weights up to 2^kLazy, exact in the input
       // type's range and in fp32), so O and l are rescaled only when the max
       // outgrows that.  The product of the previous key tile ran before S_t(j),
       // so O_t holds it.  tcgen05.ld / st are warp-wide (.sync.aligned): the
       // whole warp takes the branch, rows that need no rescale multiply by 1.
+      // Both halves decide alike (they see the same max).
       const bool grow = mx > m + kLazy;
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
         const float alpha = grow ? fast_exp2(m - mx) : 1.f;
         l *= alpha;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tmem_ld32(cO + c * 32, v);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {  // this half's D/2 columns, 16 at a time
+          float v[16];
+          tmem_ld16(cO + c * 16, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] *= alpha;
-          tmem_st32(cO + c * 32, v);
+          for (int e = 0; e < 16; ++e) v[e] *= alpha;
+          tmem_st16f(cO + c * 16, v);
         }
       }
       if (grow) m = mx;
-      // Pass 2, in two halves of 64 scores (two loads, one wait each): P =
-      // 2^(x - m) rounded to the input type, two keys per 32-bit column, over
-      // the first 64 columns of S (the columns a half writes were read by the
-      // halves before it); the sum is over the rounded weights, in packed
-      // pairs of partial sums.
+      // P = 2^(x - m) rounded to the input type, two keys per 32-bit column,
+      // this half's 32 columns over the first 64 columns of S; the sum is over
+      // the rounded weights, in packed pairs of partial sums.
       float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float x[64];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float v[32];
-          tmem_ld32(cS + hh * 64 + c * 32, v);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[c * 32 + e] = v[e];
-        }
-        tmem_wait_ld();
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const int kk = k_lo + hh * 64 + e;
+        for (int e = 0; e < 32; e += 2) {
+          const int ee = c * 32 + e;
           float p0v, p1v;
           if (masked) {
-            p0v = kk <= limit ? fast_exp2(x[e] * sl - m) : 0.f;
-            p1v = kk + 1 <= limit ? fast_exp2(x[e + 1] * sl - m) : 0.f;
+            p0v = k0 + ee <= limit ? fast_exp2(x[ee] * sl - m) : 0.f;
+            p1v = k0 + ee + 1 <= limit ? fast_exp2(x[ee + 1] * sl - m) : 0.f;
           } else {
-            p0v = fast_exp2(x[e] * sl - m);
-            p1v = fast_exp2(x[e + 1] * sl - m);
+            p0v = fast_exp2(x[ee] * sl - m);
+            p1v = fast_exp2(x[ee + 1] * sl - m);
           }
           pk[e / 2] = pack2<T>(p0v, p1v);
           sum2[(e >> 1) & 1] = __fadd2_rn(sum2[(e >> 1) & 1], unpack2<T>(pk[e / 2]));
         }
-        uint32_t lo[16], hi[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          lo[e] = pk[e];
-          hi[e] = pk[16 + e];
-        }
-        tmem_st16(cS + hh * 32, lo);
-        tmem_st16(cS + hh * 32 + 16, hi);
+        tmem_st16(cP + c * 16, pk);
       }
       l += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
       tmem_wait_st();
       // The key tile that reaches past the context: zero the V rows of the keys
-      // past it (whatever the stage held there, 0 x it must be 0).  Each chain
-      // does it before its own product (the two products may run in either
-      // order); the second chain writes zeros over zeros.
-      if (k_lo + kPrefillTileN > L) {
+      // past it (whatever the stage held there, 0 x it must be 0).  The two
+      // threads of a row zero half of its 16-byte chunks each, in both query
+      // tiles' warps, before each tile's product (the two tiles' products may
+      // run in either order); later writes are zeros over zeros.
+      if (j * kPrefillTileN + kPrefillTileN > L) {
         const int st = j % kPrefillStages;
         ok = ok && mbar_wait_bounded(&v_full[st], (j / kPrefillStages) & 1);
-        if (ok && k_lo + r >= L) {
+        if (ok && j * kPrefillTileN + r >= L) {
           uint8_t* vrow = smem + Tr::OFF_V + st * Tr::TILE + r * 128;
 #pragma unroll
           for (int pn = 0; pn < ND; ++pn)
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
+            for (int ch = 4 * hf; ch < 4 * hf + 4; ++ch)
               *reinterpret_cast<uint4*>(vrow + pn * Tr::PANEL + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();
@@ -566,30 +601,31 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    // ---- epilogue: out = O / l
+    // ---- epilogue: out = O / (l_half0 + l_half1), this half's columns
     ok = ok && (nkv_t[t] == 0 || mbar_wait_bounded(o_final, 0));
-    if (__all_sync(0xffffffffu, ok)) {
-      if (nkv_t[t] > 0) {
-        tmem_fence_after_sync();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        T* orow = static_cast<T*>(a.out) + (static_cast<int64_t>(q0 + i) * a.num_heads + h_t[t]) * D;
+    red_l[hf * kPrefillTileM + r] = l;
+    if (named_barrier_or(bar_id, 2 * kPrefillTileM, !__all_sync(0xffffffffu, ok))) {
+      if (lane == 0) set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
+    } else if (nkv_t[t] > 0) {
+      tmem_fence_after_sync();
+      const float lr = red_l[r] + red_l[kPrefillTileM + r];
+      const float inv = lr > 0.f ? 1.f / lr : 0.f;
+      T* orow = static_cast<T*>(a.out) + (static_cast<int64_t>(q0 + i) * a.num_heads + h_t[t]) * D +
+                hf * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tmem_ld32(cO + c * 32, v);
-          tmem_wait_ld();
-          if (valid) {
+      for (int c = 0; c < D / 64; ++c) {
+        float v[32];
+        tmem_ld32(cO + c * 32, v);
+        tmem_wait_ld();
+        if (valid) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              const uint4 w = make_uint4(pack2<T>(v[e] * inv, v[e + 1] * inv), pack2<T>(v[e + 2] * inv, v[e + 3] * inv),
-                                         pack2<T>(v[e + 4] * inv, v[e + 5] * inv), pack2<T>(v[e + 6] * inv, v[e + 7] * inv));
-              *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
-            }
+          for (int e = 0; e < 32; e += 8) {
+            const uint4 w = make_uint4(pack2<T>(v[e] * inv, v[e + 1] * inv), pack2<T>(v[e + 2] * inv, v[e + 3] * inv),
+                                       pack2<T>(v[e + 4] * inv, v[e + 5] * inv), pack2<T>(v[e + 6] * inv, v[e + 7] * inv));
+            *reinterpret_cast<uint4*>(orow + c * 32 + e) = w;
           }
         }
       }
-    } else if (lane == 0) {
-      set_error(a.err, PKV_DEVERR_WAIT_TIMEOUT);
     }
   }
   // Nothing of the tensor cores or the copies is in flight past here: the MMA

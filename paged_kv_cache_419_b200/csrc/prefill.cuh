@@ -33,7 +33,7 @@ struct PrefillMaps {
   CUtensorMap q, k, v;
 };
 
-constexpr int kPrefillThreads = 320;  // TMA, MMA, 2 x 4 softmax warps
+constexpr int kPrefillThreads = 576;  // TMA, MMA, 2 x 8 softmax warps
 constexpr int kPrefillTileM = 128;  // query rows per CTA
 constexpr int kPrefillTileN = 128;  // keys per tile
 constexpr int kPrefillStages = 2;
@@ -47,7 +47,8 @@ struct PrefillTraits {
   static constexpr int OFF_Q = 0;                         // two query tiles
   static constexpr int OFF_K = OFF_Q + 2 * TILE;
   static constexpr int OFF_V = OFF_K + kPrefillStages * TILE;
-  static constexpr int OFF_BAR = OFF_V + kPrefillStages * TILE;
+  static constexpr int OFF_RED = OFF_V + kPrefillStages * TILE;  // [2 tiles][2 halves][128] maxima, then sums
+  static constexpr int OFF_BAR = OFF_RED + 8 * kPrefillTileM * 4;
   // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], p_full[2], pv_done[2], o_final
   static constexpr int NUM_BARS = 1 + 4 * kPrefillStages + 6 + 1;
   static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;

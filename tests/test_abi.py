@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from paged_kv_cache_419_b200 import binding as B
 
@@ -32,6 +33,25 @@ def test_library_exports_every_declared_function():
 def test_status_strings():
     for code in (B.PKV_OK, B.PKV_EINVAL, B.PKV_EUNSUPPORTED, B.PKV_ECUDA, B.PKV_ENOMEM, B.PKV_ERANGE):
         assert B.status_string(code).startswith("PKV_")
+
+
+def test_cuda_error_names():
+    assert B.cuda_error_name(0) == "cudaSuccess"
+    assert B.cuda_error_name(2) == "cudaErrorMemoryAllocation"
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a GPU")
+def test_cuda_failure_is_reported_with_its_cuda_error():
+    """Without a GPU the first CUDA call of pkv_device_error fails; the status is
+    PKV_ECUDA and the binding's error names the CUDA error behind it."""
+    flags = ctypes.c_uint(0)
+    status = B.lib().pkv_device_error(ctypes.byref(flags), 1, None)  # default stream
+    with pytest.raises(B.PkvError) as e:
+        B._check(status, "pkv_device_error")
+    assert e.value.status == B.PKV_ECUDA
+    assert e.value.cuda_error != 0 and B.last_cuda_error() == e.value.cuda_error
+    assert B.cuda_error_name(e.value.cuda_error) in str(e.value)
+    assert B.cuda_error_name(e.value.cuda_error).startswith("cudaError")
 
 
 def _layout_bytes(S, Hq, D, ctx, part=512):
