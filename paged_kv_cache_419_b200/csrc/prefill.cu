@@ -34,9 +34,10 @@
 //    select (so garbage keys past the context never reach a sum); the halves
 //    exchange maxima through shared memory at a named barrier of the tile's
 //    256 threads, and each rescales its half of the row of O in tensor memory
-//    when the max grows.  Then each turns its scores into P (base-2
-//    exponentials, rounded to the input type, two per 32-bit column) and
-//    stores it over the first 64 columns of the tile's own score buffer.  The
+//    when the max grows.  Then each reloads its scores 32 at a time, turns
+//    them into P (base-2 exponentials, rounded to the input type, two per
+//    32-bit column) and stores P over the first 32 of its own 64 score
+//    columns (so neither half overwrites scores the other still reads).  The
 //    sum is taken over the rounded weights, so the output is an exact convex
 //    combination of V rows.  In the last key tile they zero the V rows past
 //    the context (0 x NaN would be NaN).
@@ -392,7 +393,7 @@ __global__ void __maxnreg__(96)
     // ============================================================ tensor cores
     // Order of the products: S_0(0), S_1(0); then for each key tile j:
     // O_0 += P_0(j) V_j, S_0(j+1), O_1 += P_1(j) V_j, S_1(j+1).  P_t(j) lives in
-    // tensor memory over the first 64 columns of S_t(j), so S_t(j+1) is issued
+    // tensor memory inside the columns of S_t(j), so S_t(j+1) is issued
     // only once the product that reads P_t(j) has completed (the hardware orders
     // a thread's products into the same accumulator, not these).  The fixed
     // order keeps the two tiles half a step apart: while one tile's softmax
@@ -433,7 +434,7 @@ __global__ void __maxnreg__(96)
           tmem_fence_after_sync();
 #pragma unroll 2
           for (int k = 0; k < PV_STEPS; ++k)
-            umma_f16_ts(tmem + Tr::colO(t), tmem + Tr::colS(t) + k * 8,
+            umma_f16_ts(tmem + Tr::colO(t), tmem + Tr::colS(t) + (k >> 2) * 64 + (k & 3) * 8,
                         umma_desc(sV + st * Tr::TILE + k * 2048, Tr::PANEL, 1024), IDESC_O,
                         j > 0 || k > 0);
           umma_commit(&pv_done[t]);
@@ -473,7 +474,7 @@ __global__ void __maxnreg__(96)
     const int limit = valid ? p0 + i : L - 1;     // last key this row may see
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t cS = lane_base + Tr::colS(t) + 64 * hf;          // this half's scores
-    const uint32_t cP = lane_base + Tr::colS(t) + 32 * hf;          // its P columns
+    const uint32_t cP = lane_base + Tr::colS(t) + 64 * hf;          // its P columns
     const uint32_t cO = lane_base + Tr::colO(t) + hf * (D / 2);     // its output columns
     float* red = reinterpret_cast<float*>(smem + Tr::OFF_RED) + t * 2 * kPrefillTileM;
     float* red_l = reinterpret_cast<float*>(smem + Tr::OFF_RED) + (4 + t * 2) * kPrefillTileM;
@@ -489,9 +490,15 @@ __global__ void __maxnreg__(96)
       ok = ok && mbar_wait_bounded(&s_full[t], j & 1);
       const bool wok = __all_sync(0xffffffffu, ok);
       tmem_fence_after_sync();
-      // This half's 64 scores (one wait), kept in registers for both passes.
-      float x[64];
+      // Keys past this row's limit count as -inf (by select); only tiles on
+      // the diagonal (or past the context) need that, and a warp takes the
+      // masked path only when one of its rows needs it.  The max of scale * s
+      // is scale * max s for scale >= 0 (scale * min s otherwise).
+      const bool masked = __any_sync(0xffffffffu, k0 + 63 > limit);
+      const bool pos = sl >= 0.f;
+      float part = pos ? -CUDART_INF_F : CUDART_INF_F;
       if (wok) {
+        float x[64];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           float v[32];
@@ -500,28 +507,19 @@ __global__ void __maxnreg__(96)
           for (int e = 0; e < 32; ++e) x[c * 32 + e] = v[e];
         }
         tmem_wait_ld();
-      }
-      // Keys past this row's limit count as -inf (by select); only tiles on
-      // the diagonal (or past the context) need that, and a warp takes the
-      // masked path only when one of its rows needs it.  The max of scale * s
-      // is scale * max s for scale >= 0 (scale * min s otherwise).
-      const bool masked = __any_sync(0xffffffffu, k0 + 63 > limit);
-      const bool pos = sl >= 0.f;
-      float part;
-      if (!wok) {
-        part = pos ? -CUDART_INF_F : CUDART_INF_F;
-      } else if (pos) {
-        if (masked) {
+        if (pos) {
+          if (masked) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) x[e] = k0 + e <= limit ? x[e] : -CUDART_INF_F;
-        }
-        part = max3_tree<64>(x);
-      } else {
-        if (masked) {
+            for (int e = 0; e < 64; ++e) x[e] = k0 + e <= limit ? x[e] : -CUDART_INF_F;
+          }
+          part = max3_tree<64>(x);
+        } else {
+          if (masked) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) x[e] = k0 + e <= limit ? x[e] : CUDART_INF_F;
+            for (int e = 0; e < 64; ++e) x[e] = k0 + e <= limit ? x[e] : CUDART_INF_F;
+          }
+          part = min3_tree<64>(x);
         }
-        part = min3_tree<64>(x);
       }
       red[hf * kPrefillTileM + r] = part;
       // Both halves of every row have read their scores after this barrier, so
@@ -555,22 +553,27 @@ __global__ void __maxnreg__(96)
       }
       if (grow) m = mx;
       // P = 2^(x - m) rounded to the input type, two keys per 32-bit column,
-      // this half's 32 columns over the first 64 columns of S; the sum is over
-      // the rounded weights, in packed pairs of partial sums.
+      // over the first 32 of this half's 64 score columns (the product's K
+      // step k, keys 16 k .. 16 k + 15, reads columns 64 (k / 4) + 8 (k % 4));
+      // the sum is over the rounded weights, in packed pairs of partial sums.
       float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
+        float xv[32];
+        tmem_ld32(cS + c * 32, xv);
+        tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int ee = c * 32 + e;
           float p0v, p1v;
           if (masked) {
-            p0v = k0 + ee <= limit ? fast_exp2(x[ee] * sl - m) : 0.f;
-            p1v = k0 + ee + 1 <= limit ? fast_exp2(x[ee + 1] * sl - m) : 0.f;
+            p0v = k0 + ee <= limit ? fast_exp2(xv[e] * sl - m) : 0.f;
+            p1v = k0 + ee + 1 <= limit ? fast_exp2(xv[e + 1] * sl - m) : 0.f;
           } else {
-            p0v = fast_exp2(x[ee] * sl - m);
-            p1v = fast_exp2(x[ee + 1] * sl - m);
+            const float2 y = __ffma2_rn(make_float2(xv[e], xv[e + 1]), make_float2(sl, sl), make_float2(-m, -m));
+            p0v = fast_exp2(y.x);
+            p1v = fast_exp2(y.y);
           }
           pk[e / 2] = pack2<T>(p0v, p1v);
           sum2[(e >> 1) & 1] = __fadd2_rn(sum2[(e >> 1) & 1], unpack2<T>(pk[e / 2]));

@@ -57,8 +57,9 @@ struct PrefillTraits {
   // less than 117 KB: two CTAs never share an SM, so the second never waits in
   // tcgen05.alloc for the first one's 512 tensor-memory columns.
   static constexpr int SMEM_BYTES = SMEM_USED + 1024 > 117 * 1024 ? SMEM_USED + 1024 : 117 * 1024;
-  // tensor memory: query tile t has its scores at colS(t) (128 columns; its P
-  // over the first 64 of them) and its output accumulator at colO(t) (D columns)
+  // tensor memory: query tile t has its scores at colS(t) (128 columns; P of
+  // keys 64 h .. 64 h + 63 over columns 64 h .. 64 h + 31 of them) and its
+  // output accumulator at colO(t) (D columns)
   static constexpr uint32_t colS(int t) { return 256u * static_cast<uint32_t>(t); }
   static constexpr uint32_t colO(int t) { return 256u * static_cast<uint32_t>(t) + 128u; }
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
