@@ -179,6 +179,21 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// tcgen05.wait::ld that takes the loaded registers as operands, so that no use
+// of them can be scheduled before the wait (for a load left in flight while
+// other work runs; elsewhere the plain wait directly follows its loads).
+__device__ __forceinline__ void tmem_wait_ld_tied(float (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]),
+                 "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]),
+                 "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]),
+                 "+f"(v[21]), "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]),
+                 "+f"(v[28]), "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
+               :
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // max (min) of N values, three at a time (three-input max.f32 / min.f32).
@@ -557,11 +572,22 @@ __global__ void __maxnreg__(96)
       // step k, keys 16 k .. 16 k + 15, reads columns 64 (k / 4) + 8 (k % 4));
       // the sum is over the rounded weights, in packed pairs of partial sums.
       float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      // The second 32 scores are loaded while the first 32 are turned into P.
+      float xa[32], xb[32];
+      tmem_ld32(cS, xa);
+      tmem_wait_ld_tied(xa);
+      tmem_ld32(cS + 32, xb);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float xv[32];
-        tmem_ld32(cS + c * 32, xv);
-        tmem_wait_ld();
+        if (c == 0) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) xv[e] = xa[e];
+        } else {
+          tmem_wait_ld_tied(xb);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) xv[e] = xb[e];
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
