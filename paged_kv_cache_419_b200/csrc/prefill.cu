@@ -71,16 +71,6 @@ __host__ __device__ constexpr uint32_t umma_idesc_f16(uint32_t ab_format, uint32
          ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, bool accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
-      : "memory");
-}
-
 // Arrive on `bar` once every tcgen05 operation this thread issued so far is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -167,14 +157,62 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       : "memory");
 }
 
-// A from tensor memory, B from shared memory (kind::f16, fp32 accumulation).
-__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, bool accumulate) {
+// One product S = A B^T over K = 16 NK (NK = 4 or 8) as one block of
+// instructions, so that nothing else of the issuing thread sits between the
+// steps (an MMA is accepted about when the previous one starts, so any delay
+// in issuing the next one idles the tensor cores).  Both operands K-major with
+// 128-byte rows in panels of 128 rows: K step k at descriptor offset
+// (k / 4) * 1024 + (k % 4) * 2 (16-byte units).  The first step overwrites D.
+template <int NK>
+__device__ __forceinline__ void umma_ss_steps(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc) {
+  static_assert(NK == 4 || NK == 8, "4 or 8 K steps");
+#define PKV_SS_STEP(OFF)                                                                  \
+  "add.s64 a1, %1, " #OFF ";\n\tadd.s64 b1, %2, " #OFF ";\n\t"                              \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, p;\n\t"
+  if constexpr (NK == 4) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 a1, b1;\n\t"
+        "setp.ne.b32 p, %3, %3;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "setp.eq.b32 p, %3, %3;\n\t"
+        PKV_SS_STEP(2) PKV_SS_STEP(4) PKV_SS_STEP(6) "}"
+        ::"r"(d), "l"(a), "l"(b), "r"(idesc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 a1, b1;\n\t"
+        "setp.ne.b32 p, %3, %3;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "setp.eq.b32 p, %3, %3;\n\t"
+        PKV_SS_STEP(2) PKV_SS_STEP(4) PKV_SS_STEP(6)
+        PKV_SS_STEP(1024) PKV_SS_STEP(1026) PKV_SS_STEP(1028) PKV_SS_STEP(1030) "}"
+        ::"r"(d), "l"(a), "l"(b), "r"(idesc)
+        : "memory");
+  }
+#undef PKV_SS_STEP
+}
+
+// One chunk of O += P V, A (P) from tensor memory, B (V) MN-major in shared
+// memory, as one block of instructions: K steps 2c, 2c + 1, 2c + 4, 2c + 5
+// (keys 32 c .. 32 c + 31 of each half of the key tile).  `a` is the tensor-
+// memory address of step 2c's P (the others at + 8, + 64, + 72 columns), `b`
+// the V descriptor of step 2c (the others at + 128, + 512, + 640 in 16-byte
+// units: 16 keys of 128-byte rows per step).  The first step accumulates
+// only if `acc` != 0.
+__device__ __forceinline__ void umma_ts_chunk(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p;\n\t.reg .b32 a1;\n\t.reg .b64 b1;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "setp.eq.b32 p, %3, %3;\n\t"
+      "add.s32 a1, %1, 8;\n\tadd.s64 b1, %2, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p;\n\t"
+      "add.s32 a1, %1, 64;\n\tadd.s64 b1, %2, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p;\n\t"
+      "add.s32 a1, %1, 72;\n\tadd.s64 b1, %2, 640;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, p;\n\t}"
+      ::"r"(d), "r"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
 
@@ -241,6 +279,41 @@ __device__ __forceinline__ float min3_tree(const float (&x)[N]) {
 // before the output row is rescaled: weights stay below 2^8.
 constexpr float kLazy = 8.f;
 
+// Coefficients c_0 .. c_n of p(f) ~ 2^f on |f| <= 1/2, minimax in relative
+// error (fitted by exp2_poly_fit.py beside this file): degree 3, error 2^-13.7,
+// for bf16 weights (8 significant bits); degree 4, error 2^-18.5, for fp16 (11).
+__device__ constexpr float kExp2Deg3[4] = {0.9999280571937561f, 0.6932609677314758f, 0.2426111400127411f,
+                                           0.055171627551317215f};
+__device__ constexpr float kExp2Deg4[5] = {0.9999992847442627f, 0.6931217908859253f, 0.240247443318367f,
+                                           0.05591786280274391f, 0.009570096619427204f};
+
+// 2^y for a pair, on the FMA pipe instead of MUFU (which takes 16 per clock per
+// SM): Cody-Waite range reduction y = j + f, j = rint(y) by the 1.5 * 2^23
+// rounding shift, |f| <= 1/2; then p(f) by Horner and j added to p's exponent
+// field.  y is clamped at -125, so that the result is a normal number (p(f)
+// >= 2^-1/2 puts the field at >= 1); a row's largest weight is at least 1, so
+// only negligible weights are clamped.
+template <typename T>
+__device__ __forceinline__ float2 exp2_poly2(float2 y) {
+  y.x = fmaxf(y.x, -125.f);
+  y.y = fmaxf(y.y, -125.f);
+  const float2 t = __fadd2_rn(y, make_float2(12582912.f, 12582912.f));
+  const float2 j = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), y);  // y - j, exact
+  float2 p;
+  if constexpr (std::is_same<T, __half>::value) {
+    p = make_float2(kExp2Deg4[4], kExp2Deg4[4]);
+#pragma unroll
+    for (int k = 3; k >= 0; --k) p = __ffma2_rn(p, f, make_float2(kExp2Deg4[k], kExp2Deg4[k]));
+  } else {
+    p = make_float2(kExp2Deg3[3], kExp2Deg3[3]);
+#pragma unroll
+    for (int k = 2; k >= 0; --k) p = __ffma2_rn(p, f, make_float2(kExp2Deg3[k], kExp2Deg3[k]));
+  }
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // ------------------------------------------------------------ kernel
 // Query tile t in {0, 1} of a CTA: head h_t, rows i0_t .. i0_t + 127 of the
 // chunk.  Two heads of one kv group share the rows when Hq / Hkv is even (the
@@ -255,7 +328,7 @@ __global__ void __maxnreg__(96)
   using Tr = PrefillTraits<D>;
   constexpr int ND = Tr::ND;
   constexpr int KSTEPS = D / 16;               // k-steps of S = Q K^T
-  constexpr int PV_STEPS = kPrefillTileN / 16; // k-steps of O += P V
+  static_assert(kPrefillTileN == 128, "O += P V in two chunks of K steps: {0, 1, 4, 5} and {2, 3, 6, 7}");
   constexpr uint32_t AB_FMT = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t IDESC_S = umma_idesc_f16(AB_FMT, 0u, kPrefillTileM, kPrefillTileN);
   constexpr uint32_t IDESC_O = umma_idesc_f16(AB_FMT, 1u, kPrefillTileM, D);
@@ -300,8 +373,8 @@ __global__ void __maxnreg__(96)
   uint64_t* k_empty = v_full + kPrefillStages;
   uint64_t* v_empty = k_empty + kPrefillStages;
   uint64_t* s_full = v_empty + kPrefillStages;   // [2]: scores of tile t ready
-  uint64_t* p_full = s_full + 2;                 // [2]: P of tile t in tensor memory
-  uint64_t* pv_done = p_full + 2;                // [2]: O_t += P_t V done (P_t may be overwritten)
+  uint64_t* p_full = s_full + 2;                 // [2][2]: chunk c of P of tile t in tensor memory
+  uint64_t* pv_done = p_full + 4;                // [2]: O_t += P_t V done (P_t may be overwritten)
   uint64_t* o_final = pv_done + 2;               // every product done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_TMEM);
 
@@ -316,7 +389,8 @@ __global__ void __maxnreg__(96)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 8);  // one arrival per softmax warp of the tile
+      mbar_init(&p_full[2 * t], 8);  // one arrival per softmax warp of the tile
+      mbar_init(&p_full[2 * t + 1], 8);
       mbar_init(&pv_done[t], 1);
     }
     mbar_init(o_final, 1);
@@ -418,12 +492,8 @@ __global__ void __maxnreg__(96)
     if (lane == 0) {
       bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&k_full[0], 0);
       auto issue_s = [&](int t, int st) {  // S_t = Q_t K^T of the key tile in stage st
-#pragma unroll 2
-        for (int k = 0; k < KSTEPS; ++k) {
-          const uint32_t koff = (k >> 2) * Tr::PANEL + (k & 3) * 32;
-          umma_f16(tmem + Tr::colS(t), umma_desc(sQ + t * Tr::TILE + koff, 16, 1024),
-                   umma_desc(sK + st * Tr::TILE + koff, 16, 1024), IDESC_S, k > 0);
-        }
+        umma_ss_steps<KSTEPS>(tmem + Tr::colS(t), umma_desc(sQ + t * Tr::TILE, 16, 1024),
+                              umma_desc(sK + st * Tr::TILE, 16, 1024), IDESC_S);
         umma_commit(&s_full[t]);
       };
       if (ok) {
@@ -442,16 +512,24 @@ __global__ void __maxnreg__(96)
         }
         for (int t = 0; t < 2 && ok; ++t) {
           if (j >= nkv_t[t]) continue;
-          if (!mbar_wait_bounded(&p_full[t], j & 1)) {
+          // The first chunk of P (keys 0..31 of each half: K steps 0, 1, 4, 5)
+          // is multiplied while the softmax computes the second (2, 3, 6, 7).
+          bool got = true;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            if (!mbar_wait_bounded(&p_full[2 * t + c], j & 1)) {
+              got = false;
+              break;
+            }
+            tmem_fence_after_sync();
+            umma_ts_chunk(tmem + Tr::colO(t), tmem + Tr::colS(t) + 16 * c,
+                          umma_desc(sV + st * Tr::TILE + 2 * c * 2048, Tr::PANEL, 1024), IDESC_O,
+                          j > 0 || c > 0);
+          }
+          if (!got) {
             ok = false;
             break;
           }
-          tmem_fence_after_sync();
-#pragma unroll 2
-          for (int k = 0; k < PV_STEPS; ++k)
-            umma_f16_ts(tmem + Tr::colO(t), tmem + Tr::colS(t) + (k >> 2) * 64 + (k & 3) * 8,
-                        umma_desc(sV + st * Tr::TILE + k * 2048, Tr::PANEL, 1024), IDESC_O,
-                        j > 0 || k > 0);
           umma_commit(&pv_done[t]);
           if (j + 1 < nkv_t[t]) {
             if (!mbar_wait_bounded(&pv_done[t], j & 1)) {
@@ -567,12 +645,32 @@ __global__ void __maxnreg__(96)
         }
       }
       if (grow) m = mx;
+      // The key tile that reaches past the context: zero the V rows of the keys
+      // past it (whatever the stage held there, 0 x it must be 0).  The two
+      // threads of a row zero half of its 16-byte chunks each, in both query
+      // tiles' warps, before each tile's product (the two tiles' products may
+      // run in either order); later writes are zeros over zeros.
+      if (j * kPrefillTileN + kPrefillTileN > L) {
+        const int st = j % kPrefillStages;
+        ok = ok && mbar_wait_bounded(&v_full[st], (j / kPrefillStages) & 1);
+        if (ok && j * kPrefillTileN + r >= L) {
+          uint8_t* vrow = smem + Tr::OFF_V + st * Tr::TILE + r * 128;
+#pragma unroll
+          for (int pn = 0; pn < ND; ++pn)
+#pragma unroll
+            for (int ch = 4 * hf; ch < 4 * hf + 4; ++ch)
+              *reinterpret_cast<uint4*>(vrow + pn * Tr::PANEL + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
       // P = 2^(x - m) rounded to the input type, two keys per 32-bit column,
       // over the first 32 of this half's 64 score columns (the product's K
       // step k, keys 16 k .. 16 k + 15, reads columns 64 (k / 4) + 8 (k % 4));
       // the sum is over the rounded weights, in packed pairs of partial sums.
+      // Each chunk of 32 keys is handed to the tensor cores as soon as it is
+      // stored (p_full of the chunk); the second 32 scores are loaded while the
+      // first 32 are turned into P.
       float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      // The second 32 scores are loaded while the first 32 are turned into P.
       float xa[32], xb[32];
       tmem_ld32(cS, xa);
       tmem_wait_ld_tied(xa);
@@ -592,43 +690,33 @@ __global__ void __maxnreg__(96)
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int ee = c * 32 + e;
+          const float2 y = __ffma2_rn(make_float2(xv[e], xv[e + 1]), make_float2(sl, sl), make_float2(-m, -m));
+          // One pair in eight on the FMA pipe (keys 14, 15 of every 16: the same
+          // keys whatever the rows' mask, so that a row's weights do not depend
+          // on which other rows share its warp).
           float p0v, p1v;
-          if (masked) {
-            p0v = k0 + ee <= limit ? fast_exp2(xv[e] * sl - m) : 0.f;
-            p1v = k0 + ee + 1 <= limit ? fast_exp2(xv[e + 1] * sl - m) : 0.f;
+          if ((e >> 1) % 8 == 8 - 1) {
+            const float2 pe = exp2_poly2<T>(y);
+            p0v = pe.x;
+            p1v = pe.y;
           } else {
-            const float2 y = __ffma2_rn(make_float2(xv[e], xv[e + 1]), make_float2(sl, sl), make_float2(-m, -m));
             p0v = fast_exp2(y.x);
             p1v = fast_exp2(y.y);
+          }
+          if (masked) {
+            p0v = k0 + ee <= limit ? p0v : 0.f;
+            p1v = k0 + ee + 1 <= limit ? p1v : 0.f;
           }
           pk[e / 2] = pack2<T>(p0v, p1v);
           sum2[(e >> 1) & 1] = __fadd2_rn(sum2[(e >> 1) & 1], unpack2<T>(pk[e / 2]));
         }
         tmem_st16(cP + c * 16, pk);
+        tmem_wait_st();
+        tmem_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[2 * t + c]);
       }
       l += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
-      tmem_wait_st();
-      // The key tile that reaches past the context: zero the V rows of the keys
-      // past it (whatever the stage held there, 0 x it must be 0).  The two
-      // threads of a row zero half of its 16-byte chunks each, in both query
-      // tiles' warps, before each tile's product (the two tiles' products may
-      // run in either order); later writes are zeros over zeros.
-      if (j * kPrefillTileN + kPrefillTileN > L) {
-        const int st = j % kPrefillStages;
-        ok = ok && mbar_wait_bounded(&v_full[st], (j / kPrefillStages) & 1);
-        if (ok && j * kPrefillTileN + r >= L) {
-          uint8_t* vrow = smem + Tr::OFF_V + st * Tr::TILE + r * 128;
-#pragma unroll
-          for (int pn = 0; pn < ND; ++pn)
-#pragma unroll
-            for (int ch = 4 * hf; ch < 4 * hf + 4; ++ch)
-              *reinterpret_cast<uint4*>(vrow + pn * Tr::PANEL + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
-      }
-      tmem_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[t]);
     }
     // ---- epilogue: out = O / (l_half0 + l_half1), this half's columns
     ok = ok && (nkv_t[t] == 0 || mbar_wait_bounded(o_final, 0));

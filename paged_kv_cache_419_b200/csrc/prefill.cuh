@@ -49,8 +49,9 @@ struct PrefillTraits {
   static constexpr int OFF_V = OFF_K + kPrefillStages * TILE;
   static constexpr int OFF_RED = OFF_V + kPrefillStages * TILE;  // [2 tiles][2 halves][128] maxima, then sums
   static constexpr int OFF_BAR = OFF_RED + 8 * kPrefillTileM * 4;
-  // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], p_full[2], pv_done[2], o_final
-  static constexpr int NUM_BARS = 1 + 4 * kPrefillStages + 6 + 1;
+  // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], p_full[2][2] (per query
+  // tile and chunk of P), pv_done[2], o_final
+  static constexpr int NUM_BARS = 1 + 4 * kPrefillStages + 8 + 1;
   static constexpr int OFF_TMEM = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_TMEM + 16;
   // SMEM_USED + 1024 bytes of slack for the 1024-byte aligned base, and never
