@@ -1135,16 +1135,26 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
 // summed in shared memory (fixed order) at the end.  Statistics are read in
 // chunks of kMergeChunk partitions (one chunk for up to 64).
 // The grid launches while the decode grid still runs: each pair waits for the
-// decode grid's per-pair count, and its partials are read from L2.
+// decode grid's per-pair count, and its partials are read from L2.  A pair of
+// at most NREG * SLICES (and kMergeChunk) partitions, the common case, issues
+// every load at once when it becomes ready: the thread's partials into NREG
+// registers together with the statistics into shared memory, so the merge
+// costs one memory round trip after the pair's last partition, not one for the
+// statistics and more for the partials behind them.  The launcher picks the
+// smallest NREG in {2, 4, 8, 16} that covers the call's partition count: the
+// register footprint, and with it the number of merge CTAs an SM holds, follows
+// what the call needs.
 constexpr int kMergeThreads = 256;
 constexpr int kMergeChunk = 64;
+constexpr int kMergeMaxRegs = 16;  // largest NREG
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int NREG>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a) {
   constexpr int NV = G * D / 4;  // float4 groups of one pair's output
   static_assert(NV <= kMergeThreads && kMergeThreads % NV == 0, "whole slices");
   constexpr int SLICES = kMergeThreads / NV;
   constexpr int NWARP = kMergeThreads / 32;
+  constexpr int FAST_PARTS = NREG * SLICES < kMergeChunk ? NREG * SLICES : kMergeChunk;
   __shared__ float s_m[G][kMergeChunk], s_w[G][kMergeChunk];
   __shared__ float s_M[G], s_L[G];
   __shared__ float4 s_part[SLICES > 1 ? SLICES - 1 : 1][NV];
@@ -1180,69 +1190,121 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
       continue;
     }
 
-    // ---- M and L per head (warp g reduces head g; online across chunks)
-    float M = -CUDART_INF_F, L = 0.f;  // valid in warp g < G
-    for (int c0 = 0; c0 < np; c0 += kMergeChunk) {
-      const int cn = min(kMergeChunk, np - c0);
-      if (c0 > 0) __syncthreads();  // the previous chunk's s_m / s_w are no longer read
-      for (int i = tid; i < G * cn; i += kMergeThreads) {
-        const int g = i / cn, p = i % cn;
-        s_m[g][p] = __ldcg(a.tmp_m + cell(g, c0 + p));
-        s_w[g][p] = __ldcg(a.tmp_l + cell(g, c0 + p));  // l for now
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (np <= FAST_PARTS) {
+      const float* src = a.tmp_out + cell(vg, 0) * D + vd;
+      // ---- every load at once: partials p = slice, slice + SLICES, ... into
+      // registers, the statistics into shared memory
+      float4 part[NREG];
+#pragma unroll
+      for (int i = 0; i < NREG; ++i) {
+        const int p = slice + i * SLICES;
+        if (p < np) part[i] = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(p) * D));
+      }
+      for (int i = tid; i < G * np; i += kMergeThreads) {
+        const int g = i / np, p = i % np;
+        s_m[g][p] = __ldcg(a.tmp_m + cell(g, p));
+        s_w[g][p] = __ldcg(a.tmp_l + cell(g, p));  // l for now
       }
       __syncthreads();
+      // M and L per head (warp g reduces head g)
       for (int g = warp; g < G; g += NWARP) {
         float mc = -CUDART_INF_F;
-        for (int p = lane; p < cn; p += 32) mc = fmaxf(mc, s_m[g][p]);
+        for (int p = lane; p < np; p += 32) mc = fmaxf(mc, s_m[g][p]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
-        const float Mn = fmaxf(M, mc);
         float lc = 0.f;
-        for (int p = lane; p < cn; p += 32) lc += s_w[g][p] * fast_exp2(s_m[g][p] - Mn);
+        for (int p = lane; p < np; p += 32) lc += s_w[g][p] * fast_exp2(s_m[g][p] - mc);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) lc += __shfl_xor_sync(0xffffffffu, lc, o);
-        L = L * fast_exp2(M - Mn) + lc;  // M = -inf on the first chunk: the old sum is 0
-        M = Mn;
-      }
-    }
-    if (warp < G && lane == 0) {
-      s_M[warp] = M;
-      s_L[warp] = L;
-    }
-    __syncthreads();
-
-    // ---- weighted sum of the partial outputs
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = 0; c0 < np; c0 += kMergeChunk) {
-      const int cn = min(kMergeChunk, np - c0);
-      // One chunk: its statistics are still in s_m / s_w from the pass above.
-      // Several: that pass left the last chunk there, so every chunk (the first
-      // included) is loaded again.
-      if (np > kMergeChunk) {
-        if (c0 > 0) __syncthreads();  // the previous chunk's weights are no longer read
-        for (int i = tid; i < G * cn; i += kMergeThreads) {
-          const int g = i / cn, p = i % cn;
-          s_m[g][p] = __ldcg(a.tmp_m + cell(g, c0 + p));
-          s_w[g][p] = __ldcg(a.tmp_l + cell(g, c0 + p));
+        if (lane == 0) {
+          s_M[g] = mc;
+          s_L[g] = lc;
         }
-        __syncthreads();
       }
+      __syncthreads();
       // weights, in place of l: l_p 2^(m_p - M) / L
-      for (int i = tid; i < G * cn; i += kMergeThreads) {
-        const int g = i / cn, p = i % cn;
+      for (int i = tid; i < G * np; i += kMergeThreads) {
+        const int g = i / np, p = i % np;
         s_w[g][p] = s_w[g][p] * fast_exp2(s_m[g][p] - s_M[g]) / s_L[g];
       }
       __syncthreads();
       const float* wrow = s_w[vg];
-      const float* src = a.tmp_out + cell(vg, c0) * D + vd;
+#pragma unroll
+      for (int i = 0; i < NREG; ++i) {
+        const int p = slice + i * SLICES;
+        if (p < np) {
+          const float wp = wrow[p];
+          acc.x += wp * part[i].x;
+          acc.y += wp * part[i].y;
+          acc.z += wp * part[i].z;
+          acc.w += wp * part[i].w;
+        }
+      }
+    } else {
+      // ---- M and L per head (warp g reduces head g; online across chunks)
+      float M = -CUDART_INF_F, L = 0.f;  // valid in warp g < G
+      for (int c0 = 0; c0 < np; c0 += kMergeChunk) {
+        const int cn = min(kMergeChunk, np - c0);
+        if (c0 > 0) __syncthreads();  // the previous chunk's s_m / s_w are no longer read
+        for (int i = tid; i < G * cn; i += kMergeThreads) {
+          const int g = i / cn, p = i % cn;
+          s_m[g][p] = __ldcg(a.tmp_m + cell(g, c0 + p));
+          s_w[g][p] = __ldcg(a.tmp_l + cell(g, c0 + p));  // l for now
+        }
+        __syncthreads();
+        for (int g = warp; g < G; g += NWARP) {
+          float mc = -CUDART_INF_F;
+          for (int p = lane; p < cn; p += 32) mc = fmaxf(mc, s_m[g][p]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, o));
+          const float Mn = fmaxf(M, mc);
+          float lc = 0.f;
+          for (int p = lane; p < cn; p += 32) lc += s_w[g][p] * fast_exp2(s_m[g][p] - Mn);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) lc += __shfl_xor_sync(0xffffffffu, lc, o);
+          L = L * fast_exp2(M - Mn) + lc;  // M = -inf on the first chunk: the old sum is 0
+          M = Mn;
+        }
+      }
+      if (warp < G && lane == 0) {
+        s_M[warp] = M;
+        s_L[warp] = L;
+      }
+      __syncthreads();
+
+      // ---- weighted sum of the partial outputs
+      for (int c0 = 0; c0 < np; c0 += kMergeChunk) {
+        const int cn = min(kMergeChunk, np - c0);
+        // One chunk: its statistics are still in s_m / s_w from the pass above.
+        // Several: that pass left the last chunk there, so every chunk (the first
+        // included) is loaded again.
+        if (np > kMergeChunk) {
+          if (c0 > 0) __syncthreads();  // the previous chunk's weights are no longer read
+          for (int i = tid; i < G * cn; i += kMergeThreads) {
+            const int g = i / cn, p = i % cn;
+            s_m[g][p] = __ldcg(a.tmp_m + cell(g, c0 + p));
+            s_w[g][p] = __ldcg(a.tmp_l + cell(g, c0 + p));
+          }
+          __syncthreads();
+        }
+        // weights, in place of l: l_p 2^(m_p - M) / L
+        for (int i = tid; i < G * cn; i += kMergeThreads) {
+          const int g = i / cn, p = i % cn;
+          s_w[g][p] = s_w[g][p] * fast_exp2(s_m[g][p] - s_M[g]) / s_L[g];
+        }
+        __syncthreads();
+        const float* wrow = s_w[vg];
+        const float* src = a.tmp_out + cell(vg, c0) * D + vd;
 #pragma unroll 8
-      for (int p = slice; p < cn; p += SLICES) {
-        const float4 o = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(p) * D));
-        const float wp = wrow[p];
-        acc.x += wp * o.x;
-        acc.y += wp * o.y;
-        acc.z += wp * o.z;
-        acc.w += wp * o.w;
+        for (int p = slice; p < cn; p += SLICES) {
+          const float4 o = __ldcg(reinterpret_cast<const float4*>(src + static_cast<int64_t>(p) * D));
+          const float wp = wrow[p];
+          acc.x += wp * o.x;
+          acc.y += wp * o.y;
+          acc.z += wp * o.z;
+          acc.w += wp * o.w;
+        }
       }
     }
     // ---- slices 1.. hand their sums to slice 0, which adds them in order

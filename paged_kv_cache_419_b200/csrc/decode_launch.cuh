@@ -36,6 +36,39 @@ cudaError_t decode_grid(int num_sms, int* grid) {
   return cudaSuccess;
 }
 
+// Launch of the merge grid behind the decode grid (programmatic dependent
+// launch): at most one wave (the CTAs one SM holds of this instantiation, times
+// the SMs), so that no merge CTA waits for a slot behind one that is parked at
+// its final grid wait.
+template <typename T, int D, int G, int NREG>
+cudaError_t launch_merge(const DecodeArgs& a, int num_sms, cudaStream_t stream) {
+  static const int per_sm = [] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, merge_kernel<T, D, G, NREG>, kMergeThreads, 0) !=
+            cudaSuccess ||
+        n < 1) {
+      (void)cudaGetLastError();
+      n = 1;
+    }
+    return n;
+  }();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int64_t pairs = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
+  const int64_t want = static_cast<int64_t>(num_sms) * per_sm;
+  cfg.gridDim = dim3(static_cast<unsigned>(pairs < want ? pairs : want));
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, merge_kernel<T, D, G, NREG>, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <typename T, int D, int G, int B, bool PAGED>
 cudaError_t launch_decode_one(const DecodeArgs& args, const DecodeMaps& maps, int num_sms,
                               cudaStream_t stream) {
@@ -79,17 +112,15 @@ cudaError_t launch_decode_one(const DecodeArgs& args, const DecodeMaps& maps, in
   if (e != cudaSuccess || a.max_parts <= 1) return e;
   // Partition merge, also behind its predecessor: its CTAs become resident as
   // decode CTAs retire and merge each pair once the decode grid has published
-  // it.  At most one wave (8 CTAs of 256 threads per SM), so that no merge CTA
-  // waits for a slot behind one that is parked at its final grid wait.
-  const int64_t pairs = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
-  const int64_t want = static_cast<int64_t>(num_sms) * (2048 / kMergeThreads);
-  cfg.gridDim = dim3(static_cast<unsigned>(pairs < want ? pairs : want));
-  cfg.blockDim = dim3(kMergeThreads);
-  cfg.dynamicSmemBytes = 0;
-  e = cudaLaunchKernelEx(&cfg, merge_kernel<T, D, G>, a);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  // it.
+  constexpr int slices = kMergeThreads / (G * D / 4);
+  const int need = (a.max_parts + slices - 1) / slices;  // partials per thread for one load round
+  if (need <= 2) return launch_merge<T, D, G, 2>(a, num_sms, stream);
+  if (need <= 4) return launch_merge<T, D, G, 4>(a, num_sms, stream);
+  if (need <= 8) return launch_merge<T, D, G, 8>(a, num_sms, stream);
+  return launch_merge<T, D, G, kMergeMaxRegs>(a, num_sms, stream);
 }
+
 
 template <typename T, int D, int B, bool PAGED>
 cudaError_t launch_decode_group(const DecodeArgs& a, const DecodeMaps& m, int group, int num_sms,
