@@ -87,7 +87,9 @@ def parse_args(argv=None):
     ap.add_argument("--l2-flush", choices=["clean", "dirty"], default="clean",
                     help="L2 eviction before each timed step: 256 MiB write then read (clean) or write only")
     ap.add_argument("--block-size", type=int, default=0, help="override the workload's block size")
-    ap.add_argument("--partition", type=int, default=1024)
+    ap.add_argument("--partition", type=int, default=0,
+                    help="decode partition size; 0 (the library's default policy): 1024 tokens, balanced "
+                         "per call for batches with fewer (sequence, kv head) pairs than decode CTAs")
     ap.add_argument("--num-seqs", type=int, default=0,
                     help="smaller batch of the same length law, pool sized to fit (profiling)")
     ap.add_argument("--no-contiguous", action="store_true")
@@ -699,7 +701,9 @@ def run_ours(args, world, rank, local):
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
     flush = torch.zeros(2 * L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     n_pairs = int(b["pairs"].shape[0])
-    max_parts = math.ceil(w.max_blocks_per_seq * w.block_size / part)
+    # the library launches the merge when the workspace holds more than one
+    # partition per context; under the default policy it counts 512-token ones
+    max_parts = math.ceil(w.max_blocks_per_seq * w.block_size / (part or 512))
     # cache write; plan + decode (+ partition merge when contexts can span partitions)
     decode_launches = 2 + (1 if max_parts > 1 else 0)
     launches_per_step = 1 + decode_launches + (1 if n_pairs else 0)
@@ -815,7 +819,7 @@ def run_ours(args, world, rank, local):
                    "so no dirty lines remain)"
                    if args.l2_flush == "clean" else "flushed before every timed step (256 MiB write)")
                   + "; K/V read per step > L2",
-            "execution": mode, "partition_size": part,
+            "execution": mode, "partition_size": part if part else "0 (default policy)",
         },
         "seqs_per_s": round(seqs_per_s, 1),
         "pct_of_nominal_8tbs": round(100 * value / NOMINAL_HBM_GBS, 2),

@@ -865,9 +865,18 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
   // of the item before it.  Publishing each item as soon as it is written lets
   // the merge of a context start as soon as its last partition is done.
   // s_pub[kPubSlots] holds the count (thread 0 alone touches the list).
+  // The plan grid zeroes the counters while this grid already runs (under the
+  // round-robin schedule nothing else here waits for it), so thread 0 waits for
+  // the plan to complete before its first increment; by then it has, one item
+  // after the start.
   if (threadIdx.x == 0) s_pub[kPubSlots] = 0u;
+  bool plan_seen = false;  // thread 0: the plan grid has completed
   auto publish = [&]() {
     const uint32_t n = s_pub[kPubSlots];
+    if (n > 0 && !plan_seen) {
+      grid_dependency_wait();
+      plan_seen = true;
+    }
     for (uint32_t i = 0; i < n; ++i) red_add_release_gpu(&a.pair_done[s_pub[i]], 1u);
     s_pub[kPubSlots] = 0u;
   };
