@@ -910,13 +910,42 @@ def contiguous_compare(args, inp, b, ws, flush, part, device):
             "overhead": round(t_paged / t_contig - 1.0, 4), "outputs_identical": same}
 
 
+class WriteCombinedHost:
+    """Pinned, write-combined host memory (cudaHostAlloc with
+    cudaHostAllocWriteCombined) as a uint8 CPU tensor: the staging buffer for a
+    step's inputs.  The host only writes it; its stores bypass the CPU caches, so
+    the GPU's reads of it over the host link do not snoop freshly written lines
+    (a cached pinned buffer that the host has just written reads at ~15 GB/s on
+    these boxes, a write-combined one at ~50).  Freed with the object."""
+
+    def __init__(self, nbytes: int):
+        import ctypes
+        from cuda.bindings import runtime as rt
+
+        self._rt = rt
+        err, ptr = rt.cudaHostAlloc(nbytes, rt.cudaHostAllocWriteCombined)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaHostAlloc: {err}")
+        self.ptr = int(ptr)
+        arr = np.ctypeslib.as_array((ctypes.c_uint8 * nbytes).from_address(self.ptr))
+        self.tensor = torch.from_numpy(arr)
+
+    def __del__(self):
+        try:
+            self.tensor = None
+            self._rt.cudaFreeHost(self.ptr)
+        except Exception:
+            pass
+
+
 def e2e_run(args, inp, b, ws, part, nbytes, device):
     """The same step through the public API from pinned host buffers: host->device
     copies of the step's inputs (q, the new token's K/V, its slots, the block tables
     and context lengths), the cache write and decode, and the device->host read of
     the step's output, every step.
 
-    The inputs of a step cross the host link as one packed copy.  Steps are
+    The inputs of a step cross the host link as one packed copy, from a pinned,
+    write-combined staging buffer (the host writes it and never reads it).  Steps are
     pipelined the way a serving loop overlaps its transfers: inputs and
     outputs are double-buffered, the copies in run on one stream, the kernels on
     another and the copies out on a third, so step k+1's inputs and step k-1's
@@ -940,7 +969,14 @@ def e2e_run(args, inp, b, ws, part, nbytes, device):
         return {n: buf[offs[n]:offs[n] + b[n].numel() * b[n].element_size()].view(b[n].dtype).view(b[n].shape)
                 for n in names}
 
-    host_buf = [torch.zeros(pos, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    try:
+        staging = [WriteCombinedHost(pos) for _ in range(2)]
+        host_buf = [st.tensor for st in staging]
+        host_kind = "pinned, write-combined (cudaHostAllocWriteCombined)"
+    except Exception as e:  # no cuda-python: cached pinned memory
+        staging = None
+        host_buf = [torch.zeros(pos, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        host_kind = f"pinned (write-combined unavailable: {type(e).__name__})"
     for i in range(2):
         for n, t in views(host_buf[i]).items():
             t.copy_(b[n].cpu())
@@ -1018,7 +1054,34 @@ def e2e_run(args, inp, b, ws, part, nbytes, device):
     ms_max, _, _ = aggregate(ms, 0.0, 0.0, device)
     return {"value": round(nbytes["step"] / (ms_max * 1e-3) / 1e9, 1), "unit": "GB/s",
             "ms_per_step": round(ms_max, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "execution": mode}
+            "execution": mode, "input_staging": host_kind,
+            "host_link": host_link(copy_in, copy_out, s_in, s_out, h2d, d2h)}
+
+
+def host_link(copy_in, copy_out, s_in, s_out, h2d, d2h, reps=10):
+    """The step's own copies timed alone on their streams: the packed input copy
+    host->device, the output copy device->host, and both at once (the pipelined
+    steady state can go no faster than the slower direction)."""
+    def timed(fns):
+        evs = {s: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _, s in fns}
+        torch.cuda.synchronize()
+        for f, s in fns:
+            with torch.cuda.stream(s):
+                evs[s][0].record()
+                for r in range(reps):
+                    f(r % 2)
+                evs[s][1].record()
+        torch.cuda.synchronize()
+        return {s: evs[s][0].elapsed_time(evs[s][1]) / reps for _, s in fns}
+
+    t_in = timed([(copy_in, s_in)])[s_in]
+    t_out = timed([(copy_out, s_out)])[s_out]
+    both = timed([(copy_in, s_in), (copy_out, s_out)])
+    gbs = lambda nbytes, ms: round(nbytes / (ms * 1e-3) / 1e9, 1)
+    return {"h2d_gbs": gbs(h2d, t_in), "d2h_gbs": gbs(d2h, t_out),
+            "h2d_gbs_concurrent": gbs(h2d, both[s_in]), "d2h_gbs_concurrent": gbs(d2h, both[s_out]),
+            "h2d_us": round(1e3 * t_in, 1), "d2h_us": round(1e3 * t_out, 1),
+            "concurrent_us": round(1e3 * max(both.values()), 1)}
 
 
 # ------------------------------------------------------------------ cache ops alone
