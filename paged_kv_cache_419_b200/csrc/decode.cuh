@@ -31,7 +31,10 @@
 //    separately) and item slots over.
 //  * Consumer warp w owns tokens 16w..16w+15 of each stage with its own
 //    online-softmax state.  Scores: S^T = Q K^T as mma.sync m16n8k16 tiles (fp32
-//    accumulation), K fragments read with ldmatrix from the swizzled stage.  PV:
+//    accumulation), K fragments read with ldmatrix from the swizzled stage, Q
+//    fragments read from the item slot in every stage (rows padded against bank
+//    conflicts; held in registers for the whole item they made the consumers
+//    spill at their 128-register budget).  PV:
 //    O^T += V^T P^T, P^T taken from the score accumulators as they lie (as two
 //    16-bit parts, hi + lo, so that the weights keep about 16 significant bits),
 //    V^T read with transposing ldmatrix.
@@ -216,12 +219,17 @@ struct DecodeTraits {
   static constexpr int TILE_BYTES = ND * PANEL_BYTES;        // K (or V) of one stage
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int Q_BYTES = G * D * 2;
+  // Q slot in shared memory: one row per head, rows 16 bytes apart beyond
+  // their 2D bytes, so that the 8 heads' 32-bit reads of one instruction fall
+  // in different banks.
+  static constexpr int Q_PITCH = ROW_BYTES + 16;
+  static constexpr int Q_SLOT = G * Q_PITCH;
   static constexpr int ACC_PITCH = D + 4;                    // floats per head row of a merge slot
   static constexpr int HG = G <= 2 ? G : G / 2;              // heads per merge round
   static constexpr int MAX_TABLE = PAGED ? kMaxPartTokens / B : 4;  // table entries of one item
   // shared memory carve-up (bytes from a 1024-byte aligned base)
   static constexpr int OFF_Q = STAGES * STAGE_BYTES;
-  static constexpr int OFF_ACC = OFF_Q + kItemSlots * Q_BYTES;          // [warps][HG][ACC_PITCH] f32
+  static constexpr int OFF_ACC = OFF_Q + kItemSlots * Q_SLOT;          // [warps][HG][ACC_PITCH] f32
   static constexpr int OFF_REC = OFF_ACC + kConsumerWarps * HG * ACC_PITCH * 4;  // record slots
   static constexpr int OFF_TAB = OFF_REC + kRecSlots * kRecordBytes;    // 2 table buffers
   static constexpr int OFF_STAT = OFF_TAB + 2 * MAX_TABLE * 4;          // m, l per warp and head
@@ -707,7 +715,10 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
         mbar_arrive_expect_tx(&item_full[slot], Tr::Q_BYTES);
         const uint8_t* qsrc = static_cast<const uint8_t*>(a.q) +
                               (static_cast<int64_t>(s) * a.num_heads + kvh * G) * Tr::ROW_BYTES;
-        bulk_load(smem + Tr::OFF_Q + slot * Tr::Q_BYTES, qsrc, Tr::Q_BYTES, &item_full[slot]);
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          bulk_load(smem + Tr::OFF_Q + slot * Tr::Q_SLOT + g * Tr::Q_PITCH, qsrc + g * Tr::ROW_BYTES,
+                    Tr::ROW_BYTES, &item_full[slot]);
       }
       const int32_t* tab = s_tab + (k & 1) * Tr::MAX_TABLE;
       const int n_stages = (n_tok + TS - 1) / TS;
@@ -891,19 +902,10 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
     if (threadIdx.x == 0) publish();
     const int h0 = info.kvh * G;
 
-    // Q as the A operand: lane holds head `quad`, dims 16 ks + 2 qc (+1) and the
-    // same + 8 (zero for rows >= G).
-    uint32_t qa[KS][2];
-    {
-      const uint8_t* sq = smem + Tr::OFF_Q + slot * Tr::Q_BYTES + (quad * D + 2 * qc) * 2;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        qa[ks][0] = quad < G ? *reinterpret_cast<const uint32_t*>(sq + ks * 32) : 0u;
-        qa[ks][1] = quad < G ? *reinterpret_cast<const uint32_t*>(sq + ks * 32 + 16) : 0u;
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&item_empty[slot]);
+    // Q as the A operand, read from the item's Q slot in each stage (the slot is
+    // released after the item's last stage): lane holds head `quad`, dims
+    // 16 ks + 2 qc (+1) and the same + 8 (zero for rows >= G).
+    const uint8_t* sq = smem + Tr::OFF_Q + slot * Tr::Q_SLOT + quad * Tr::Q_PITCH + 2 * qc * 2;
 
     float m_run = -CUDART_INF_F;  // running max of head `quad` over this warp's tokens (base 2)
     float l_lane = 0.f;           // sum of this lane's probabilities of head `quad`
@@ -927,8 +929,12 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
         for (int nt = 0; nt < 2; ++nt) {
           uint32_t kb[4];
           ldmatrix_x4(kb, sK + (kp >> 1) * Tr::PANEL_BYTES + nt * 1024 + (k_lane ^ ((kp & 1) << 6)));
-          const uint32_t a0[4] = {qa[2 * kp][0], 0u, qa[2 * kp][1], 0u};
-          const uint32_t a1[4] = {qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u};
+          const uint32_t q00 = quad < G ? *reinterpret_cast<const uint32_t*>(sq + 2 * kp * 32) : 0u;
+          const uint32_t q01 = quad < G ? *reinterpret_cast<const uint32_t*>(sq + 2 * kp * 32 + 16) : 0u;
+          const uint32_t q10 = quad < G ? *reinterpret_cast<const uint32_t*>(sq + 2 * kp * 32 + 32) : 0u;
+          const uint32_t q11 = quad < G ? *reinterpret_cast<const uint32_t*>(sq + 2 * kp * 32 + 48) : 0u;
+          const uint32_t a0[4] = {q00, 0u, q01, 0u};
+          const uint32_t a1[4] = {q10, 0u, q11, 0u};
           mma_16816<T>(sacc[nt], a0, kb[0], kb[1]);
           mma_16816<T>(sacc[nt], a1, kb[2], kb[3]);
         }
@@ -1040,6 +1046,9 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
         ph ^= 1;
       }
     }
+    // every read of this item's Q slot is done: the producer may refill it
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&item_empty[slot]);
 
     // ---- combine the four warps: weight of warp w for head g is
     // 2^(m_w - M) / L with M = max_w m_w and L = sum_w 2^(m_w - M) l_w.
