@@ -80,9 +80,10 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["decode", "cache-ops", "prefill"], default="decode",
+    ap.add_argument("--op", choices=["decode", "cache-ops", "prefill", "shared"], default="decode",
                     help="cache-ops: time reshape_and_cache and copy_blocks alone at HBM-bound sizes; "
-                         "prefill: time the chunked-prefill batch alone")
+                         "prefill: time the chunked-prefill batch alone; shared: the shared-prefix "
+                         "decode batch alone")
     ap.add_argument("--workload", default="gqa8b", choices=["tiny", "mha13b", "gqa8b", "long"])
     ap.add_argument("--l2-flush", choices=["clean", "dirty"], default="clean",
                     help="L2 eviction before each timed step: 256 MiB write then read (clean) or write only")
@@ -1411,6 +1412,14 @@ def main(argv=None):
             device = torch.device("cuda", local)
             flush = torch.zeros(2 * L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
             print(json.dumps({"op": "prefill", **time_prefill(args, flush, device)}), flush=True)
+    elif args.op == "shared":
+        if rank == 0:
+            torch.cuda.set_device(local)
+            device = torch.device("cuda", local)
+            flush = torch.zeros(2 * L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+            peak, kind = measured_hbm_peak()
+            res = time_shared_decode(args, flush, device, peak, args.partition)
+            print(json.dumps({"op": "shared", "peak_gbs": peak, "peak_kind": kind, **res}), flush=True)
     else:
         run_ours(args, world, rank, local)
 
