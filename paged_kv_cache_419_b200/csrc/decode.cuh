@@ -95,7 +95,12 @@ struct DecodeArgs {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
-constexpr int kMaxPartTokens = 2048;
+constexpr int kMaxPartTokens = 2048;  // largest partition_size a caller may ask for
+// Block-table entries of one item (a shared-memory buffer of the producer): the
+// balanced policy's partitions reach kMaxTableEntries x block_size tokens
+// (2048 at 8-token blocks, 8192 at 32).
+constexpr int kMaxTableEntries = 256;
+constexpr int kMaxBalancedPartTokens = kMaxTableEntries * 32;
 constexpr int kPlanThreads = 1024;
 constexpr int kItemSlots = 2;
 constexpr int kRecSlots = 2;   // records of items k and k+1
@@ -124,24 +129,29 @@ __device__ __forceinline__ void partition_of(int L, int part_tokens, int& n, int
 // Balanced partitioning, for batches with fewer (sequence, kv head) pairs than
 // decode CTAs: there, fixed-size partitions leave a last wave of a few items
 // on an otherwise idle grid.  The batch's U = Hkv x sum L token-heads are cut
-// into about k x grid items of near-equal size, k = max(1, round(U / (grid x
-// 1024))): a context of L tokens gets n = round(L k grid / U) partitions (at
-// least ceil(L / kMaxPartTokens), at most max_parts and ceil(L / 64)) of equal
-// size rounded up to a multiple of 64 (the last one shorter).  Integer
+// into at most k x grid items of near-equal size (k whole waves of the grid):
+// k = round(U / (grid x 2048)), raised to the fewest waves whose items fit in
+// max_part tokens, and at least 1.  One item per CTA while a CTA's share stays
+// below ~3 K tokens: an item boundary costs a CTA about 2 us of its streaming
+// time, more than a finer split recovers in balance.  A context of L tokens
+// gets n = floor(L k grid / U) partitions (so the batch makes at most k x grid
+// items), at least ceil(L / max_part), at most max_parts and ceil(L / 64), of
+// equal size rounded up to a multiple of 64 (the last one shorter).  Integer
 // arithmetic only: the plan, the statically started CTAs and the merge agree.
 __device__ __forceinline__ void partition_balanced(int L, unsigned long long U, int grid,
-                                                   int max_parts, int& n, int& size) {
+                                                   int max_parts, int max_part, int& n, int& size) {
   if (L <= 0 || U == 0) {
     n = 1;
     size = L > 0 ? L : 0;
     return;
   }
-  const long long g = grid;
-  long long k = (static_cast<long long>(U) + g * 512) / (g * 1024);
+  const long long g = grid, uu = static_cast<long long>(U);
+  long long k = (uu + g * 1024) / (g * 2048);
+  const long long k_fit = (uu + g * max_part - 1) / (g * max_part);
+  if (k < k_fit) k = k_fit;
   if (k < 1) k = 1;
-  long long nn = (static_cast<long long>(L) * k * g + static_cast<long long>(U / 2)) /
-                 static_cast<long long>(U);
-  const long long lo = (L + kMaxPartTokens - 1) / kMaxPartTokens;
+  long long nn = static_cast<long long>(L) * k * g / uu;
+  const long long lo = (L + max_part - 1) / max_part;
   const long long hi = min(static_cast<long long>(max_parts), static_cast<long long>((L + 63) / 64));
   nn = nn < lo ? lo : nn;
   nn = nn > hi ? hi : nn;
@@ -155,7 +165,7 @@ __device__ __forceinline__ void partition_balanced(int L, unsigned long long U, 
 __device__ __forceinline__ void partition_for(int L, const DecodeArgs& a, unsigned long long U,
                                               int& n, int& size) {
   if (a.balanced)
-    partition_balanced(L, U, a.grid_ctas, a.max_parts, n, size);
+    partition_balanced(L, U, a.grid_ctas, a.max_parts, a.part_tokens, n, size);
   else
     partition_of(L, a.part_tokens, n, size);
 }
@@ -226,7 +236,7 @@ struct DecodeTraits {
   static constexpr int Q_SLOT = G * Q_PITCH;
   static constexpr int ACC_PITCH = D + 4;                    // floats per head row of a merge slot
   static constexpr int HG = G <= 2 ? G : G / 2;              // heads per merge round
-  static constexpr int MAX_TABLE = PAGED ? kMaxPartTokens / B : 4;  // table entries of one item
+  static constexpr int MAX_TABLE = PAGED ? kMaxTableEntries : 4;  // table entries of one item
   // shared memory carve-up (bytes from a 1024-byte aligned base)
   static constexpr int OFF_Q = STAGES * STAGE_BYTES;
   static constexpr int OFF_ACC = OFF_Q + kItemSlots * Q_SLOT;          // [warps][HG][ACC_PITCH] f32
@@ -282,7 +292,7 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
   grid_dependency_wait();
   allow_dependent_launch();
   const int n_static = static_first_seqs(a.num_seqs, a.grid_ctas, a.num_kv_heads);
-  constexpr int kMaxClasses = kMaxPartTokens / 32 + 2;
+  constexpr int kMaxClasses = kMaxBalancedPartTokens / 32 + 2;
   __shared__ uint32_t count[kMaxClasses];
   __shared__ uint32_t cursor[kMaxClasses];
   __shared__ uint32_t total, n_multi, n_wide;
