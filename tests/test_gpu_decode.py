@@ -257,6 +257,23 @@ def test_shapes_and_ragged_lengths(dtype, D, G, bs):
     run_and_compare(inp, partition_size=512)
 
 
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_ragged_lengths_default_policy(bs):
+    """The ragged lengths at the default partition policy: 36 (sequence, kv head)
+    pairs, fewer than decode CTAs, so partitions are balanced per call under the
+    round-robin schedule (their largest size depends on the block size)."""
+    Hkv, G = 2, 4
+    lens = np.array([1, 2, 7, 8, 9, 15, 16, 17, 31, 32, 33, 63, 64, 65, 511, 512, 513, 9030],
+                    np.int32)
+    max_blocks = -(-int(lens.max()) // bs) + 1
+    w = wl.Workload("edge", 8, len(lens), G * Hkv, Hkv, 128, bs, max_blocks * len(lens) + 5, wl.BF16,
+                    max_blocks, 1.0 / np.sqrt(128), lengths=("uniform", 1, 2))
+    inp = wl.make_decode_inputs(w, lengths=lens)
+    out, ref, err, b, _ = run_and_compare(inp, partition_size=0)
+    st = rounded_oracle_stats(out, ref, wl.BF16)
+    assert st["within_1_ulp"] >= 0.99, st
+
+
 def test_zero_length_context_writes_zeros():
     lens = np.array([0, 5, 0, 40], np.int32)
     w = wl.Workload("zero", 8, 4, 8, 2, 128, 16, 64, wl.BF16, 4, 0.088, lengths=("uniform", 1, 2))
