@@ -138,6 +138,15 @@ __device__ __forceinline__ void partition_of(int L, int part_tokens, int& n, int
 // items), at least ceil(L / max_part), at most max_parts and ceil(L / 64), of
 // equal size rounded up to a multiple of 64 (the last one shorter).  Integer
 // arithmetic only: the plan, the statically started CTAs and the merge agree.
+// k of the balanced rule: round(U / (grid x 2048)), raised to the fewest waves
+// whose items fit in max_part tokens, at least 1.
+__device__ __forceinline__ long long balanced_waves(long long uu, long long g, long long max_part) {
+  long long k = (uu + g * 1024) / (g * 2048);
+  const long long k_fit = (uu + g * max_part - 1) / (g * max_part);
+  if (k < k_fit) k = k_fit;
+  return k < 1 ? 1 : k;
+}
+
 __device__ __forceinline__ void partition_balanced(int L, unsigned long long U, int grid,
                                                    int max_parts, int max_part, int& n, int& size) {
   if (L <= 0 || U == 0) {
@@ -146,10 +155,7 @@ __device__ __forceinline__ void partition_balanced(int L, unsigned long long U, 
     return;
   }
   const long long g = grid, uu = static_cast<long long>(U);
-  long long k = (uu + g * 1024) / (g * 2048);
-  const long long k_fit = (uu + g * max_part - 1) / (g * max_part);
-  if (k < k_fit) k = k_fit;
-  if (k < 1) k = 1;
+  const long long k = balanced_waves(uu, g, max_part);
   long long nn = static_cast<long long>(L) * k * g / uu;
   const long long lo = (L + max_part - 1) / max_part;
   const long long hi = min(static_cast<long long>(max_parts), static_cast<long long>((L + 63) / 64));
@@ -168,6 +174,53 @@ __device__ __forceinline__ void partition_for(int L, const DecodeArgs& a, unsign
     partition_balanced(L, U, a.grid_ctas, a.max_parts, a.part_tokens, n, size);
   else
     partition_of(L, a.part_tokens, n, size);
+}
+
+// Partitions of the round-robin schedule, two sizes.  With one static item
+// per CTA the grid's finishing times spread with the SMs' streaming rates (per
+// SM mean item time 55-70 us on the long batch), and the last CTAs stream alone.
+// So each context is cut into "big" partitions of p_big ~ 7/8 of a CTA's
+// share, U / (k grid) token-heads, rounded up to a multiple of 64 (at most
+// floor(7/8 L / p_big) of them, so the batch has at most k x grid big items,
+// handed out round-robin), followed by "small" partitions of p_small ~ p_big / 4
+// for the rest, which CTAs claim one at a time from a counter near the end of
+// their current item: the fast SMs take more of them.  The split applies when
+// p_small would reach 256 tokens; then p_small grows if needed so that a
+// context keeps within max_parts partitions.  Otherwise, and off the round-robin
+// schedule, every partition is a big one by the balanced rule (n_big = n).
+// Partition p < n_big covers tokens [p p_big, (p + 1) p_big); partition
+// n_big + q covers [n_big p_big + q p_small, ...), the last one shorter.  Per
+// sequence and from U alone: the plan, the decode grid and the merge agree.
+constexpr int kBigNum = 14, kBigDen = 16, kSmallDiv = 4, kMinSmallTokens = 256;
+constexpr int kClaimLead = 3;
+__device__ __forceinline__ void partition_rr(int L, const DecodeArgs& a, unsigned long long U,
+                                             int& n_big, int& n, int& p_big, int& p_small) {
+  const long long g = a.grid_ctas, uu = static_cast<long long>(U);
+  const long long k = uu > 0 ? balanced_waves(uu, g, a.part_tokens) : 1;
+  long long pb = uu > 0 ? (uu * kBigNum + k * g * kBigDen - 1) / (k * g * kBigDen) : 0;
+  pb = (pb + kStageTokens - 1) & ~static_cast<long long>(kStageTokens - 1);
+  if (pb > a.part_tokens) pb = a.part_tokens;
+  long long ps = (pb / kSmallDiv + kStageTokens - 1) & ~static_cast<long long>(kStageTokens - 1);
+  if (L <= 0 || uu == 0 || ps < kMinSmallTokens) {  // one size: the balanced rule
+    int size = 0;
+    partition_balanced(L, U, a.grid_ctas, a.max_parts, a.part_tokens, n, size);
+    n_big = n;
+    p_big = p_small = size;
+    return;
+  }
+  const long long nb = static_cast<long long>(L) * kBigNum / (kBigDen * pb);
+  const long long rest = L - nb * pb;
+  long long ns = (rest + ps - 1) / ps;
+  if (nb + ns > a.max_parts) {  // fewer, larger small partitions (max_parts > nb here)
+    const long long room = a.max_parts - nb > 0 ? a.max_parts - nb : 1;
+    ps = (((rest + room - 1) / room) + kStageTokens - 1) & ~static_cast<long long>(kStageTokens - 1);
+    ns = (rest + ps - 1) / ps;
+  }
+  n_big = static_cast<int>(nb);
+  n = static_cast<int>(nb + (ns > 0 ? ns : 0));
+  if (n < 1) n = 1;  // L > 0 here, so rest > 0 when nb = 0
+  p_big = static_cast<int>(pb);
+  p_small = static_cast<int>(ps);
 }
 
 // Round-robin schedule: under the balanced policy the items are near-equal by
@@ -325,14 +378,19 @@ static __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const DecodeA
     const int L = clamp_len(raw, a.max_ctx);
     if (cached) s_len[s] = L;
     int n, size;
-    partition_for(L, a, U, n, size);
-    // listed partitions: skip .. n-1 (partition 0 of a static sequence is not
-    // listed); partitions below n-1 have `size` tokens, the last one the rest
-    const int skip = s < n_static ? 1 : 0;
-    const int n_full = n - 1 - skip;
-    if (n_full > 0) atomicAdd(&count[size_class(size)], static_cast<uint32_t>(n_full));
-    if (n - 1 >= skip) atomicAdd(&count[size_class(L - (n - 1) * size)], 1u);
-    atomicAdd(&total, static_cast<uint32_t>(n - skip));
+    if (round_robin(a)) {  // no list: only the merge's sequences and counters
+      int n_big, p_big, p_small;
+      partition_rr(L, a, U, n_big, n, p_big, p_small);
+    } else {
+      partition_for(L, a, U, n, size);
+      // listed partitions: skip .. n-1 (partition 0 of a static sequence is not
+      // listed); partitions below n-1 have `size` tokens, the last one the rest
+      const int skip = s < n_static ? 1 : 0;
+      const int n_full = n - 1 - skip;
+      if (n_full > 0) atomicAdd(&count[size_class(size)], static_cast<uint32_t>(n_full));
+      if (n - 1 >= skip) atomicAdd(&count[size_class(L - (n - 1) * size)], 1u);
+      atomicAdd(&total, static_cast<uint32_t>(n - skip));
+    }
     if (n > 1) {
       a.merge_seqs[atomicAdd(&n_multi, 1u)] = s;
       for (int h = 0; h < a.num_kv_heads; ++h) a.pair_done[s * a.num_kv_heads + h] = 0u;
@@ -564,31 +622,42 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
 
     bool ok = true;
     const bool rr = round_robin(a);
-    // Round-robin schedule (see round_robin): lane l describes sequences l and
-    // l + 32: length, partitions, partition size and the index of its first
-    // (sequence, partition) pair in the enumeration.
-    int rr_L[2] = {0, 0}, rr_n[2] = {0, 0}, rr_size[2] = {0, 0}, rr_first[2] = {0, 0};
+    // Round-robin schedule (see round_robin and partition_rr): lane l describes
+    // sequences l and l + 32: length, big and small partition counts, and the
+    // index of its first big and first small (sequence, partition) pair in the
+    // enumeration, all big pairs first.  Items (pair, kv head) below
+    // n_items_big are taken round-robin, the rest from the claim counter.
+    int rr_L[2] = {0, 0}, rr_nb[2] = {0, 0}, rr_ns[2] = {0, 0}, rr_fb[2] = {0, 0}, rr_fs[2] = {0, 0};
+    int rr_pb[2] = {0, 0}, rr_ps[2] = {0, 0};  // big and small partition sizes
+    uint32_t n_items_big = 0;
     auto rr_record = [&](uint32_t j, uint32_t idx) {  // whole warp; record of item idx -> slot j % 2
-      const int pair = static_cast<int>(idx / Hkv);
+      const bool big = idx < n_items_big;
+      const int pair = static_cast<int>((big ? idx : idx - n_items_big) / Hkv);
       int own = -1;
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        if (pair >= rr_first[h] && pair < rr_first[h] + rr_n[h]) own = h;
+      for (int h = 0; h < 2; ++h) {
+        const int f = big ? rr_fb[h] : rr_fs[h], c = big ? rr_nb[h] : rr_ns[h];
+        if (pair >= f && pair < f + c) own = h;
+      }
       const uint32_t mask = __ballot_sync(0xffffffffu, own >= 0);
       const int src = __ffs(mask) - 1;  // exactly one lane owns the pair
       const int h = __shfl_sync(0xffffffffu, own, src);
       const int L = __shfl_sync(0xffffffffu, h ? rr_L[1] : rr_L[0], src);
-      const int n = __shfl_sync(0xffffffffu, h ? rr_n[1] : rr_n[0], src);
-      const int size = __shfl_sync(0xffffffffu, h ? rr_size[1] : rr_size[0], src);
-      const int first = __shfl_sync(0xffffffffu, h ? rr_first[1] : rr_first[0], src);
+      const int nb = __shfl_sync(0xffffffffu, h ? rr_nb[1] : rr_nb[0], src);
+      const int ns = __shfl_sync(0xffffffffu, h ? rr_ns[1] : rr_ns[0], src);
+      const int first = __shfl_sync(0xffffffffu, big ? (h ? rr_fb[1] : rr_fb[0]) : (h ? rr_fs[1] : rr_fs[0]), src);
+      const int pbig = __shfl_sync(0xffffffffu, h ? rr_pb[1] : rr_pb[0], src);
+      const int psmall = __shfl_sync(0xffffffffu, h ? rr_ps[1] : rr_ps[0], src);
       if (lane == 0) {
         int32_t* r = reinterpret_cast<int32_t*>(smem + Tr::OFF_REC + (j & 1) * kRecordBytes);
-        const int p = pair - first, t_begin = p * size;
+        const int q = pair - first;
+        const int p = big ? q : nb + q;
+        const int t_begin = big ? q * pbig : nb * pbig + q * psmall;
         r[0] = src + 32 * h;
         r[1] = p;
-        r[2] = n;
+        r[2] = nb + ns;
         r[3] = t_begin;
-        r[4] = min(size, L - t_begin);
+        r[4] = min(big ? pbig : psmall, L - t_begin);
         r[5] = L;
         // complete the slot's barrier phase as a copy would have
         mbar_arrive(&rec_bar[j & 1]);
@@ -606,38 +675,55 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) U += __shfl_xor_sync(0xffffffffu, U, o);
       U *= static_cast<unsigned long long>(a.num_kv_heads);
-      int n_lane[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int t = lane + 32 * h;
-        partition_for(rr_L[h], a, U, rr_n[h], rr_size[h]);
-        n_lane[h] = t < a.num_seqs ? rr_n[h] : 0;
+        int nb, n, pb, ps;
+        partition_rr(rr_L[h], a, U, nb, n, pb, ps);
+        rr_nb[h] = t < a.num_seqs ? nb : 0;  // 0 past the last sequence: no pair maps there
+        rr_ns[h] = t < a.num_seqs ? n - nb : 0;
+        rr_pb[h] = pb;
+        rr_ps[h] = ps;
       }
-      // exclusive prefix of the partition counts in sequence order
+      // exclusive prefixes of the big and small counts in sequence order
       // (sequences 0..31 on lanes 0..31, then 32..63)
-      int incl0 = n_lane[0], incl1 = n_lane[1];
+      int b0 = rr_nb[0], b1 = rr_nb[1], s0 = rr_ns[0], s1 = rr_ns[1];
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int a0 = __shfl_up_sync(0xffffffffu, incl0, o);
-        const int a1 = __shfl_up_sync(0xffffffffu, incl1, o);
+        const int x0 = __shfl_up_sync(0xffffffffu, b0, o), x1 = __shfl_up_sync(0xffffffffu, b1, o);
+        const int y0 = __shfl_up_sync(0xffffffffu, s0, o), y1 = __shfl_up_sync(0xffffffffu, s1, o);
         if (lane >= o) {
-          incl0 += a0;
-          incl1 += a1;
+          b0 += x0;
+          b1 += x1;
+          s0 += y0;
+          s1 += y1;
         }
       }
-      const int total0 = __shfl_sync(0xffffffffu, incl0, 31);
-      rr_first[0] = incl0 - n_lane[0];
-      rr_first[1] = total0 + incl1 - n_lane[1];
-      rr_n[0] = n_lane[0];  // 0 past the last sequence: no pair maps there
-      rr_n[1] = n_lane[1];
-      n_items = static_cast<uint32_t>(total0 + __shfl_sync(0xffffffffu, incl1, 31)) * Hkv;
+      const int tb0 = __shfl_sync(0xffffffffu, b0, 31), ts0 = __shfl_sync(0xffffffffu, s0, 31);
+      rr_fb[0] = b0 - rr_nb[0];
+      rr_fb[1] = tb0 + b1 - rr_nb[1];
+      rr_fs[0] = s0 - rr_ns[0];
+      rr_fs[1] = ts0 + s1 - rr_ns[1];
+      const uint32_t big_pairs = static_cast<uint32_t>(tb0 + __shfl_sync(0xffffffffu, b1, 31));
+      const uint32_t small_pairs = static_cast<uint32_t>(ts0 + __shfl_sync(0xffffffffu, s1, 31));
+      n_items_big = big_pairs * Hkv;
+      n_items = (big_pairs + small_pairs) * Hkv;
     }
+    // Next item under the round-robin schedule: the CTA's next big item, or a
+    // claimed small one (the plan zeroed the claim counter: wait for it first).
+    auto rr_next = [&](uint32_t after_big) {
+      if (after_big < n_items_big) return after_big;
+      plan_wait();
+      uint32_t c = 0;
+      if (lane == 0) c = n_items_big + atomicAdd(a.work, 1u);
+      return __shfl_sync(0xffffffffu, c, 0);
+    };
     const bool static_first =
         !rr &&
         blockIdx.x < static_cast<uint32_t>(static_first_seqs(a.num_seqs, a.grid_ctas, a.num_kv_heads)) * Hkv;
     uint32_t cur = 0;  // list index of the current item (items after a static first one)
     if (rr) {
-      cur = blockIdx.x;
+      cur = rr_next(blockIdx.x);
       if (cur < n_items) {
         rr_record(0, cur);
         ok = wait_record(0);
@@ -738,7 +824,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
         if (step == 0) {
           if (!rr) plan_wait();
           if (rr) {
-            nxt = cur + gridDim.x;
+            nxt = rr_next(cur < n_items_big ? cur + gridDim.x : n_items_big);
             if (nxt < n_items) rr_record(k + 1, nxt);
           } else {
             if (lane == 0) {
@@ -756,6 +842,10 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
         }
         return true;
       };
+      // A claimed next item is claimed near the end of this one (kClaimLead
+      // stages before it), so that a CTA takes more items the faster it streams;
+      // a listed or round-robin one is prepared at once.
+      const int prep_at = rr && cur + gridDim.x >= n_items_big ? max(0, n_stages - kClaimLead) : 0;
       for (int i = 0; i < n_stages; ++i) {
         const int t0 = i * TS;  // relative to the partition start (block aligned)
         // Boxes: full chunks of CH rows, the ragged end in 8-row boxes, so a
@@ -817,7 +907,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (G <= 4 ? 3 : 2))
           st = 0;
           ph ^= 1;
         }
-        if (i <= 1 && !prepare_next(i)) {
+        if ((i == prep_at || i == prep_at + 1) && !prepare_next(i - prep_at)) {
           ok = false;
           break;
         }
@@ -1200,7 +1290,12 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const DecodeArgs a
     const int kvh = static_cast<int>(t % Hkv);
     const int h0 = kvh * G;
     int np, psize;
-    partition_for(clamp_len(a.lens[s], a.max_ctx), a, U, np, psize);
+    if (round_robin(a)) {
+      int n_big, p_small;
+      partition_rr(clamp_len(a.lens[s], a.max_ctx), a, U, n_big, np, psize, p_small);
+    } else {
+      partition_for(clamp_len(a.lens[s], a.max_ctx), a, U, np, psize);
+    }
     const int64_t base0 = (static_cast<int64_t>(s) * a.num_heads + h0) * a.max_parts;
     auto cell = [&](int g, int p) { return base0 + static_cast<int64_t>(g) * a.max_parts + p; };
     // Wait (bounded) until the decode grid has published all np partitions of

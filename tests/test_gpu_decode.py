@@ -149,6 +149,35 @@ def test_default_policy_balances_few_long_contexts():
     assert torch.equal(out_c, out)
 
 
+def test_default_policy_two_size_partitions():
+    """A few sequences with about a million (token, kv head) pairs in all: at
+    the default size the long contexts are cut into large partitions of about
+    7/8 of a CTA's share, which CTAs take in turn, and a tail of quarter-size
+    partitions that CTAs claim as they finish.  The lengths give contexts made
+    only of large items plus a tail (the 24K-32K ones), of both (7000), and of
+    tail items alone, down to a single ragged one (1, 200, 1500): every element
+    against the oracle, and bit-identical on a repeat (the claimed items land
+    on different CTAs from call to call, but each partition's partial result
+    does not depend on which CTA computed it)."""
+    B = _bin()
+    lens = np.array([32768, 30001, 1, 24000, 200, 1500, 7000, 29999], np.int32)
+    bs = 32
+    max_blocks = -(-int(lens.max()) // bs)
+    w = wl.Workload("two-size", 12, len(lens), 32, 8, 128, bs, max_blocks * len(lens) + 3, wl.BF16,
+                    max_blocks, 1.0 / np.sqrt(128), lengths=("uniform", 1, 2))
+    inp = wl.make_decode_inputs(w, lengths=lens)
+    out, ref, err, b, _ = run_and_compare(inp, check_cache=False)
+    st = rounded_oracle_stats(out, ref, wl.BF16)
+    print(f"two-size partitions, default policy: max-abs {err:.3e}, vs rounded oracle {st}")
+    assert st["within_1_ulp"] >= 0.99, st
+    out2 = torch.empty_like(out)
+    for _ in range(3):
+        B.paged_attention_decode(out2, b.q, b.k_cache, b.v_cache, b.tables, b.lens, w.scale)
+        torch.cuda.synchronize()
+        assert B.device_error() == 0
+        assert torch.equal(out2, out)
+
+
 # ------------------------------------------------------------ normalisation pins
 # Contexts that run as one stage, as a ragged stage, and across 2, 3 and 5
 # partitions of the default 1024 tokens (so both normalisers run: the one at the
