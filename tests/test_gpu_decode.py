@@ -178,6 +178,38 @@ def test_default_policy_two_size_partitions():
         assert torch.equal(out2, out)
 
 
+@pytest.mark.parametrize("S,Hq,Hkv", [(64, 16, 4), (65, 16, 4), (120, 8, 2), (200, 8, 1)])
+def test_default_policy_balanced_partitions_many_sequences(S, Hq, Hkv):
+    """Fewer (sequence, kv head) pairs than decode CTAs, so the partitions are
+    balanced per call at the default size, with many sequences.  64 is the
+    most the round-robin schedule takes (every producer lane holds two
+    sequences), and this batch is large enough for its two partition sizes;
+    from 65 sequences on, the first partition of the first sequences runs
+    statically and the rest comes from the plan's largest-first list.  Ragged
+    lengths from 1 token to a few thousand, with some long contexts that span
+    many partitions; every element against the oracle, and bit-identical on a
+    repeat."""
+    B = _bin()
+    rng = np.random.default_rng(31 + S)
+    lens = rng.integers(1, 3000, size=S).astype(np.int32)
+    lens[rng.choice(S, size=4, replace=False)] = [6000, 7777, 9000, 8191]
+    bs = 16
+    max_blocks = -(-int(lens.max()) // bs)
+    w = wl.Workload("balanced-list", 12, S, Hq, Hkv, 128, bs, int(np.sum(-(-lens // bs))) + S + 8,
+                    wl.BF16, max_blocks, 1.0 / np.sqrt(128), lengths=("uniform", 1, 2))
+    inp = wl.make_decode_inputs(w, lengths=lens)
+    out, ref, err, b, _ = run_and_compare(inp, check_cache=False)
+    st = rounded_oracle_stats(out, ref, wl.BF16)
+    print(f"balanced partitions S={S} Hkv={Hkv}: max-abs {err:.3e}, vs rounded oracle {st}")
+    assert st["within_1_ulp"] >= 0.99, st
+    out2 = torch.empty_like(out)
+    for _ in range(2):
+        B.paged_attention_decode(out2, b.q, b.k_cache, b.v_cache, b.tables, b.lens, w.scale)
+        torch.cuda.synchronize()
+        assert B.device_error() == 0
+        assert torch.equal(out2, out)
+
+
 # ------------------------------------------------------------ normalisation pins
 # Contexts that run as one stage, as a ragged stage, and across 2, 3 and 5
 # partitions of the default 1024 tokens (so both normalisers run: the one at the
