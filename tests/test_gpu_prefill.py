@@ -82,6 +82,8 @@ def oracle_prefill_batch(inp, poison=True, rows=None):
     for s in range(S):
         a = int(inp.query_start[s])
         p0 = int(inp.cached[s])
+        if int(inp.chunk[s]) == 0:
+            continue  # no new tokens: no rows
         if rows is None:
             out[a:a + int(inp.chunk[s])] = oracle.paged_prefill(
                 inp.q[a:a + int(inp.chunk[s])], kc, vc, tables[s], p0, w.scale, w.num_kv_heads,
@@ -240,6 +242,34 @@ def test_prefill_bad_lengths_set_flags_without_faulting():
                     torch.from_numpy(lens).cuda(), w.scale, 60)
     torch.cuda.synchronize()
     assert B.device_error() & B.DEVERR_CONTEXT_LEN
+
+
+def test_prefill_odd_group_empty_chunk_and_spare_row_tiles():
+    """Three query heads per kv head (an odd group: each CTA takes two
+    consecutive 128-row tiles of one head), a sequence with no new tokens in the
+    batch, and max_query_len above the longest chunk, so the grid has row tiles
+    with no rows.  Every row of every chunk against the oracle; the q rows past
+    the last chunk belong to no sequence and their output rows stay untouched."""
+    B = _bin()
+    cached, chunk = [5, 0, 64, 17, 200], [0, 1, 129, 300, 45]
+    mb = -(-max(c + t for c, t in zip(cached, chunk)) // 16) + 1
+    w = _workload(wl.BF16, 128, 3, 16, frames=len(cached) * mb + 7, max_blocks=mb, seed=97)
+    inp = wl.make_prefill_inputs(w, cached=cached, chunk=chunk)
+    kc, vc, table, lens = gpu_prefill_batch(inp)
+    spare = 9
+    q = to_dev(inp.q, w.dtype)
+    q = torch.cat([q, torch.zeros((spare,) + tuple(q.shape[1:]), dtype=q.dtype, device=q.device)])
+    out = torch.full_like(q, float("nan"))
+    B.paged_prefill(out, q, kc, vc, torch.from_numpy(table).cuda(),
+                    torch.from_numpy(inp.query_start).cuda(), torch.from_numpy(lens).cuda(), w.scale, 512)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    rows = int(inp.query_start[-1])
+    assert torch.isnan(out[rows:]).all()
+    ref, tables = oracle_prefill_batch(inp)
+    assert np.array_equal(tables, table)
+    assert torch.isfinite(out[:rows]).all()
+    assert_within_tolerance(out[:rows], ref, wl.BF16)
 
 
 def test_prefill_full_size_batch_sampled_rows():
