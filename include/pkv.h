@@ -101,6 +101,28 @@ pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t str
  */
 pkv_status pkv_test_set_merge_wait(uint64_t limit_ns, uint32_t extra);
 
+/*
+ * Test hook for the partition rules (host only, no GPU needed).  How a decode
+ * call cuts each context into partitions is not fixed by the pages (any cut
+ * gives the same result within the tolerance; it sets the work split).  This
+ * runs the same code the decode, planning and merge kernels run, for a call
+ * with these arguments on a decode grid of grid_ctas CTAs (444 for the G <= 4
+ * kernels on a 148-SM B200, 296 for G = 8).
+ *   context_lens  host int32 [num_seqs], clamped to [0, max_context_len] as the
+ *                 kernels do
+ *   max_context_len, block_size, partition_size  as in the decode call
+ *                 (max_context_len = max_blocks_per_seq * block_size)
+ *   n_parts, n_big, p_big, p_small  host int32 [num_seqs], written: context s
+ *                 has n_parts partitions, the first n_big of p_big tokens, then
+ *                 p_small tokens each, the last one shorter (a single-size rule
+ *                 gives n_big = n_parts and p_big = p_small).
+ * PKV_EINVAL for a bad argument or an unsupported partition_size.
+ */
+pkv_status pkv_test_partitions(const int32_t* context_lens, int32_t num_seqs, int32_t num_kv_heads,
+                               int32_t max_context_len, int32_t block_size, int32_t partition_size,
+                               int32_t grid_ctas, int32_t* n_parts, int32_t* n_big, int32_t* p_big,
+                               int32_t* p_small);
+
 /* ------------------------------------------------------------------------ */
 /* Decode attention                                                         */
 /* ------------------------------------------------------------------------ */

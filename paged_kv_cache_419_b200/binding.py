@@ -11,6 +11,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,6 +32,7 @@ EXPORTS = (
     "pkv_alloc_fork", "pkv_alloc_append", "pkv_alloc_append_batch", "pkv_alloc_free_seq",
     "pkv_alloc_beam_step", "pkv_alloc_block_table", "pkv_alloc_refcount", "pkv_alloc_stats",
     "pkv_alloc_add_seq_cached", "pkv_block_hash", "pkv_test_set_merge_wait", "pkv_paged_prefill",
+    "pkv_test_partitions",
 )
 
 
@@ -110,6 +112,7 @@ def lib() -> ctypes.CDLL:
             "pkv_alloc_refcount": ([P, i32, P], ctypes.c_int),
             "pkv_alloc_stats": ([P, ctypes.POINTER(AllocStats)], ctypes.c_int),
             "pkv_test_set_merge_wait": ([ctypes.c_uint64, ctypes.c_uint32], ctypes.c_int),
+            "pkv_test_partitions": ([P, i32, i32, i32, i32, i32, i32, P, P, P, P], ctypes.c_int),
             "pkv_last_cuda_error": ([], ctypes.c_int),
             "pkv_cuda_error_name": ([ctypes.c_int], ctypes.c_char_p),
             "pkv_paged_prefill": ([P, P, P, P, P, P, P, i32, i32, i32, i32, i32, f32, i32, i32, i32, i32,
@@ -282,6 +285,20 @@ def set_merge_wait_hook(limit_ns: int = 0, extra: int = 0):
     the partition merge wait for ``extra`` more publications than the decode grid
     makes and give up after ``limit_ns`` (0, 0 restores normal operation)."""
     _check(lib().pkv_test_set_merge_wait(int(limit_ns), int(extra)), "pkv_test_set_merge_wait")
+
+
+def partitions(context_lens, num_kv_heads: int, max_context_len: int, block_size: int,
+               partition_size: int, grid_ctas: int):
+    """Partition rule test hook (pkv_test_partitions, host only): per context,
+    (n_parts, n_big, p_big, p_small) as int32 arrays; the first n_big partitions
+    hold p_big tokens, the others p_small, the last one shorter."""
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S = int(lens.shape[0])
+    outs = [np.zeros(S, np.int32) for _ in range(4)]
+    _check(lib().pkv_test_partitions(lens.ctypes.data, S, int(num_kv_heads), int(max_context_len),
+                                     int(block_size), int(partition_size), int(grid_ctas),
+                                     *[o.ctypes.data for o in outs]), "pkv_test_partitions")
+    return tuple(outs)
 
 
 # ---------------------------------------------------------------- allocator

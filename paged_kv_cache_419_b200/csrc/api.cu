@@ -99,6 +99,22 @@ int workspace_partition(int32_t partition_size) {
 
 bool valid_partition(int p) { return p >= kStageTokens && p <= kMaxPartTokens && p % kStageTokens == 0; }
 
+// The partition arguments of a call (a.max_ctx set): the size, whether the
+// default size may become the balanced policy at launch, and the workspace's
+// partitions per context.  False for an unsupported partition_size.
+bool set_partition_args(DecodeArgs& a, int32_t partition_size) {
+  const int part = resolve_partition(partition_size);
+  if (!valid_partition(part)) return false;
+  const int ws_part = workspace_partition(partition_size);
+  a.part_tokens = part;
+  // default size: the launcher switches to the balanced policy when the batch
+  // has fewer (sequence, kv head) pairs than decode CTAs
+  a.balanced = partition_size == 0 ? 1 : 0;
+  a.max_parts = (a.max_ctx + ws_part - 1) / ws_part;
+  if (a.max_parts < 1) a.max_parts = 1;
+  return true;
+}
+
 int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
 
 // Workspace layout: [work counters | list of multi-partition sequences (S) |
@@ -188,16 +204,9 @@ pkv_status decode_common(DecodeArgs& a, int32_t head_dim, int32_t block_size, pk
                          int32_t partition_size, void* workspace, size_t ws_bytes, bool paged,
                          float scale, cudaStream_t stream) {
   if (a.num_seqs == 0) return PKV_OK;
-  const int part = resolve_partition(partition_size);
-  if (!valid_partition(part)) return PKV_EINVAL;
+  if (!set_partition_args(a, partition_size)) return PKV_EINVAL;
   const int ws_part = workspace_partition(partition_size);
   const int group = a.num_heads / a.num_kv_heads;
-  a.part_tokens = part;
-  // default size: the launcher switches to the balanced policy when the batch
-  // has fewer (sequence, kv head) pairs than decode CTAs
-  a.balanced = partition_size == 0 ? 1 : 0;
-  a.max_parts = (a.max_ctx + ws_part - 1) / ws_part;
-  if (a.max_parts < 1) a.max_parts = 1;
   const WorkspaceLayout lay = workspace_layout(a.num_seqs, a.num_heads, head_dim, a.max_ctx, ws_part);
   if (!workspace || ws_bytes < static_cast<size_t>(lay.total) || !aligned16(workspace))
     return PKV_EINVAL;
@@ -382,6 +391,42 @@ pkv_status pkv_device_error(unsigned int* flags_out, int clear, cudaStream_t str
 pkv_status pkv_test_set_merge_wait(uint64_t limit_ns, uint32_t extra) {
   g_merge_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
   g_merge_wait_extra.store(extra, std::memory_order_relaxed);
+  return PKV_OK;
+}
+
+pkv_status pkv_test_partitions(const int32_t* context_lens, int32_t num_seqs, int32_t num_kv_heads,
+                               int32_t max_context_len, int32_t block_size, int32_t partition_size,
+                               int32_t grid_ctas, int32_t* n_parts, int32_t* n_big, int32_t* p_big,
+                               int32_t* p_small) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || max_context_len < 0 || grid_ctas <= 0 ||
+      (block_size != 8 && block_size != 16 && block_size != 32))
+    return PKV_EINVAL;
+  if (num_seqs == 0) return PKV_OK;
+  if (!context_lens || !n_parts || !n_big || !p_big || !p_small) return PKV_EINVAL;
+  DecodeArgs a = {};
+  a.num_seqs = num_seqs;
+  a.num_kv_heads = num_kv_heads;
+  a.max_ctx = max_context_len;
+  if (!set_partition_args(a, partition_size)) return PKV_EINVAL;
+  apply_partition_policy(a, grid_ctas, block_size, true);
+  unsigned long long U = 0;  // the batch's token-heads, as the kernels sum them
+  for (int32_t s = 0; s < num_seqs; ++s) U += static_cast<unsigned long long>(clamp_len(context_lens[s], a.max_ctx));
+  U *= static_cast<unsigned long long>(num_kv_heads);
+  for (int32_t s = 0; s < num_seqs; ++s) {
+    const int L = clamp_len(context_lens[s], a.max_ctx);
+    int n = 0, nb = 0, pb = 0, ps = 0;
+    if (round_robin(a)) {
+      partition_rr(L, a, U, nb, n, pb, ps);
+    } else {
+      partition_for(L, a, U, n, pb);
+      nb = n;
+      ps = pb;
+    }
+    n_parts[s] = n;
+    n_big[s] = nb;
+    p_big[s] = pb;
+    p_small[s] = ps;
+  }
   return PKV_OK;
 }
 

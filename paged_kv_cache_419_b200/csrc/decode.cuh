@@ -115,7 +115,7 @@ constexpr int kRecordBytes = 32;
 // Partitioning of a context of L tokens (L already clamped to [0, max_ctx]):
 // n partitions of `size` tokens (a multiple of the 64-token stage), the last
 // one shorter.  part_tokens is a multiple of 64, so size <= part_tokens.
-__device__ __forceinline__ void partition_of(int L, int part_tokens, int& n, int& size) {
+__host__ __device__ __forceinline__ void partition_of(int L, int part_tokens, int& n, int& size) {
   if (L <= 0) {
     n = 1;
     size = 0;
@@ -140,15 +140,16 @@ __device__ __forceinline__ void partition_of(int L, int part_tokens, int& n, int
 // arithmetic only: the plan, the statically started CTAs and the merge agree.
 // k of the balanced rule: round(U / (grid x 2048)), raised to the fewest waves
 // whose items fit in max_part tokens, at least 1.
-__device__ __forceinline__ long long balanced_waves(long long uu, long long g, long long max_part) {
+__host__ __device__ __forceinline__ long long balanced_waves(long long uu, long long g, long long max_part) {
   long long k = (uu + g * 1024) / (g * 2048);
   const long long k_fit = (uu + g * max_part - 1) / (g * max_part);
   if (k < k_fit) k = k_fit;
   return k < 1 ? 1 : k;
 }
 
-__device__ __forceinline__ void partition_balanced(int L, unsigned long long U, int grid,
-                                                   int max_parts, int max_part, int& n, int& size) {
+__host__ __device__ __forceinline__ void partition_balanced(int L, unsigned long long U, int grid,
+                                                            int max_parts, int max_part, int& n,
+                                                            int& size) {
   if (L <= 0 || U == 0) {
     n = 1;
     size = L > 0 ? L : 0;
@@ -158,7 +159,8 @@ __device__ __forceinline__ void partition_balanced(int L, unsigned long long U, 
   const long long k = balanced_waves(uu, g, max_part);
   long long nn = static_cast<long long>(L) * k * g / uu;
   const long long lo = (L + max_part - 1) / max_part;
-  const long long hi = min(static_cast<long long>(max_parts), static_cast<long long>((L + 63) / 64));
+  const long long by_stage = (L + 63) / 64;
+  const long long hi = max_parts < by_stage ? max_parts : by_stage;
   nn = nn < lo ? lo : nn;
   nn = nn > hi ? hi : nn;
   if (nn < 1) nn = 1;
@@ -168,8 +170,8 @@ __device__ __forceinline__ void partition_balanced(int L, unsigned long long U, 
 
 // Partitions of a context of L tokens under this call's policy (U: the batch's
 // token-heads, used by the balanced policy only).
-__device__ __forceinline__ void partition_for(int L, const DecodeArgs& a, unsigned long long U,
-                                              int& n, int& size) {
+__host__ __device__ __forceinline__ void partition_for(int L, const DecodeArgs& a,
+                                                       unsigned long long U, int& n, int& size) {
   if (a.balanced)
     partition_balanced(L, U, a.grid_ctas, a.max_parts, a.part_tokens, n, size);
   else
@@ -193,8 +195,9 @@ __device__ __forceinline__ void partition_for(int L, const DecodeArgs& a, unsign
 // sequence and from U alone: the plan, the decode grid and the merge agree.
 constexpr int kBigNum = 14, kBigDen = 16, kSmallDiv = 4, kMinSmallTokens = 256;
 constexpr int kClaimLead = 3;
-__device__ __forceinline__ void partition_rr(int L, const DecodeArgs& a, unsigned long long U,
-                                             int& n_big, int& n, int& p_big, int& p_small) {
+__host__ __device__ __forceinline__ void partition_rr(int L, const DecodeArgs& a,
+                                                      unsigned long long U, int& n_big, int& n,
+                                                      int& p_big, int& p_small) {
   const long long g = a.grid_ctas, uu = static_cast<long long>(U);
   const long long k = uu > 0 ? balanced_waves(uu, g, a.part_tokens) : 1;
   long long pb = uu > 0 ? (uu * kBigNum + k * g * kBigDen - 1) / (k * g * kBigDen) : 0;
@@ -230,8 +233,21 @@ __device__ __forceinline__ void partition_rr(int L, const DecodeArgs& a, unsigne
 // kv head), kv head fastest, which it computes from the context lengths alone:
 // no CTA waits for the planning kernel's list.
 constexpr int kRoundRobinSeqs = 64;
-__device__ __forceinline__ bool round_robin(const DecodeArgs& a) {
+__host__ __device__ __forceinline__ bool round_robin(const DecodeArgs& a) {
   return a.balanced && a.num_seqs <= kRoundRobinSeqs;
+}
+
+// The call's partition policy once the decode grid is known (host, at launch):
+// the default size becomes the balanced policy when the batch has fewer
+// (sequence, kv head) pairs than CTAs (then every pair's partition 0 is a
+// static first item, and a partition may take a whole table buffer:
+// kMaxTableEntries blocks, part_tokens = its largest size).
+inline void apply_partition_policy(DecodeArgs& a, int grid, int block_size, bool paged) {
+  a.grid_ctas = grid;
+  if (a.balanced) {
+    a.balanced = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads < grid ? 1 : 0;
+    if (a.balanced) a.part_tokens = paged ? kMaxTableEntries * block_size : kMaxPartTokens;
+  }
 }
 
 // Sequences whose partition 0 runs as a static first item: decode CTA c
@@ -243,7 +259,7 @@ __device__ __forceinline__ int static_first_seqs(const int num_seqs, const int g
   return n < num_seqs ? n : num_seqs;
 }
 
-__device__ __forceinline__ int clamp_len(int L, int max_ctx) {
+__host__ __device__ __forceinline__ int clamp_len(int L, int max_ctx) {
   return L < 0 ? 0 : (L > max_ctx ? max_ctx : L);
 }
 

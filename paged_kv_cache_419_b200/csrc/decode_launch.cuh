@@ -77,15 +77,7 @@ cudaError_t launch_decode_one(const DecodeArgs& args, const DecodeMaps& maps, in
   cudaError_t e = decode_grid<T, D, G, B, PAGED>(num_sms, &grid);
   if (e != cudaSuccess) return e;
   DecodeArgs a = args;
-  a.grid_ctas = grid;
-  // The default partition size becomes the balanced policy when the batch has
-  // fewer (sequence, kv head) pairs than CTAs (then every pair's partition 0 is
-  // a static first item, and a partition may take a whole table buffer:
-  // kMaxTableEntries blocks, part_tokens = its largest size).
-  if (a.balanced) {
-    a.balanced = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads < grid ? 1 : 0;
-    if (a.balanced) a.part_tokens = PAGED ? kMaxTableEntries * B : kMaxPartTokens;
-  }
+  apply_partition_policy(a, grid, B, PAGED);
   // All three grids use programmatic dependent launch: each may become resident
   // while its predecessor runs.  The plan waits in-kernel for its predecessor
   // (whatever the caller queued before the call) to complete before it lets the
