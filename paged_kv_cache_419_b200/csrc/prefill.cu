@@ -555,9 +555,13 @@ __global__ void __maxnreg__(96)
     // Query tile t has 8 warps, two threads per query row (tensor-memory lane =
     // row): half hf holds keys 64 hf .. 64 hf + 63 of every key tile, and output
     // columns hf D/2 .. hf D/2 + D/2 - 1.  The two halves of a row combine their
-    // maxima (and, at the end, their sums) through shared memory at a named
-    // barrier of the tile's 256 threads; a failed wait anywhere in the tile is
-    // carried by that barrier, so all of the tile's threads stop together.
+    // maxima through shared memory at a named barrier of the two warps that hold
+    // the row's lanes (one per half), so a warp waits only for its partner, not
+    // for the slowest of the tile's 8 warps; at the end the sums meet at a
+    // barrier of the tile's 256 threads.  A failed wait is carried by these
+    // barriers; a warp pair that stops leaves the tensor-core thread without its
+    // weights, so every wait of the tile runs out and all of its threads reach
+    // the final barrier.
     const int t = (warp - 2) >> 3;                // query tile of this warp group
     const int hf = ((warp - 2) >> 2) & 1;         // half of the keys / output columns
     const int quarter = warp & 3;                 // tensor-memory lanes 32 quarter ..
@@ -572,6 +576,7 @@ __global__ void __maxnreg__(96)
     float* red = reinterpret_cast<float*>(smem + Tr::OFF_RED) + t * 2 * kPrefillTileM;
     float* red_l = reinterpret_cast<float*>(smem + Tr::OFF_RED) + (4 + t * 2) * kPrefillTileM;
     const int bar_id = 1 + t;
+    const int pair_bar = 3 + 4 * t + quarter;     // the two warps of these 32 rows
     // Running state of the row, in base-2 units: m is the max the weights are
     // taken against (at most kLazy below the true running max, see below) and
     // l this half's sum of the rounded weights.
@@ -615,9 +620,9 @@ __global__ void __maxnreg__(96)
         }
       }
       red[hf * kPrefillTileM + r] = part;
-      // Both halves of every row have read their scores after this barrier, so
+      // Both halves of these rows have read their scores after this barrier, so
       // the P writes below (over score columns) cannot race with a read.
-      if (named_barrier_or(bar_id, 2 * kPrefillTileM, !wok)) {
+      if (named_barrier_or(pair_bar, 64, !wok)) {
         ok = false;
         break;
       }
