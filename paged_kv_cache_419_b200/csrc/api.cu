@@ -410,7 +410,8 @@ pkv_status pkv_test_partitions(const int32_t* context_lens, int32_t num_seqs, in
   if (!set_partition_args(a, partition_size)) return PKV_EINVAL;
   apply_partition_policy(a, grid_ctas, block_size, true);
   unsigned long long U = 0;  // the batch's token-heads, as the kernels sum them
-  for (int32_t s = 0; s < num_seqs; ++s) U += static_cast<unsigned long long>(clamp_len(context_lens[s], a.max_ctx));
+  for (int32_t s = 0; s < num_seqs; ++s)
+    U += static_cast<unsigned long long>(clamp_len(context_lens[s], a.max_ctx));
   U *= static_cast<unsigned long long>(num_kv_heads);
   for (int32_t s = 0; s < num_seqs; ++s) {
     const int L = clamp_len(context_lens[s], a.max_ctx);
